@@ -1,0 +1,155 @@
+"""Double-precision CPU oracle for the ESA gated linear recurrence.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py`` may import this package.  The GPU
+library does not import it, link it or call it, and the two share no code.
+
+The arithmetic lives in ``esa_oracle.c`` (plain C, double precision,
+sequential per head and per time step).  This module compiles it with gcc
+when needed and exposes three numpy-level functions with the semantics of the
+three GPU entry points:
+
+* :func:`scan_fwd` -- the forward scan with the per-head RMS readout,
+* :func:`scan_bwd` -- the backward (reverse) scan,
+* :func:`step`     -- the one-token recurrent update.
+
+Sources for each formula are given in the C file's header: the recurrence and
+its two modes ("entangled-state-attention 0.1.0", section "Core idea"), the
+readout (same section), the state shape (mlbricks-web.pages.dev/esa,
+"Generation / memory"), and the chain-rule derivation of the backward pass.
+
+Parity pins: every function here is checked against closed forms, invariants,
+special cases, a high-precision brute-force evaluation and finite differences
+in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "esa_oracle.c")
+_LIB = os.path.join(_HERE, "libesa_oracle.so")
+
+DIRECT = 0
+CONTROLLED = 1
+EPS = 1e-6
+
+_lock = threading.Lock()
+_lib = None
+
+# Mutation testing only: load a deliberately altered build of the oracle from
+# this path instead of the real one (see tests/test_oracle_mutations.py).
+_LIB_OVERRIDE_ENV = "ESA_ORACLE_LIB_OVERRIDE"
+
+
+def build(force: bool = False) -> str:
+    """Compile ``esa_oracle.c`` into ``libesa_oracle.so`` with gcc (-O2, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+               "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            override = os.environ.get(_LIB_OVERRIDE_ENV)
+            if override:
+                lib = ctypes.CDLL(override)
+            else:
+                build()
+                lib = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            L = ctypes.c_long
+            I = ctypes.c_int
+            lib.esa_oracle_scan_fwd.argtypes = [P, P, P, P, P, L, L, L, L, I, P, P]
+            lib.esa_oracle_scan_fwd.restype = I
+            lib.esa_oracle_scan_bwd.argtypes = [P, P, P, P, P, P, P, P, P, L, L, L, L, I, P]
+            lib.esa_oracle_scan_bwd.restype = I
+            lib.esa_oracle_step.argtypes = [P, P, P, P, P, L, L, L, I]
+            lib.esa_oracle_step.restype = I
+            _lib = lib
+    return _lib
+
+
+def _f64(x, shape=None):
+    arr = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    if shape is not None and arr.shape != tuple(shape):
+        raise ValueError(f"expected shape {tuple(shape)}, got {arr.shape}")
+    return arr
+
+
+def _ptr(arr):
+    return None if arr is None else arr.ctypes.data_as(ctypes.c_void_p)
+
+
+def scan_fwd(a, v, q, mode, E_init=None, return_states=False):
+    """Forward scan of [B, T, H, D] inputs.
+
+    Returns ``(y, E_final)`` or, with ``return_states``, ``(y, E_final, E_all)``
+    where ``E_all[b, t]`` is the state after token t.
+    """
+    a = _f64(a)
+    if a.ndim != 4:
+        raise ValueError("a must be [B, T, H, D]")
+    B, T, H, D = a.shape
+    v = _f64(v, a.shape)
+    q = _f64(q, a.shape)
+    E0 = None if E_init is None else _f64(E_init, (B, H, D))
+    y = np.empty_like(a)
+    E_final = np.empty((B, H, D), dtype=np.float64)
+    E_all = np.empty_like(a) if return_states else None
+    rc = _load().esa_oracle_scan_fwd(_ptr(a), _ptr(v), _ptr(q), _ptr(y), _ptr(E_final),
+                                     B, T, H, D, int(mode), _ptr(E0), _ptr(E_all))
+    if rc != 0:
+        raise ValueError(f"esa_oracle_scan_fwd failed with {rc}")
+    return (y, E_final, E_all) if return_states else (y, E_final)
+
+
+def scan_bwd(a, v, q, dy, mode, E_init=None, dE_final=None):
+    """Backward scan.  Returns ``(da, dv, dq, dE_init)``."""
+    a = _f64(a)
+    if a.ndim != 4:
+        raise ValueError("a must be [B, T, H, D]")
+    B, T, H, D = a.shape
+    v = _f64(v, a.shape)
+    q = _f64(q, a.shape)
+    dy = _f64(dy, a.shape)
+    E0 = None if E_init is None else _f64(E_init, (B, H, D))
+    dEf = None if dE_final is None else _f64(dE_final, (B, H, D))
+    da = np.empty_like(a)
+    dv = np.empty_like(a)
+    dq = np.empty_like(a)
+    dE_init = np.empty((B, H, D), dtype=np.float64)
+    rc = _load().esa_oracle_scan_bwd(_ptr(a), _ptr(v), _ptr(q), _ptr(dy), _ptr(dEf),
+                                     _ptr(da), _ptr(dv), _ptr(dq), _ptr(dE_init),
+                                     B, T, H, D, int(mode), _ptr(E0))
+    if rc != 0:
+        raise ValueError(f"esa_oracle_scan_bwd failed with {rc}")
+    return da, dv, dq, dE_init
+
+
+def step(a_t, v_t, q_t, E, mode):
+    """One-token update of [B, H, D] inputs.  Returns ``(y_t, E_new)``; E is not modified."""
+    a_t = _f64(a_t)
+    if a_t.ndim != 3:
+        raise ValueError("a_t must be [B, H, D]")
+    B, H, D = a_t.shape
+    v_t = _f64(v_t, a_t.shape)
+    q_t = _f64(q_t, a_t.shape)
+    E_new = np.array(_f64(E, a_t.shape), copy=True)
+    y_t = np.empty_like(a_t)
+    rc = _load().esa_oracle_step(_ptr(a_t), _ptr(v_t), _ptr(q_t), _ptr(E_new), _ptr(y_t),
+                                 B, H, D, int(mode))
+    if rc != 0:
+        raise ValueError(f"esa_oracle_step failed with {rc}")
+    return y_t, E_new
