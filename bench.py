@@ -1,0 +1,387 @@
+#!/usr/bin/env python
+"""Benchmark of the ESA scan hot path: forward + backward tokens/s.
+
+Workload (one step): controlled mode, fp16 I/O, fp32 state, B=64, T=65536,
+H=4, D=32 (C=128), gate logits ~ N(4, 1), v, q, dy ~ N(0, 1); one
+esa_scan_fwd followed by one esa_scan_bwd over the whole batch.  The inputs
+(4.3 GB per step) are larger than the 126 MB L2, so no flush is needed
+between steps.
+
+Prints ONE JSON line (rank 0):
+  value  -- tokens/s over all ranks, device-timed with CUDA events, inputs
+            resident in HBM; max over ranks.
+  e2e    -- the same metric through the public binding with pinned HOST
+            buffers: every step copies a, v, q, dy host->device and y, da,
+            dv, dq, E_final, dE_init device->host inside the timed region.
+  roofline -- the dominant kernel's algorithmic bytes per launch / its mean
+            CUDA-event duration, against the measured HBM copy peak.
+  cpu_baseline -- the fp64 oracle on a bounded sample, one host core.
+
+Multi-GPU (torchrun): every rank runs its own independent batch (the
+sequences are independent, so there is no data-path collective): weak
+scaling.  `--impl reference` times the oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "scan fwd+bwd tokens/s at B64 T64K C128; achieved HBM GB/s as % of peak"
+WORKLOAD_NAME = "controlled_f16_B64_T65536_H4_D32"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description="ESA scan fwd+bwd benchmark")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+def workload():
+    from gated_linear_recurrence_b200 import inputs
+    return inputs.WORKLOADS[WORKLOAD_NAME]
+
+
+def config_dict(w):
+    return {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "D": w.D, "C": w.C,
+            "mode": "controlled" if w.mode == 1 else "direct", "io_dtype": w.dtype, "state_dtype": "f32",
+            "gate_logit_mean": w.a_mean, "step": "esa_scan_fwd + esa_scan_bwd",
+            "l2": "inputs larger than L2 (4.3 GB read per step vs 126 MB L2); no flush"}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, torch copy)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "gated_linear_recurrence_b200", "csrc", "*"))):
+        if p.endswith((".cu", ".cuh", ".h")):
+            with open(p, "rb") as f:
+                h.update(os.path.basename(p).encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current sources."""
+    for p in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        text = open(p).read()
+        m_k = re.search(r"^kernel:\s*(\S+)", text, re.M)
+        m_h = re.search(r"^source_hash:\s*(\S+)", text, re.M)
+        m_t = re.search(r"^dram_bytes_per_full_launch:\s*([0-9.eE+]+)", text, re.M)
+        if m_k and m_h and m_t and m_k.group(1) == kernel and m_h.group(1) == source_hash():
+            return float(m_t.group(1))
+    return None
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index, period_s=0.01):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = self._handle(device_index)
+            self.max_mhz = int(pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self._h = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _handle(self, idx):
+        import torch
+        nv = self._nv
+        try:
+            uuid = str(torch.cuda.get_device_properties(idx).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            if vis:
+                idx = int(vis.split(",")[idx])
+            return nv.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        nv = self._nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(int(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)))
+                bits = int(get_reasons(self._h))
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def start(self):
+        if self._h is not None:
+            self._t.start()
+        return self
+
+    def stop(self):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples), "source": "NVML, polled every 10 ms during the timed region"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs (the oracle is test infrastructure; only these legs use it).
+# ---------------------------------------------------------------------------
+
+def oracle_sample_tokens_per_s(w, rows, T, seed):
+    """Time the fp64 oracle (fwd + bwd) on `rows` batch rows x T tokens."""
+    import torch
+
+    import oracle
+    from gated_linear_recurrence_b200 import inputs
+    x = inputs.make_scan_inputs(rows, T, w.H, w.D, w.dtype, w.a_mean, seed)
+    f64 = {k: x[k].to(torch.float64).numpy() for k in ("a", "v", "q", "dy")}
+    t0 = time.perf_counter()
+    oracle.scan_fwd(f64["a"], f64["v"], f64["q"], w.mode)
+    oracle.scan_bwd(f64["a"], f64["v"], f64["q"], f64["dy"], w.mode)
+    dt = time.perf_counter() - t0
+    return rows * T / dt, dt
+
+
+def run_reference(args):
+    """Reference arm: the oracle, as it stands, on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = workload()
+    rows, T = 1, 8192
+    for i in range(args.warmup):
+        oracle_sample_tokens_per_s(w, rows, T, seed=1000 + i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_sample_tokens_per_s(w, rows, T, seed=2000 + i)
+    dt = time.perf_counter() - t0
+    value = args.steps * rows * T / dt
+    sample = (f"each step: fwd+bwd of {rows} batch row x {T} tokens x C={w.C} (controlled, fp16-rounded "
+              f"inputs in fp64) through the sequential C oracle on one host core")
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(w), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# Our arm.
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from gated_linear_recurrence_b200 import esa, inputs
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    w = workload()
+    B, T, H, D, mode = w.B, w.T, w.H, w.D, w.mode
+    x = inputs.make_scan_inputs(B, T, H, D, w.dtype, w.a_mean, w.seed + 17 * rank, device=dev)
+    a, v, q, dy = x["a"], x["v"], x["q"], x["dy"]
+    y = torch.empty_like(a)
+    da, dv, dq = torch.empty_like(a), torch.empty_like(a), torch.empty_like(a)
+    Ef = torch.empty(B, H, D, dtype=torch.float32, device=dev)
+    dE0 = torch.empty_like(Ef)
+    ws = esa.new_workspace(B, T, H, D, a.dtype, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        esa.esa_scan_fwd(a, v, q, y=y, E_final=Ef, mode=mode, workspace=ws)
+        esa.esa_scan_bwd(a, v, q, dy, ws, mode=mode, da=da, dv=dv, dq=dq, dE_init=dE0)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    esa.esa_check(ws)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local).start()
+    barrier()
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for k in range(K):
+        ev[k][0].record(stream)
+        esa.esa_scan_fwd(a, v, q, y=y, E_final=Ef, mode=mode, workspace=ws)
+        ev[k][1].record(stream)
+        esa.esa_scan_bwd(a, v, q, dy, ws, mode=mode, da=da, dv=dv, dq=dq, dE_init=dE0)
+        ev[k][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    esa.esa_check(ws)
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    value = world * B * T * K / (elapsed_ms / 1e3)
+
+    s = a.element_size()
+    C = H * D
+    tokens = B * T
+    fwd_bytes = 4 * s * C * tokens
+    bwd_bytes = 7 * s * C * tokens
+    peak, peak_src = measured_peak()
+    if bwd_ms >= fwd_ms:
+        dom, dom_ms, dom_bytes = "esa_scan_bwd_kernel", bwd_ms, bwd_bytes
+    else:
+        dom, dom_ms, dom_bytes = "esa_scan_fwd_kernel", fwd_ms, fwd_bytes
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+    step_gbs = (fwd_bytes + bwd_bytes) * K / (elapsed_ms / 1e3) / 1e9
+
+    # ---- end to end through the binding, with pinned host buffers ----------
+    e2e = None
+    if not args.no_e2e:
+        K2 = max(1, args.e2e_steps)
+        h_in = {k: torch.empty(a.shape, dtype=a.dtype, pin_memory=True) for k in ("a", "v", "q", "dy")}
+        for k, t in (("a", a), ("v", v), ("q", q), ("dy", dy)):
+            h_in[k].copy_(t)
+        h_out = {k: torch.empty(a.shape, dtype=a.dtype, pin_memory=True) for k in ("y", "da", "dv", "dq")}
+        h_st = {k: torch.empty(B, H, D, dtype=torch.float32, pin_memory=True) for k in ("Ef", "dE0")}
+        d_in = {k: torch.empty_like(a) for k in ("a", "v", "q", "dy")}
+
+        def e2e_step():
+            for k in ("a", "v", "q", "dy"):
+                d_in[k].copy_(h_in[k], non_blocking=True)
+            yy, EE, _ = esa.esa_scan_fwd(d_in["a"], d_in["v"], d_in["q"], y=y, E_final=Ef, mode=mode,
+                                         workspace=ws)
+            g = esa.esa_scan_bwd(d_in["a"], d_in["v"], d_in["q"], d_in["dy"], ws, mode=mode, da=da, dv=dv,
+                                 dq=dq, dE_init=dE0)
+            for k, t in (("y", yy), ("da", g[0]), ("dv", g[1]), ("dq", g[2])):
+                h_out[k].copy_(t, non_blocking=True)
+            h_st["Ef"].copy_(EE, non_blocking=True)
+            h_st["dE0"].copy_(g[3], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(K2):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        esa.esa_check(ws)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+        h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+        d2h = sum(t.numel() * t.element_size() for t in h_out.values()) + \
+            sum(t.numel() * t.element_size() for t in h_st.values())
+        e2e = {"value": world * tokens * K2 / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": K2,
+               "path": "pinned host -> esa_scan_fwd -> esa_scan_bwd -> pinned host, one stream, device-timed"}
+        del h_in, h_out, h_st, d_in
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = 2
+        tps, secs = oracle_sample_tokens_per_s(w, rows, T, seed=4242)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"fwd+bwd of {rows} batch rows x {T} tokens x C={C} (controlled, fp16-rounded inputs "
+                         f"in fp64) through the sequential C oracle on one host core: {secs:.1f} s"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_dict(w),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(dom), "kernel": dom,
+                     "algorithmic_bytes_per_launch": dom_bytes, "launch_ms": dom_ms, "peak_source": peak_src,
+                     "frac_of_nominal_8TBs": achieved / NOMINAL_HBM_GBS},
+        "detail": {"fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "fwd_GBs": fwd_bytes / (fwd_ms / 1e3) / 1e9,
+                   "bwd_GBs": bwd_bytes / (bwd_ms / 1e3) / 1e9, "step_GBs": step_gbs,
+                   "step_frac_of_measured_peak": step_gbs / peak, "step_frac_of_nominal_8TBs":
+                   step_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes_per_step": fwd_bytes + bwd_bytes},
+        "clocks": clk,
+        "e2e": e2e,
+        "gpu_launches": 2 * K,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,27 @@
+"""B200-native (sm_100a) library for the ESA gated linear recurrence scan.
+
+The hot path -- forward scan with fused gate sigmoid and per-head RMS
+readout, its backward scan, and the one-token decode update -- is
+hand-written CUDA behind a C ABI (``include/esa.h``); this package is the thin
+ctypes binding over it plus the build script and seeded input generators.
+"""
+from .esa import (  # noqa: F401
+    CONTROLLED,
+    DIRECT,
+    EsaError,
+    LIB_PATH,
+    esa_check,
+    esa_scan_bwd,
+    esa_scan_fwd,
+    esa_step,
+    esa_strerror,
+    esa_version,
+    esa_workspace_size,
+    load_library,
+    new_workspace,
+)
+
+__all__ = [
+    "CONTROLLED", "DIRECT", "EsaError", "LIB_PATH", "esa_check", "esa_scan_bwd", "esa_scan_fwd",
+    "esa_step", "esa_strerror", "esa_version", "esa_workspace_size", "load_library", "new_workspace",
+]

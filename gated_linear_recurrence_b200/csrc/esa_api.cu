@@ -1,0 +1,314 @@
+// esa_api.cu -- the C ABI of the ESA scan library (declared in include/esa.h).
+//
+// Host responsibilities: argument and alignment checks (before anything is
+// enqueued), the workspace layout, TMA tensor-map encoding, the per-call
+// reset of the look-back flags, and kernel dispatch on the caller's stream.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "esa.h"
+#include "esa_launch.h"
+
+namespace {
+
+using esa::tile_cols;
+using esa::tile_rows;
+
+constexpr int kVersion = 100;   // 0.1.0
+
+bool supported_d(int D) {
+  return D == 8 || D == 16 || D == 32 || D == 64 || D == 128 || D == 256;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t elem_bytes(int dtype) { return dtype == ESA_F32 ? 4 : 2; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Workspace layout (byte offsets from the workspace base):
+//   [0, 4)            device status word (sticky until esa_check)
+//   [16, 32)          forward header: [1] tile ticket, [2] abort flag
+//   [32, 32+4n)       forward per-tile flags
+//   bwd               backward header (16 B) + per-tile flags
+//   agg               n * CT float2   per-tile affine carry maps
+//   fstate            n * CT float    forward state at each chunk end
+//   bstate            n * CT float    backward carry at each chunk start
+// with n = B * ceil(C / CT) * ceil(T / L) tiles.
+struct Layout {
+  int L = 0, CT = 0, nct = 0, nchunks = 0, nchains = 0;
+  long long ntiles = 0;
+  size_t fwd_bytes = 0;   // bytes cleared before each forward (status + header + flags)
+  size_t bwd_off = 0, bwd_bytes = 0;
+  size_t agg_off = 0, fstate_off = 0, bstate_off = 0, total = 0;
+};
+
+bool make_layout(int B, int T, int H, int D, int dtype, Layout *lo) {
+  if (B < 0 || T < 0 || H < 1 || D < 1) return false;
+  if (dtype < ESA_F32 || dtype > ESA_BF16) return false;
+  if (!supported_d(D)) return false;
+  const long long C = static_cast<long long>(H) * D;
+  if (C > INT_MAX / 2) return false;
+  lo->L = tile_rows(dtype);
+  lo->CT = tile_cols(D);
+  lo->nct = static_cast<int>((C + lo->CT - 1) / lo->CT);
+  lo->nchunks = (T + lo->L - 1) / lo->L;
+  const long long nchains = static_cast<long long>(B) * lo->nct;
+  if (nchains > INT_MAX) return false;
+  lo->nchains = static_cast<int>(nchains);
+  lo->ntiles = nchains * lo->nchunks;
+  if (lo->ntiles > INT_MAX) return false;
+  const size_t n = static_cast<size_t>(lo->ntiles);
+  lo->fwd_bytes = 32 + 4 * n;
+  size_t off = align_up(lo->fwd_bytes, 256);
+  lo->bwd_off = off;
+  lo->bwd_bytes = 16 + 4 * n;
+  off = align_up(off + lo->bwd_bytes, 256);
+  lo->agg_off = off;
+  off = align_up(off + n * lo->CT * sizeof(float2), 256);
+  lo->fstate_off = off;
+  off = align_up(off + n * lo->CT * sizeof(float), 256);
+  lo->bstate_off = off;
+  off = align_up(off + n * lo->CT * sizeof(float), 256);
+  lo->total = off;
+  return true;
+}
+
+esa::Workspace workspace_view(void *base, const Layout &lo) {
+  unsigned char *p = static_cast<unsigned char *>(base);
+  esa::Workspace ws;
+  ws.status = reinterpret_cast<unsigned *>(p);
+  ws.fwd_hdr = reinterpret_cast<unsigned *>(p + 16);
+  ws.fwd_flags = reinterpret_cast<unsigned *>(p + 32);
+  ws.bwd_hdr = reinterpret_cast<unsigned *>(p + lo.bwd_off);
+  ws.bwd_flags = reinterpret_cast<unsigned *>(p + lo.bwd_off + 16);
+  ws.agg = reinterpret_cast<float2 *>(p + lo.agg_off);
+  ws.fstate = reinterpret_cast<float *>(p + lo.fstate_off);
+  ws.bstate = reinterpret_cast<float *>(p + lo.bstate_off);
+  return ws;
+}
+
+// The current device must be compute capability 10.0 (B200, sm_100a code).
+int check_device() {
+  static std::atomic<int> cache[64];   // 0 unknown, 1 ok, 2 unsupported
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    cudaGetLastError();
+    return ESA_ERR_DEVICE;
+  }
+  if (dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c == 1) return ESA_OK;
+    if (c == 2) return ESA_ERR_DEVICE;
+  }
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return ESA_ERR_DEVICE;
+  }
+  const bool ok = (major == 10 && minor == 0);
+  if (dev < 64) cache[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
+  return ok ? ESA_OK : ESA_ERR_DEVICE;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// [B][T][C] tensor in the I/O dtype, read in boxes of [L rows][CT channels].
+int make_tmap(CUtensorMap *map, const void *ptr, int dtype, int B, int T, int C, const Layout &lo) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return ESA_ERR_LAUNCH;
+  const CUtensorMapDataType dt = dtype == ESA_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : dtype == ESA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const cuuint64_t s = elem_bytes(dtype);
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(T),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(C) * s,
+                                 static_cast<cuuint64_t>(T) * static_cast<cuuint64_t>(C) * s};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(lo.CT), static_cast<cuuint32_t>(lo.L), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  std::memset(map, 0, sizeof(*map));
+  const CUresult r = fn(map, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ESA_OK : ESA_ERR_LAUNCH;
+}
+
+int check_shape(int B, int T, int H, int D, int mode, int dtype) {
+  if (B < 0 || T < 0 || H < 1 || D < 1) return ESA_ERR_ARG;
+  if (mode != ESA_DIRECT && mode != ESA_CONTROLLED) return ESA_ERR_ARG;
+  if (dtype < ESA_F32 || dtype > ESA_BF16) return ESA_ERR_ARG;
+  if (!supported_d(D)) return ESA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(H) * D > INT_MAX / 2) return ESA_ERR_ARG;
+  return ESA_OK;
+}
+
+esa::ScanShape scan_shape(int B, int T, int H, int D, const Layout &lo) {
+  esa::ScanShape s;
+  s.B = B;
+  s.T = T;
+  s.C = H * D;
+  s.nchunks = lo.nchunks;
+  s.nct = lo.nct;
+  s.nchains = lo.nchains;
+  s.inv_D = 1.0f / static_cast<float>(D);
+  return s;
+}
+
+int rt(cudaError_t e) {
+  if (e == cudaSuccess) return ESA_OK;
+  cudaGetLastError();
+  return ESA_ERR_LAUNCH;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t esa_workspace_size(int B, int T, int H, int D, int dtype) {
+  Layout lo;
+  if (!make_layout(B, T, H, D, dtype, &lo)) return 0;
+  return lo.total;
+}
+
+int esa_scan_fwd(const void *a, const void *v, const void *q, void *y, float *E_final, int B, int T,
+                 int H, int D, int mode, const float *E_init, int dtype, void *workspace,
+                 size_t workspace_bytes, void *stream) {
+  int rc = check_shape(B, T, H, D, mode, dtype);
+  if (rc) return rc;
+  if (!a || !v || !q || !y) return ESA_ERR_ARG;
+  for (const void *p : {a, v, q, static_cast<const void *>(y), static_cast<const void *>(E_final),
+                        static_cast<const void *>(E_init), static_cast<const void *>(workspace)})
+    if (p && !aligned16(p)) return ESA_ERR_ALIGN;
+  Layout lo;
+  if (!make_layout(B, T, H, D, dtype, &lo)) return ESA_ERR_ARG;
+  if (!workspace || workspace_bytes < lo.total) return ESA_ERR_WORKSPACE;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int C = H * D;
+  if (B == 0) return ESA_OK;
+  if (T == 0) {   // no tokens: the final state is the initial one
+    if (!E_final) return ESA_OK;
+    const size_t bytes = static_cast<size_t>(B) * C * sizeof(float);
+    return E_init ? rt(cudaMemcpyAsync(E_final, E_init, bytes, cudaMemcpyDeviceToDevice, st))
+                  : rt(cudaMemsetAsync(E_final, 0, bytes, st));
+  }
+  CUtensorMap ta, tv, tq;
+  if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo))) return rc;
+  if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo))) return rc;
+  if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo))) return rc;
+  if ((rc = rt(cudaMemsetAsync(workspace, 0, lo.fwd_bytes, st)))) return rc;
+  esa::FwdArgs args;
+  args.s = scan_shape(B, T, H, D, lo);
+  args.y = y;
+  args.E_final = E_final;
+  args.E_init = E_init;
+  args.ws = workspace_view(workspace, lo);
+  return esa::launch_fwd(dtype, mode, D, ta, tv, tq, args, static_cast<int>(lo.ntiles), st);
+}
+
+int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy, const float *dE_final,
+                 void *da, void *dv, void *dq, float *dE_init, int B, int T, int H, int D, int mode,
+                 const float *E_init, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+  int rc = check_shape(B, T, H, D, mode, dtype);
+  if (rc) return rc;
+  if (!a || !v || !q || !dy || !da || !dv || !dq) return ESA_ERR_ARG;
+  for (const void *p : {a, v, q, dy, static_cast<const void *>(dE_final), static_cast<const void *>(da),
+                        static_cast<const void *>(dv), static_cast<const void *>(dq),
+                        static_cast<const void *>(dE_init), static_cast<const void *>(E_init),
+                        static_cast<const void *>(workspace)})
+    if (p && !aligned16(p)) return ESA_ERR_ALIGN;
+  Layout lo;
+  if (!make_layout(B, T, H, D, dtype, &lo)) return ESA_ERR_ARG;
+  if (!workspace || workspace_bytes < lo.total) return ESA_ERR_WORKSPACE;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int C = H * D;
+  if (B == 0) return ESA_OK;
+  if (T == 0) {   // no tokens: the gradient passes straight through
+    if (!dE_init) return ESA_OK;
+    const size_t bytes = static_cast<size_t>(B) * C * sizeof(float);
+    return dE_final ? rt(cudaMemcpyAsync(dE_init, dE_final, bytes, cudaMemcpyDeviceToDevice, st))
+                    : rt(cudaMemsetAsync(dE_init, 0, bytes, st));
+  }
+  CUtensorMap ta, tv, tq, tdy;
+  if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo))) return rc;
+  if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo))) return rc;
+  if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo))) return rc;
+  if ((rc = make_tmap(&tdy, dy, dtype, B, T, C, lo))) return rc;
+  unsigned char *base = static_cast<unsigned char *>(workspace);
+  if ((rc = rt(cudaMemsetAsync(base + lo.bwd_off, 0, lo.bwd_bytes, st)))) return rc;
+  esa::BwdArgs args;
+  args.s = scan_shape(B, T, H, D, lo);
+  args.da = da;
+  args.dv = dv;
+  args.dq = dq;
+  args.dE_final = dE_final;
+  args.dE_init = dE_init;
+  args.E_init = E_init;
+  args.ws = workspace_view(workspace, lo);
+  return esa::launch_bwd(dtype, mode, D, ta, tv, tq, tdy, args, static_cast<int>(lo.ntiles), st);
+}
+
+int esa_step(const void *a_t, const void *v_t, const void *q_t, float *E, void *y_t, int B, int H, int D,
+             int mode, int dtype, void *stream) {
+  int rc = check_shape(B, 1, H, D, mode, dtype);
+  if (rc) return rc;
+  if (!a_t || !v_t || !q_t || !E || !y_t) return ESA_ERR_ARG;
+  for (const void *p : {a_t, v_t, q_t, static_cast<const void *>(E), static_cast<const void *>(y_t)})
+    if (!aligned16(p)) return ESA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  if (B == 0) return ESA_OK;
+  const long nvec = static_cast<long>(B) * H * D / 8;
+  return esa::launch_step(dtype, mode, D, a_t, v_t, q_t, E, y_t, nvec, 1.0f / static_cast<float>(D),
+                          static_cast<cudaStream_t>(stream));
+}
+
+int esa_check(void *workspace, void *stream) {
+  if (!workspace) return ESA_ERR_ARG;
+  if (!aligned16(workspace)) return ESA_ERR_ALIGN;
+  int rc = check_device();
+  if (rc) return rc;
+  if ((rc = rt(cudaStreamSynchronize(static_cast<cudaStream_t>(stream))))) return rc;
+  unsigned status = 0;
+  if ((rc = rt(cudaMemcpy(&status, workspace, sizeof(status), cudaMemcpyDeviceToHost)))) return rc;
+  if (status == 0) return ESA_OK;
+  if ((rc = rt(cudaMemset(workspace, 0, sizeof(status))))) return rc;
+  return ESA_ERR_TIMEOUT;
+}
+
+const char *esa_strerror(int status) {
+  switch (status) {
+    case ESA_OK: return "ok";
+    case ESA_ERR_ARG: return "invalid argument (size, mode, dtype or a required NULL pointer)";
+    case ESA_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case ESA_ERR_UNSUPPORTED: return "head dimension D must be one of 8, 16, 32, 64, 128, 256";
+    case ESA_ERR_WORKSPACE: return "workspace missing or smaller than esa_workspace_size()";
+    case ESA_ERR_LAUNCH: return "the CUDA runtime rejected a launch, copy or tensor map";
+    case ESA_ERR_TIMEOUT: return "a bounded device-side wait gave up; outputs of the call are invalid";
+    case ESA_ERR_DEVICE: return "no CUDA device, or the current device is not sm_100 (B200)";
+    default: return "unknown esa status";
+  }
+}
+
+int esa_version(void) { return kVersion; }
+
+}  // extern "C"

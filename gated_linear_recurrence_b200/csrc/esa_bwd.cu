@@ -1,0 +1,33 @@
+// esa_bwd.cu -- instantiations and launcher of the backward scan kernel.
+#include "esa_dispatch.cuh"
+
+namespace esa {
+
+namespace {
+struct BwdLauncher {
+  const CUtensorMap &ta, &tv, &tq, &tdy;
+  const BwdArgs &args;
+  int ntiles;
+  cudaStream_t stream;
+
+  template <typename T, int MODE, int LPH, int VPR, int L, int K>
+  int operator()() const {
+    using Cfg = TileCfg<T, LPH, VPR, L, K>;
+    const size_t smem = scan_smem_bytes<Cfg, 4>();
+    auto kern = esa_scan_bwd_kernel<T, MODE, LPH, VPR, L, K>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return launch_status(e);
+    kern<<<ntiles, Cfg::NT, smem, stream>>>(ta, tv, tq, tdy, args);
+    return launch_status(cudaGetLastError());
+  }
+};
+}  // namespace
+
+int launch_bwd(int dtype, int mode, int D, const CUtensorMap &ta, const CUtensorMap &tv,
+               const CUtensorMap &tq, const CUtensorMap &tdy, const BwdArgs &args, int ntiles,
+               cudaStream_t stream) {
+  return dispatch(dtype, mode, D, BwdLauncher{ta, tv, tq, tdy, args, ntiles, stream});
+}
+
+}  // namespace esa

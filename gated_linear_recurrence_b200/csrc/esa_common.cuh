@@ -1,0 +1,234 @@
+// esa_common.cuh -- device helpers shared by the ESA scan kernels (sm_100a).
+//
+// Contents: I/O vector loads/stores of 8 channels, the gate sigmoid, the
+// per-tile workspace view, and thin inline-PTX wrappers for mbarriers, TMA
+// tensor loads and acquire/release flag accesses.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace esa {
+
+constexpr float kEps = 1e-6f;          // RMS-norm epsilon (inside the square root)
+constexpr unsigned kFlagAgg = 1u;      // chunk aggregate published
+constexpr unsigned kFlagIncl = 2u;     // chunk's inclusive carry published
+constexpr unsigned kStatusTimeout = 1u;
+// Iteration cap of every device-side wait.  With the back-off below this is
+// at most a second or two, far above any legitimate wait (microseconds).
+constexpr unsigned kSpinLimit = 1u << 21;
+
+// ---------------------------------------------------------------------------
+// Workspace view.  Every time chunk of every sequence owns one "slot":
+//   slot = chain * nchunks + chunk,  chain = b * nct + ct
+// where ct indexes channel tiles of CT channels.  Per slot and channel:
+//   agg   (P, S): the chunk's affine carry map  x -> P x + S
+//   fstate       : forward state at the chunk's end (checkpoint for backward)
+//   bstate       : backward carry leaving the chunk towards earlier time
+// ---------------------------------------------------------------------------
+struct Workspace {
+  unsigned *fwd_hdr;    // [1] tile ticket counter, [2] abort flag
+  unsigned *fwd_flags;
+  unsigned *bwd_hdr;
+  unsigned *bwd_flags;
+  unsigned *status;     // sticky device status (0 = ok)
+  float2 *agg;
+  float *fstate;
+  float *bstate;
+};
+
+// ---------------------------------------------------------------------------
+// I/O element traits: 8 consecutive channels per thread.
+// ---------------------------------------------------------------------------
+template <typename T> struct Io;
+
+template <> struct Io<float> {
+  static constexpr int kBytes = 4;
+  static __device__ __forceinline__ void load8(const float *p, float (&x)[8]) {
+    const float4 u = reinterpret_cast<const float4 *>(p)[0];
+    const float4 w = reinterpret_cast<const float4 *>(p)[1];
+    x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+    x[4] = w.x; x[5] = w.y; x[6] = w.z; x[7] = w.w;
+  }
+  static __device__ __forceinline__ void store8(float *p, const float (&x)[8]) {
+    reinterpret_cast<float4 *>(p)[0] = make_float4(x[0], x[1], x[2], x[3]);
+    reinterpret_cast<float4 *>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
+  }
+};
+
+template <> struct Io<__half> {
+  static constexpr int kBytes = 2;
+  static __device__ __forceinline__ void load8(const __half *p, float (&x)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(h[i]);
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  }
+  static __device__ __forceinline__ void store8(__half *p, const float (&x)[8]) {
+    uint4 u;
+    __half2 *h = reinterpret_cast<__half2 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(x[2 * i], x[2 * i + 1]);
+    *reinterpret_cast<uint4 *>(p) = u;
+  }
+};
+
+template <> struct Io<__nv_bfloat16> {
+  static constexpr int kBytes = 2;
+  static __device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&x)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  }
+  static __device__ __forceinline__ void store8(__nv_bfloat16 *p, const float (&x)[8]) {
+    uint4 u;
+    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    *reinterpret_cast<uint4 *>(p) = u;
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Gate.  u = exp(-x) with x clamped at -80 so u stays finite; then
+//   A = 1 / (1 + u)      (sigmoid)
+//   1 - A = u * A        (no cancellation when A is close to 1)
+// CUDA's fast exp and divide intrinsics are used as-is.
+// ---------------------------------------------------------------------------
+struct Gate {
+  float A;    // sigmoid(x)
+  float Ac;   // 1 - sigmoid(x)
+};
+
+__device__ __forceinline__ Gate gate_of(float x) {
+  const float u = __expf(-fmaxf(x, -80.0f));
+  const float A = __fdividef(1.0f, 1.0f + u);
+  return Gate{A, u * A};
+}
+
+// Sum over the `LPH` adjacent lanes that hold one head (LPH a power of two).
+template <int LPH>
+__device__ __forceinline__ float head_sum(float s) {
+#pragma unroll
+  for (int o = 1; o < LPH; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
+
+// ---------------------------------------------------------------------------
+// Inline PTX: shared-memory addresses, mbarriers, TMA tensor loads, flags.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+// Non-blocking test of an mbarrier phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, unsigned phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
+
+// 3-D tiled TMA load (no multicast): box at coordinates (x, y, z) of the
+// tensor map into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ unsigned ld_relaxed(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Named barrier over the first `nthreads` threads of the CTA (id 1; id 0 is __syncthreads).
+__device__ __forceinline__ void bar_sync_first(unsigned nthreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+// Wait for the TMA transaction on `bar` (phase 0).  Bounded: on giving up it
+// records a timeout in the status word and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned phase, unsigned *status) {
+  for (unsigned it = 0; it < kSpinLimit; ++it) {
+    if (mbar_test_wait(bar, phase)) return true;
+    if (it > 16) __nanosleep(64);
+  }
+  atomicOr(status, kStatusTimeout);
+  return false;
+}
+
+// Wait until *flag != 0 and return it.  Bounded: gives up (returns 0) after
+// kSpinLimit polls or as soon as another CTA raised the abort flag, and then
+// records a timeout and raises the abort flag itself.
+__device__ __forceinline__ unsigned wait_flag_bounded(const unsigned *flag, unsigned *abort_flag,
+                                                      unsigned *status) {
+  unsigned f = ld_acquire(flag);
+  if (f) return f;
+  unsigned ns = 32;
+  for (unsigned it = 0; it < kSpinLimit; ++it) {
+    f = ld_acquire(flag);
+    if (f) return f;
+    if ((it & 63u) == 63u && ld_relaxed(abort_flag)) break;
+    if (it > 16) {
+      __nanosleep(ns);
+      ns = ns < 256 ? ns * 2 : 256;
+    }
+  }
+  atomicOr(status, kStatusTimeout);
+  atomicExch(abort_flag, 1u);
+  return 0;
+}
+
+}  // namespace esa

@@ -1,0 +1,39 @@
+// esa_dispatch.cuh -- maps runtime (dtype, mode, D) onto kernel template
+// instantiations.  Internal to the library.
+#pragma once
+
+#include "esa_launch.h"
+
+namespace esa {
+
+// Calls f.template operator()<T, MODE, LPH, VPR, L, K>() for the runtime
+// (dtype, mode, D); returns ESA_ERR_UNSUPPORTED (-3) for an unknown D.
+template <typename T, int MODE, typename F>
+int dispatch_d(int D, F &&f) {
+  constexpr int L = sizeof(T) == 4 ? 32 : 64;
+  constexpr int K = kStepsPerThread;
+  switch (D) {
+    case 8: return f.template operator()<T, MODE, 1, 16, L, K>();
+    case 16: return f.template operator()<T, MODE, 2, 16, L, K>();
+    case 32: return f.template operator()<T, MODE, 4, 16, L, K>();
+    case 64: return f.template operator()<T, MODE, 8, 16, L, K>();
+    case 128: return f.template operator()<T, MODE, 16, 16, L, K>();
+    case 256: return f.template operator()<T, MODE, 32, 32, L, K>();
+    default: return -3;
+  }
+}
+
+template <typename F>
+int dispatch(int dtype, int mode, int D, F &&f) {
+  if (mode != 0 && mode != 1) return -1;
+  switch (dtype) {
+    case 0: return mode ? dispatch_d<float, 1>(D, f) : dispatch_d<float, 0>(D, f);
+    case 1: return mode ? dispatch_d<__half, 1>(D, f) : dispatch_d<__half, 0>(D, f);
+    case 2: return mode ? dispatch_d<__nv_bfloat16, 1>(D, f) : dispatch_d<__nv_bfloat16, 0>(D, f);
+    default: return -1;
+  }
+}
+
+inline int launch_status(cudaError_t e) { return e == cudaSuccess ? 0 : -5; }
+
+}  // namespace esa

@@ -1,0 +1,32 @@
+// esa_fwd.cu -- instantiations and launcher of the forward scan kernel.
+#include "esa_dispatch.cuh"
+
+namespace esa {
+
+namespace {
+struct FwdLauncher {
+  const CUtensorMap &ta, &tv, &tq;
+  const FwdArgs &args;
+  int ntiles;
+  cudaStream_t stream;
+
+  template <typename T, int MODE, int LPH, int VPR, int L, int K>
+  int operator()() const {
+    using Cfg = TileCfg<T, LPH, VPR, L, K>;
+    const size_t smem = scan_smem_bytes<Cfg, 3>();
+    auto kern = esa_scan_fwd_kernel<T, MODE, LPH, VPR, L, K>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return launch_status(e);
+    kern<<<ntiles, Cfg::NT, smem, stream>>>(ta, tv, tq, args);
+    return launch_status(cudaGetLastError());
+  }
+};
+}  // namespace
+
+int launch_fwd(int dtype, int mode, int D, const CUtensorMap &ta, const CUtensorMap &tv,
+               const CUtensorMap &tq, const FwdArgs &args, int ntiles, cudaStream_t stream) {
+  return dispatch(dtype, mode, D, FwdLauncher{ta, tv, tq, args, ntiles, stream});
+}
+
+}  // namespace esa

@@ -1,0 +1,29 @@
+// esa_launch.h -- host-side launch interface between the C ABI layer and the
+// kernel instantiation units.  Internal to the library.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "esa_kernels.cuh"
+
+namespace esa {
+
+// Tile rows per chunk and channels per tile, as chosen for each I/O dtype and
+// head dimension.  The workspace layout and the kernels both follow these.
+inline int tile_rows(int dtype) { return dtype == 0 ? 32 : 64; }   // f32 : 16-bit
+inline int tile_cols(int D) { return D <= 128 ? 128 : 256; }
+constexpr int kStepsPerThread = 4;
+
+// Launch the forward / backward scan for (dtype, mode, D).  The tensor maps
+// describe a, v, q (and dy) as [B][T][C] boxes of [L][CT].  Return 0 or a
+// negative esa_status.
+int launch_fwd(int dtype, int mode, int D, const CUtensorMap &ta, const CUtensorMap &tv,
+               const CUtensorMap &tq, const FwdArgs &args, int ntiles, cudaStream_t stream);
+int launch_bwd(int dtype, int mode, int D, const CUtensorMap &ta, const CUtensorMap &tv,
+               const CUtensorMap &tq, const CUtensorMap &tdy, const BwdArgs &args, int ntiles,
+               cudaStream_t stream);
+int launch_step(int dtype, int mode, int D, const void *a, const void *v, const void *q, float *E,
+                void *y, long nvec, float inv_D, cudaStream_t stream);
+
+}  // namespace esa

@@ -1,0 +1,235 @@
+"""ctypes binding of the ESA scan C ABI (``include/esa.h``).
+
+Argument marshalling only: every step of the scan runs in the CUDA library
+``lib/libesa_b200.so``.  PyTorch supplies device memory and the current CUDA
+stream.  There is no CPU path: CPU tensors, a missing library or a non-B200
+device raise an error.
+
+The functions carry the C names:
+
+* :func:`esa_scan_fwd`  -- forward scan (+ E_final, + checkpoints in the workspace)
+* :func:`esa_scan_bwd`  -- backward scan (da, dv, dq, dE_init)
+* :func:`esa_step`      -- one-token decode update (in place on E)
+* :func:`esa_check`     -- synchronise and read the device status of a workspace
+* :func:`esa_workspace_size`, :func:`esa_strerror`, :func:`esa_version`
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libesa_b200.so")
+
+DIRECT = 0
+CONTROLLED = 1
+_DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+
+ESA_OK = 0
+ESA_ERR_ARG = -1
+ESA_ERR_ALIGN = -2
+ESA_ERR_UNSUPPORTED = -3
+ESA_ERR_WORKSPACE = -4
+ESA_ERR_LAUNCH = -5
+ESA_ERR_TIMEOUT = -6
+ESA_ERR_DEVICE = -7
+
+_lock = threading.Lock()
+_lib = None
+
+
+class EsaError(RuntimeError):
+    """A non-zero status returned by the C ABI."""
+
+    def __init__(self, func, code):
+        self.code = code
+        super().__init__(f"{func} failed: {esa_strerror(code)} (status {code})")
+
+
+def load_library():
+    """Load ``libesa_b200.so`` (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"ESA CUDA library not found at {LIB_PATH}; build it with "
+                "`python -m gated_linear_recurrence_b200.build` (there is no CPU fallback)")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        lib.esa_workspace_size.argtypes = [I, I, I, I, I]
+        lib.esa_workspace_size.restype = S
+        lib.esa_scan_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I, P, S, P]
+        lib.esa_scan_fwd.restype = I
+        lib.esa_scan_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, P, I, P, S, P]
+        lib.esa_scan_bwd.restype = I
+        lib.esa_step.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
+        lib.esa_step.restype = I
+        lib.esa_check.argtypes = [P, P]
+        lib.esa_check.restype = I
+        lib.esa_strerror.argtypes = [I]
+        lib.esa_strerror.restype = ctypes.c_char_p
+        lib.esa_version.argtypes = []
+        lib.esa_version.restype = I
+        _lib = lib
+        return lib
+
+
+def esa_strerror(code: int) -> str:
+    return load_library().esa_strerror(int(code)).decode()
+
+
+def esa_version() -> int:
+    return int(load_library().esa_version())
+
+
+def esa_workspace_size(B: int, T: int, H: int, D: int, dtype) -> int:
+    code = _DTYPE_CODE[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    return int(load_library().esa_workspace_size(B, T, H, D, code))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device, stream):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_seq(name, t, ref):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (the ESA library has no CPU path)")
+    if t.shape != ref.shape or t.dtype != ref.dtype or t.device != ref.device:
+        raise ValueError(f"{name} must match a: shape {tuple(ref.shape)}, dtype {ref.dtype}, {ref.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous [B, T, H, D]")
+
+
+def _check_state(name, t, B, H, D, device):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.device != device:
+        raise TypeError(f"{name} must be a CUDA tensor on {device}")
+    if tuple(t.shape) != (B, H, D) or t.dtype != torch.float32 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous float32 tensor of shape {(B, H, D)}")
+
+
+def _dims(a):
+    if not isinstance(a, torch.Tensor) or not a.is_cuda:
+        raise TypeError("a must be a CUDA tensor (the ESA library has no CPU path)")
+    if a.dim() != 4:
+        raise ValueError("sequence tensors must be [B, T, H, D]")
+    if a.dtype not in _DTYPE_CODE:
+        raise TypeError(f"unsupported dtype {a.dtype}")
+    if not a.is_contiguous():
+        raise ValueError("a must be contiguous [B, T, H, D]")
+    return tuple(int(s) for s in a.shape)
+
+
+def new_workspace(B, T, H, D, dtype, device):
+    """Allocate a workspace of the size the C ABI asks for (torch memory, caller-owned)."""
+    n = esa_workspace_size(B, T, H, D, dtype)
+    if n == 0:
+        raise ValueError("unsupported shape for the ESA scan")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def esa_scan_fwd(a, v, q, y=None, E_final=None, mode=CONTROLLED, E_init=None, workspace=None,
+                 stream=None, want_E_final=True):
+    """Forward scan.  Returns ``(y, E_final, workspace)``.
+
+    ``workspace`` (uint8 CUDA tensor) is allocated when not given; keep it for
+    :func:`esa_scan_bwd`.  ``E_final`` is allocated when not given unless
+    ``want_E_final`` is False.
+    """
+    B, T, H, D = _dims(a)
+    _check_seq("v", v, a)
+    _check_seq("q", q, a)
+    if y is None:
+        y = torch.empty_like(a)
+    _check_seq("y", y, a)
+    if E_final is None and want_E_final:
+        E_final = torch.empty((B, H, D), dtype=torch.float32, device=a.device)
+    _check_state("E_final", E_final, B, H, D, a.device)
+    _check_state("E_init", E_init, B, H, D, a.device)
+    if workspace is None:
+        workspace = new_workspace(B, T, H, D, a.dtype, a.device)
+    lib = load_library()
+    with torch.cuda.device(a.device):
+        rc = lib.esa_scan_fwd(_ptr(a), _ptr(v), _ptr(q), _ptr(y), _ptr(E_final), B, T, H, D, int(mode),
+                              _ptr(E_init), _DTYPE_CODE[a.dtype], _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(a.device, stream))
+    if rc != 0:
+        raise EsaError("esa_scan_fwd", rc)
+    return y, E_final, workspace
+
+
+def esa_scan_bwd(a, v, q, dy, workspace, mode=CONTROLLED, E_init=None, dE_final=None, da=None, dv=None,
+                 dq=None, dE_init=None, stream=None, want_dE_init=True):
+    """Backward scan.  ``workspace`` must be the one the matching forward wrote.
+
+    Returns ``(da, dv, dq, dE_init)``.
+    """
+    B, T, H, D = _dims(a)
+    for name, t in (("v", v), ("q", q), ("dy", dy)):
+        _check_seq(name, t, a)
+    da = torch.empty_like(a) if da is None else da
+    dv = torch.empty_like(a) if dv is None else dv
+    dq = torch.empty_like(a) if dq is None else dq
+    for name, t in (("da", da), ("dv", dv), ("dq", dq)):
+        _check_seq(name, t, a)
+    if dE_init is None and want_dE_init:
+        dE_init = torch.empty((B, H, D), dtype=torch.float32, device=a.device)
+    _check_state("dE_init", dE_init, B, H, D, a.device)
+    _check_state("dE_final", dE_final, B, H, D, a.device)
+    _check_state("E_init", E_init, B, H, D, a.device)
+    if workspace is None or not workspace.is_cuda:
+        raise ValueError("esa_scan_bwd needs the CUDA workspace written by the matching esa_scan_fwd")
+    lib = load_library()
+    with torch.cuda.device(a.device):
+        rc = lib.esa_scan_bwd(_ptr(a), _ptr(v), _ptr(q), _ptr(dy), _ptr(dE_final), _ptr(da), _ptr(dv),
+                              _ptr(dq), _ptr(dE_init), B, T, H, D, int(mode), _ptr(E_init),
+                              _DTYPE_CODE[a.dtype], _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(a.device, stream))
+    if rc != 0:
+        raise EsaError("esa_scan_bwd", rc)
+    return da, dv, dq, dE_init
+
+
+def esa_step(a_t, v_t, q_t, E, y_t=None, mode=CONTROLLED, stream=None):
+    """One-token update: E (float32 [B, H, D]) is updated in place.  Returns ``y_t``."""
+    if not isinstance(a_t, torch.Tensor) or not a_t.is_cuda or a_t.dim() != 3:
+        raise TypeError("a_t must be a CUDA tensor [B, H, D] (the ESA library has no CPU path)")
+    if a_t.dtype not in _DTYPE_CODE or not a_t.is_contiguous():
+        raise ValueError("a_t must be contiguous with dtype float32, float16 or bfloat16")
+    B, H, D = (int(s) for s in a_t.shape)
+    for name, t in (("v_t", v_t), ("q_t", q_t)):
+        if t.shape != a_t.shape or t.dtype != a_t.dtype or t.device != a_t.device or not t.is_contiguous():
+            raise ValueError(f"{name} must match a_t")
+    _check_state("E", E, B, H, D, a_t.device)
+    if E is None:
+        raise ValueError("E (the recurrent state) is required")
+    if y_t is None:
+        y_t = torch.empty_like(a_t)
+    lib = load_library()
+    with torch.cuda.device(a_t.device):
+        rc = lib.esa_step(_ptr(a_t), _ptr(v_t), _ptr(q_t), _ptr(E), _ptr(y_t), B, H, D, int(mode),
+                          _DTYPE_CODE[a_t.dtype], _stream(a_t.device, stream))
+    if rc != 0:
+        raise EsaError("esa_step", rc)
+    return y_t
+
+
+def esa_check(workspace, stream=None):
+    """Synchronise the stream and raise :class:`EsaError` if a device-side wait gave up."""
+    lib = load_library()
+    with torch.cuda.device(workspace.device):
+        rc = lib.esa_check(_ptr(workspace), _stream(workspace.device, stream))
+    if rc != 0:
+        raise EsaError("esa_check", rc)

@@ -1,0 +1,151 @@
+/*
+ * esa.h -- C ABI of the B200 (sm_100a) ESA scan library.
+ *
+ * The library evaluates the gated linear recurrence of Entangled State
+ * Attention (ESA),
+ *
+ *     E_t = A_t (.) E_{t-1} + B_t,      A_t = sigmoid(a_t),
+ *     B_t = v_t                  (direct mode),
+ *     B_t = (1 - A_t) (.) v_t    (controlled mode),
+ *     y_t = q_t (.) E_t / sqrt(mean_d(E_t^2) + 1e-6)   (per-head RMS readout),
+ *
+ * for every (batch, head, channel), as a chunked associative prefix scan over
+ * time on the GPU, together with its backward pass and the one-token decode
+ * update.  Sources: the recurrence is stated in "Entangled State Attention
+ * v2.1" (entangled_state_attention-2.1.0 PKG-INFO, opening section) and in
+ * the "Core recurrence" panel of mlbricks-web.pages.dev/esa; the direct and
+ * controlled modes and the readout y_t = W_O(q_t (.) Norm(E_t)) are in
+ * "entangled-state-attention 0.1.0" (PyPI), section "Core idea".  Norm is
+ * left open there and is fixed here as an RMS over the D channels of a head,
+ * eps = 1e-6 inside the square root, no learned scale.  The projections
+ * (x W_A, x W_V, x W_Q, W_O) are not part of this library: a, v, q are their
+ * outputs (a is the gate logit, before the sigmoid) and y is q (.) Norm(E).
+ *
+ * Conventions shared by every entry point:
+ *   - All pointers are DEVICE pointers owned by the caller; the library never
+ *     allocates, frees or retains them.  Every pointer must be 16-byte
+ *     aligned.  Optional pointers may be NULL where stated.
+ *   - Sequence tensors (a, v, q, y, dy, da, dv, dq) are contiguous
+ *     [B, T, H, D] in the I/O dtype; state tensors (E_init, E_final, E,
+ *     dE_final, dE_init) are contiguous [B, H, D] in float32.  C = H * D.
+ *   - dtype is one of esa_dtype; all arithmetic and the state are float32,
+ *     outputs are rounded to the I/O dtype with round-to-nearest-even.
+ *   - D must be one of 8, 16, 32, 64, 128, 256; H >= 1; B >= 0; T >= 0.
+ *   - stream is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Every call only enqueues work and returns; it does not
+ *     synchronise.  Calls that share a workspace must be ordered (same
+ *     stream, or events) and must not overlap.
+ *   - Return value: ESA_OK (0) or a negative esa_status.  Argument errors are
+ *     detected on the host before anything is enqueued.  A device-side
+ *     failure (a bounded wait that gave up) is recorded in the workspace and
+ *     reported by esa_check().
+ */
+#ifndef ESA_H_
+#define ESA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Recurrence mode ("entangled-state-attention 0.1.0", "Direct vs controlled mode"). */
+typedef enum { ESA_DIRECT = 0, ESA_CONTROLLED = 1 } esa_mode;
+
+/* I/O element type of the sequence tensors. */
+typedef enum { ESA_F32 = 0, ESA_F16 = 1, ESA_BF16 = 2 } esa_dtype;
+
+typedef enum {
+    ESA_OK = 0,
+    ESA_ERR_ARG = -1,         /* bad size, mode, dtype or a required NULL pointer */
+    ESA_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned */
+    ESA_ERR_UNSUPPORTED = -3, /* head dimension D outside {8,16,32,64,128,256} */
+    ESA_ERR_WORKSPACE = -4,   /* workspace NULL or smaller than esa_workspace_size() */
+    ESA_ERR_LAUNCH = -5,      /* the CUDA runtime rejected a launch or copy */
+    ESA_ERR_TIMEOUT = -6,     /* a bounded device-side wait gave up (see esa_check) */
+    ESA_ERR_DEVICE = -7       /* no CUDA device, or the current device is not sm_100 */
+} esa_status;
+
+/*
+ * Bytes of device workspace that esa_scan_fwd / esa_scan_bwd need for a
+ * problem of this shape and dtype (0 on a bad argument).  The workspace
+ * holds the float32 state at the end of every time chunk of every sequence
+ * (written by the forward, read by the backward) plus the per-chunk carry
+ * descriptors and status words of the single-pass scan.  About
+ * 16 * B * C * ceil(T / L) bytes, L = 64 for 16-bit I/O and 32 for float32.
+ */
+size_t esa_workspace_size(int B, int T, int H, int D, int dtype);
+
+/*
+ * Forward scan (prefill / training forward).
+ *   a, v, q   [B,T,H,D] inputs: gate logits, values, queries (required).
+ *   y         [B,T,H,D] output: q (.) E_t / rms(E_t) (required).
+ *   E_final   [B,H,D] float32 output: E_T, the state to continue decoding
+ *             from (NULL = not written).  With T = 0 it equals E_init.
+ *   E_init    [B,H,D] float32 initial state E_0 (NULL = zeros).
+ *   workspace device buffer of at least esa_workspace_size() bytes; its
+ *             previous contents are irrelevant.  After the call it holds the
+ *             chunk-boundary states that esa_scan_bwd needs, so keep it
+ *             unchanged until the matching backward has run.
+ * Sources: state recurrence and modes ("entangled-state-attention 0.1.0",
+ * "Core idea"); prefill returning the state (mlbricks-web.pages.dev/esa,
+ * Quick start: prefill returns (out, state)).
+ */
+int esa_scan_fwd(const void *a, const void *v, const void *q, void *y, float *E_final,
+                 int B, int T, int H, int D, int mode, const float *E_init,
+                 int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Backward scan: gradients of  sum(dy . y) + sum(dE_final . E_final)
+ * with respect to a, v, q and E_init.
+ *   a, v, q, E_init  exactly the forward's inputs (E_init NULL = zeros).
+ *   dy        [B,T,H,D] upstream gradient of y (required).
+ *   dE_final  [B,H,D] float32 upstream gradient of E_final (NULL = zeros).
+ *   da, dv, dq [B,T,H,D] outputs in the I/O dtype (required).
+ *   dE_init   [B,H,D] float32 output (NULL = not written).
+ *   workspace the buffer the matching esa_scan_fwd wrote, unchanged since;
+ *             the chunk-boundary states in it are read, the rest is scratch.
+ * The pages do not print the backward; it is the chain rule of the forward
+ * (training through the layer with loss.backward(), "Entangled State
+ * Attention v2.1", Trainer section):
+ *   G_t = ghat_t + A_{t+1} G_{t+1}, G_T = ghat_T + dE_final,
+ *   ghat_t = r (dn - n mean_d(dn n)), n = E r, dn = dy q, dq = dy n,
+ *   direct: dv = G, da = G E_{t-1} A(1-A);
+ *   controlled: dv = G (1-A), da = G (E_{t-1} - v) A(1-A);  dE_init = A_1 G_1.
+ */
+int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy,
+                 const float *dE_final, void *da, void *dv, void *dq, float *dE_init,
+                 int B, int T, int H, int D, int mode, const float *E_init,
+                 int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One-token recurrent update (decode): E <- A (.) E + B in place, then
+ * y_t = q_t (.) E / rms(E).
+ *   a_t, v_t, q_t [B,H,D] inputs of one token; y_t [B,H,D] output (I/O dtype).
+ *   E             [B,H,D] float32 state, read and overwritten.
+ * Needs no workspace.  Sources: mlbricks-web.pages.dev/esa, Architecture
+ * step "One-token update" and Quick start decode_step(token, state);
+ * "Entangled State Attention v2.1", ESA-Lightning lightning_step.
+ */
+int esa_step(const void *a_t, const void *v_t, const void *q_t, float *E, void *y_t,
+             int B, int H, int D, int mode, int dtype, void *stream);
+
+/*
+ * Synchronise `stream`, then read and clear the device status word in
+ * `workspace`.  Returns ESA_OK, ESA_ERR_TIMEOUT if a bounded wait inside a
+ * scan kernel gave up since the last check (the outputs of that call are
+ * then invalid), or ESA_ERR_LAUNCH if the stream reports a CUDA error.
+ */
+int esa_check(void *workspace, void *stream);
+
+/* Static, human-readable text for an esa_status code. */
+const char *esa_strerror(int status);
+
+/* Library version as 10000 * major + 100 * minor + patch. */
+int esa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ESA_H_ */

@@ -1,0 +1,143 @@
+"""Host-side checks of the C ABI: no GPU needed, no compute launched.
+
+* the shared library loads and exports every function ``include/esa.h`` declares;
+* workspace sizing follows the documented layout;
+* argument, alignment and workspace errors are reported before any CUDA call;
+* on a machine without a CUDA device a well-formed call reports ESA_ERR_DEVICE
+  (it never falls back to a CPU path).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "esa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_linear_recurrence_b200 import build
+    build.build()
+    from gated_linear_recurrence_b200 import esa
+    return esa.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(esa_[a-z_]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_three_entry_points():
+    names = declared_functions()
+    for n in ("esa_scan_fwd", "esa_scan_bwd", "esa_step", "esa_workspace_size", "esa_check",
+              "esa_strerror", "esa_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/esa.h but not exported"
+
+
+def test_exports_are_c_linkage():
+    import subprocess
+    from gated_linear_recurrence_b200 import esa
+    out = subprocess.run(["nm", "-D", "--defined-only", esa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT\s+(esa_[a-z_]+)\b", out))
+    assert set(declared_functions()) <= exported
+
+
+def test_version_and_strerror(lib):
+    from gated_linear_recurrence_b200 import esa
+    assert esa.esa_version() == 100
+    for code in range(-7, 1):
+        assert esa.esa_strerror(code)
+    assert "unknown" in esa.esa_strerror(-99)
+
+
+@pytest.mark.parametrize("dtype,L", [(0, 32), (1, 64), (2, 64)])
+def test_workspace_size_layout(lib, dtype, L):
+    B, T, H, D = 3, 1000, 5, 64          # C = 320 -> 3 channel tiles of 128
+    n = B * 3 * -(-T // L)
+    expect = 0
+
+    def up(x):
+        return -(-x // 256) * 256
+    expect = up(32 + 4 * n)
+    expect = up(expect + 16 + 4 * n)
+    expect = up(expect + n * 128 * 8)
+    expect = up(expect + n * 128 * 4)
+    expect = up(expect + n * 128 * 4)
+    assert lib.esa_workspace_size(B, T, H, D, dtype) == expect
+
+
+def test_workspace_size_rejects_bad_shapes(lib):
+    assert lib.esa_workspace_size(1, 10, 2, 24, 1) == 0     # D not supported
+    assert lib.esa_workspace_size(-1, 10, 2, 32, 1) == 0
+    assert lib.esa_workspace_size(1, 10, 0, 32, 1) == 0
+    assert lib.esa_workspace_size(1, 10, 2, 32, 7) == 0
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def _fwd(lib, a=0x1000, v=0x2000, q=0x3000, y=0x4000, Ef=0, B=2, T=8, H=2, D=32, mode=1, Ei=0,
+         dtype=1, ws=0x10000, wsb=1 << 30):
+    return lib.esa_scan_fwd(_fake(a), _fake(v), _fake(q), _fake(y), _fake(Ef) if Ef else None, B, T, H, D,
+                            mode, _fake(Ei) if Ei else None, dtype, _fake(ws) if ws else None, wsb, None)
+
+
+def test_fwd_argument_errors(lib):
+    from gated_linear_recurrence_b200 import esa
+    assert _fwd(lib, mode=2) == esa.ESA_ERR_ARG
+    assert _fwd(lib, dtype=3) == esa.ESA_ERR_ARG
+    assert _fwd(lib, B=-1) == esa.ESA_ERR_ARG
+    assert _fwd(lib, H=0) == esa.ESA_ERR_ARG
+    assert _fwd(lib, D=24) == esa.ESA_ERR_UNSUPPORTED
+    assert _fwd(lib, D=512) == esa.ESA_ERR_UNSUPPORTED
+    assert _fwd(lib, a=0) == esa.ESA_ERR_ARG
+    assert _fwd(lib, y=0) == esa.ESA_ERR_ARG
+    assert _fwd(lib, q=0x3008) == esa.ESA_ERR_ALIGN
+    assert _fwd(lib, Ef=0x5004) == esa.ESA_ERR_ALIGN
+    assert _fwd(lib, ws=0) == esa.ESA_ERR_WORKSPACE
+    assert _fwd(lib, wsb=64) == esa.ESA_ERR_WORKSPACE
+
+
+def test_bwd_and_step_argument_errors(lib):
+    from gated_linear_recurrence_b200 import esa
+    P = _fake
+    rc = lib.esa_scan_bwd(P(0x1000), P(0x2000), P(0x3000), None, None, P(0x5000), P(0x6000), P(0x7000),
+                          None, 2, 8, 2, 32, 1, None, 1, P(0x10000), 1 << 30, None)
+    assert rc == esa.ESA_ERR_ARG                                   # dy missing
+    rc = lib.esa_scan_bwd(P(0x1000), P(0x2000), P(0x3000), P(0x4000), None, P(0x5000), P(0x6000),
+                          P(0x7001), None, 2, 8, 2, 32, 1, None, 1, P(0x10000), 1 << 30, None)
+    assert rc == esa.ESA_ERR_ALIGN                                 # dq misaligned
+    rc = lib.esa_step(P(0x1000), P(0x2000), P(0x3000), None, P(0x5000), 2, 2, 32, 1, 1, None)
+    assert rc == esa.ESA_ERR_ARG                                   # E missing
+    rc = lib.esa_step(P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000), 2, 2, 40, 1, 1, None)
+    assert rc == esa.ESA_ERR_UNSUPPORTED
+
+
+def test_no_device_is_an_error_not_a_fallback(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present; this checks the device-less path")
+    from gated_linear_recurrence_b200 import esa
+    assert _fwd(lib) == esa.ESA_ERR_DEVICE
+    assert lib.esa_step(_fake(0x1000), _fake(0x2000), _fake(0x3000), _fake(0x4000), _fake(0x5000),
+                        2, 2, 32, 1, 1, None) == esa.ESA_ERR_DEVICE
+
+
+def test_binding_rejects_cpu_tensors(lib):
+    import torch
+    from gated_linear_recurrence_b200 import esa
+    x = torch.zeros(1, 4, 2, 32, dtype=torch.float16)
+    with pytest.raises(TypeError):
+        esa.esa_scan_fwd(x, x, x)
+    with pytest.raises(TypeError):
+        esa.esa_step(x[:, 0], x[:, 0], x[:, 0], torch.zeros(1, 2, 32))
