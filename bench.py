@@ -53,12 +53,19 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="run a smaller batch of the same workload (profiling cases only)")
     return ap.parse_args(argv)
 
 
-def workload():
+def workload(batch=None):
+    import dataclasses
+
     from gated_linear_recurrence_b200 import inputs
-    return inputs.WORKLOADS[WORKLOAD_NAME]
+    w = inputs.WORKLOADS[WORKLOAD_NAME]
+    if batch is not None and batch != w.B:
+        w = dataclasses.replace(w, B=int(batch), name=f"{w.name} (batch reduced to {batch})")
+    return w
 
 
 def config_dict(w):
@@ -168,8 +175,8 @@ class ClockSampler:
 # CPU oracle legs (the oracle is test infrastructure; only these legs use it).
 # ---------------------------------------------------------------------------
 
-def oracle_sample_tokens_per_s(w, rows, T, seed):
-    """Time the fp64 oracle (fwd + bwd) on `rows` batch rows x T tokens."""
+def oracle_sample_seconds(w, rows, T, seed):
+    """Seconds the fp64 oracle takes for fwd + bwd of `rows` batch rows x T tokens."""
     import torch
 
     import oracle
@@ -179,8 +186,20 @@ def oracle_sample_tokens_per_s(w, rows, T, seed):
     t0 = time.perf_counter()
     oracle.scan_fwd(f64["a"], f64["v"], f64["q"], w.mode)
     oracle.scan_bwd(f64["a"], f64["v"], f64["q"], f64["dy"], w.mode)
-    dt = time.perf_counter() - t0
-    return rows * T / dt, dt
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, budget_s=10.0):
+    """The oracle on whole batch rows of the workload, one row at a time, until
+    about `budget_s` seconds of CPU work (or the whole batch) are done."""
+    secs, rows = 0.0, 0
+    while rows < w.B and secs < budget_s:
+        secs += oracle_sample_seconds(w, 1, w.T, seed=4242 + rows)
+        rows += 1
+    return {"value": rows * w.T / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"fwd+bwd of {rows} of the {w.B} batch rows x {w.T} tokens x C={w.C} (controlled, "
+                      f"fp16-rounded inputs in fp64) through the sequential C oracle on one host core: "
+                      f"{secs:.1f} s"}
 
 
 def run_reference(args):
@@ -188,17 +207,16 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = workload()
-    rows, T = 1, 8192
+    w = workload(args.batch)
+    rows, T = 1, 16384
     for i in range(args.warmup):
-        oracle_sample_tokens_per_s(w, rows, T, seed=1000 + i)
-    t0 = time.perf_counter()
+        oracle_sample_seconds(w, rows, T, seed=1000 + i)
+    dt = 0.0
     for i in range(args.steps):
-        oracle_sample_tokens_per_s(w, rows, T, seed=2000 + i)
-    dt = time.perf_counter() - t0
+        dt += oracle_sample_seconds(w, rows, T, seed=2000 + i)
     value = args.steps * rows * T / dt
-    sample = (f"each step: fwd+bwd of {rows} batch row x {T} tokens x C={w.C} (controlled, fp16-rounded "
-              f"inputs in fp64) through the sequential C oracle on one host core")
+    sample = (f"each step: fwd+bwd of {rows} batch row x the first {T} tokens x C={w.C} (controlled, "
+              f"fp16-rounded inputs in fp64) through the sequential C oracle on one host core")
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -240,7 +258,7 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    w = workload()
+    w = workload(args.batch)
     B, T, H, D, mode = w.B, w.T, w.H, w.D, w.mode
     x = inputs.make_scan_inputs(B, T, H, D, w.dtype, w.a_mean, w.seed + 17 * rank, device=dev)
     a, v, q, dy = x["a"], x["v"], x["q"], x["dy"]
@@ -344,11 +362,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rows = 2
-        tps, secs = oracle_sample_tokens_per_s(w, rows, T, seed=4242)
-        cpu = {"value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-               "sample": f"fwd+bwd of {rows} batch rows x {T} tokens x C={C} (controlled, fp16-rounded inputs "
-                         f"in fp64) through the sequential C oracle on one host core: {secs:.1f} s"}
+        cpu = cpu_baseline(w)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,

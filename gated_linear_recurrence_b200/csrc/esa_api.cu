@@ -169,6 +169,7 @@ esa::ScanShape scan_shape(int B, int T, int H, int D, const Layout &lo) {
   s.nchunks = lo.nchunks;
   s.nct = lo.nct;
   s.nchains = lo.nchains;
+  s.ntiles = static_cast<int>(lo.ntiles);
   s.inv_D = 1.0f / static_cast<float>(D);
   return s;
 }
@@ -194,7 +195,8 @@ int esa_scan_fwd(const void *a, const void *v, const void *q, void *y, float *E_
                  size_t workspace_bytes, void *stream) {
   int rc = check_shape(B, T, H, D, mode, dtype);
   if (rc) return rc;
-  if (!a || !v || !q || !y) return ESA_ERR_ARG;
+  const bool has_tokens = B > 0 && T > 0;   // empty tensors may carry NULL pointers
+  if (has_tokens && (!a || !v || !q || !y)) return ESA_ERR_ARG;
   for (const void *p : {a, v, q, static_cast<const void *>(y), static_cast<const void *>(E_final),
                         static_cast<const void *>(E_init), static_cast<const void *>(workspace)})
     if (p && !aligned16(p)) return ESA_ERR_ALIGN;
@@ -230,7 +232,8 @@ int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy, co
                  const float *E_init, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
   int rc = check_shape(B, T, H, D, mode, dtype);
   if (rc) return rc;
-  if (!a || !v || !q || !dy || !da || !dv || !dq) return ESA_ERR_ARG;
+  const bool has_tokens = B > 0 && T > 0;   // empty tensors may carry NULL pointers
+  if (has_tokens && (!a || !v || !q || !dy || !da || !dv || !dq)) return ESA_ERR_ARG;
   for (const void *p : {a, v, q, dy, static_cast<const void *>(dE_final), static_cast<const void *>(da),
                         static_cast<const void *>(dv), static_cast<const void *>(dq),
                         static_cast<const void *>(dE_init), static_cast<const void *>(E_init),
@@ -272,9 +275,9 @@ int esa_step(const void *a_t, const void *v_t, const void *q_t, float *E, void *
              int mode, int dtype, void *stream) {
   int rc = check_shape(B, 1, H, D, mode, dtype);
   if (rc) return rc;
-  if (!a_t || !v_t || !q_t || !E || !y_t) return ESA_ERR_ARG;
+  if (B > 0 && (!a_t || !v_t || !q_t || !E || !y_t)) return ESA_ERR_ARG;
   for (const void *p : {a_t, v_t, q_t, static_cast<const void *>(E), static_cast<const void *>(y_t)})
-    if (!aligned16(p)) return ESA_ERR_ALIGN;
+    if (p && !aligned16(p)) return ESA_ERR_ALIGN;
   if ((rc = check_device())) return rc;
   if (B == 0) return ESA_OK;
   const long nvec = static_cast<long>(B) * H * D / 8;

@@ -101,19 +101,42 @@ template <> struct Io<__nv_bfloat16> {
 };
 
 // ---------------------------------------------------------------------------
-// Gate.  u = exp(-x) with x clamped at -80 so u stays finite; then
-//   A = 1 / (1 + u)      (sigmoid)
+// Approximate transcendental instructions (PTX ex2/rcp/rsqrt .approx.ftz).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float rsqrt_approx(float x) {
+  float y;
+  asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ---------------------------------------------------------------------------
+// Gate.  With u = exp(-x) = 2^(-x log2 e) (x clamped at -80 so u stays
+// finite):
+//   A = 1 / (1 + u)      (the logistic sigmoid)
 //   1 - A = u * A        (no cancellation when A is close to 1)
-// CUDA's fast exp and divide intrinsics are used as-is.
 // ---------------------------------------------------------------------------
 struct Gate {
   float A;    // sigmoid(x)
   float Ac;   // 1 - sigmoid(x)
 };
 
+constexpr float kLog2e = 1.4426950408889634f;
+
 __device__ __forceinline__ Gate gate_of(float x) {
-  const float u = __expf(-fmaxf(x, -80.0f));
-  const float A = __fdividef(1.0f, 1.0f + u);
+  const float u = ex2_approx(fmaxf(x, -80.0f) * -kLog2e);
+  const float A = rcp_approx(1.0f + u);
   return Gate{A, u * A};
 }
 
@@ -149,15 +172,16 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, unsigned bytes) {
                : "memory");
 }
 
-// Non-blocking test of an mbarrier phase.
-__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, unsigned phase) {
+// Wait on an mbarrier phase; the hardware may suspend the thread for up to
+// about a microsecond (the hint) before returning false.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned phase) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(phase)
+      : "r"(smem_u32(bar)), "r"(phase), "r"(1000u)
       : "memory");
   return ok != 0;
 }
@@ -189,8 +213,15 @@ __device__ __forceinline__ unsigned ld_relaxed(const unsigned *p) {
   return v;
 }
 
-__device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+__device__ __forceinline__ void st_relaxed(unsigned *p, unsigned v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Release fence at GPU scope.  Issued by one thread after a CTA barrier, it
+// orders the barrier participants' earlier writes before the thread's next
+// (flag) store, as seen by any thread that acquires that flag.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
 // Named barrier over the first `nthreads` threads of the CTA (id 1; id 0 is __syncthreads).
@@ -198,37 +229,13 @@ __device__ __forceinline__ void bar_sync_first(unsigned nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
-// Wait for the TMA transaction on `bar` (phase 0).  Bounded: on giving up it
-// records a timeout in the status word and returns false.
+// Wait for the TMA transaction on `bar` (given phase parity).  Bounded: on
+// giving up it records a timeout in the status word and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned phase, unsigned *status) {
-  for (unsigned it = 0; it < kSpinLimit; ++it) {
-    if (mbar_test_wait(bar, phase)) return true;
-    if (it > 16) __nanosleep(64);
-  }
+  for (unsigned it = 0; it < kSpinLimit; ++it)
+    if (mbar_try_wait(bar, phase)) return true;
   atomicOr(status, kStatusTimeout);
   return false;
-}
-
-// Wait until *flag != 0 and return it.  Bounded: gives up (returns 0) after
-// kSpinLimit polls or as soon as another CTA raised the abort flag, and then
-// records a timeout and raises the abort flag itself.
-__device__ __forceinline__ unsigned wait_flag_bounded(const unsigned *flag, unsigned *abort_flag,
-                                                      unsigned *status) {
-  unsigned f = ld_acquire(flag);
-  if (f) return f;
-  unsigned ns = 32;
-  for (unsigned it = 0; it < kSpinLimit; ++it) {
-    f = ld_acquire(flag);
-    if (f) return f;
-    if ((it & 63u) == 63u && ld_relaxed(abort_flag)) break;
-    if (it > 16) {
-      __nanosleep(ns);
-      ns = ns < 256 ? ns * 2 : 256;
-    }
-  }
-  atomicOr(status, kStatusTimeout);
-  atomicExch(abort_flag, 1u);
-  return 0;
 }
 
 }  // namespace esa

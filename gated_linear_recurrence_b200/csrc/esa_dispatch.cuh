@@ -36,4 +36,21 @@ int dispatch(int dtype, int mode, int D, F &&f) {
 
 inline int launch_status(cudaError_t e) { return e == cudaSuccess ? 0 : -5; }
 
+// Grid of a persistent scan kernel: as many CTAs as can be resident at once
+// (occupancy x SM count), never more than there are tiles.
+template <typename Kern>
+int persistent_grid(Kern kern, int nthreads, size_t smem, int ntiles, int *grid) {
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -5;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return -5;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nthreads, smem) != cudaSuccess) return -5;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -5;
+  if (per_sm < 1 || sms < 1) return -5;
+  const long long g = static_cast<long long>(per_sm) * sms;
+  *grid = static_cast<int>(g < ntiles ? g : ntiles);
+  return 0;
+}
+
 }  // namespace esa

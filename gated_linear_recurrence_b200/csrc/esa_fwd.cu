@@ -13,12 +13,12 @@ struct FwdLauncher {
   template <typename T, int MODE, int LPH, int VPR, int L, int K>
   int operator()() const {
     using Cfg = TileCfg<T, LPH, VPR, L, K>;
-    const size_t smem = scan_smem_bytes<Cfg, 3>();
+    const size_t smem = FwdSmem<Cfg>::kBytes;
     auto kern = esa_scan_fwd_kernel<T, MODE, LPH, VPR, L, K>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return launch_status(e);
-    kern<<<ntiles, Cfg::NT, smem, stream>>>(ta, tv, tq, args);
+    int grid = 0;
+    const int rc = persistent_grid(kern, Cfg::NT, smem, ntiles, &grid);
+    if (rc) return rc;
+    kern<<<grid, Cfg::NT, smem, stream>>>(ta, tv, tq, args);
     return launch_status(cudaGetLastError());
   }
 };

@@ -5,23 +5,26 @@
 //   * A "chain" is one batch row b and one tile of CT consecutive channels
 //     (CT = 128, or 256 when the head dimension is 256).  Heads never straddle
 //     a channel tile, so the per-head RMS readout stays inside one CTA.
-//   * A chain is cut into time chunks of L steps.  One CTA processes one
-//     (chain, chunk) tile; the tile's a/v/q(/dy) boxes [L x CT] are staged in
-//     shared memory by TMA tensor loads (cp.async.bulk.tensor, no multicast).
+//   * A chain is cut into time chunks of L steps.  A tile is one (chain,
+//     chunk); its a/v/q(/dy) boxes [L x CT] are staged in shared memory by TMA
+//     tensor loads (cp.async.bulk.tensor, no multicast).
 //   * Inside a tile every thread owns 8 consecutive channels (one 16-byte
 //     vector for 16-bit I/O) and a run of K consecutive time steps.  Pass 1
 //     folds its run into an affine map x -> P x + S per channel; the runs of a
 //     tile are combined by a short serial scan per channel in shared memory;
-//     the tile map is then chained to earlier tiles by a single-pass
-//     decoupled look-back over per-chunk flags in the workspace.  Pass 2
-//     replays the run from its exact carry-in and emits the readout.
+//     the tile map is chained to earlier tiles by a single-pass decoupled
+//     look-back over per-chunk flags in the workspace, one warp polling a
+//     window of 32 predecessors at a time.  Pass 2 replays the run from its
+//     exact carry-in and emits the readout.
 //   * The carry is always applied in chunk order, oldest first, with the same
 //     fused multiply-add that the producing tile used for its own inclusive
 //     state, so the result is bitwise independent of how far a look-back
 //     reached: outputs are deterministic run to run.
-//   * Tiles are numbered by an atomic ticket (not blockIdx) with the chain as
-//     the fast index, so a tile's predecessor is always a tile whose CTA is
-//     already running; every wait is bounded.
+//   * CTAs are persistent and software-pipelined: tiles are numbered by an
+//     atomic ticket (taken one tile ahead, chain as the fast index, so a
+//     tile's predecessor always belongs to a running CTA), and the TMA loads
+//     of the next tile are in flight while the current one is processed.
+//     Every wait is bounded (iteration cap, then an error status).
 //   * The forward stores the state at every chunk end (fstate); the backward
 //     replays each chunk from that checkpoint, so nothing of size T x C is
 //     stored besides the outputs.
@@ -36,6 +39,7 @@ struct ScanShape {
   int nchunks;          // ceil(T / L)
   int nct;              // channel tiles per batch row
   int nchains;          // B * nct
+  int ntiles;           // nchains * nchunks
   float inv_D;
 };
 
@@ -70,20 +74,33 @@ struct TileCfg {
   static constexpr int VW = VW0 < VPR ? VW0 : VPR; // vectors per warp row segment
   static constexpr int RW = 32 / VW;               // runs per warp
   static constexpr int NVSEG = VPR / VW;
+  static constexpr int LB_WARP = CT / 32 - 1;      // the warp that polls look-back flags
   static constexpr unsigned kBoxBytes = L * CT * sizeof(T);
   static_assert(L % K == 0, "K must divide L");
   static_assert(NT % 32 == 0 && NT <= 1024, "bad block size");
   static_assert(RUNS % RW == 0, "runs must fill warps");
-  static_assert(CT % 32 == 0 && NT >= CT, "look-back needs CT threads");
+  static_assert(CT % 32 == 0 && NT >= CT && CT >= 64, "look-back needs CT threads");
   static_assert(RUNS * CT * sizeof(float2) <= kBoxBytes, "scan scratch must fit in the gate box");
   static_assert(VW % LPH == 0, "a head must stay inside a warp");
+  static_assert(kBoxBytes % 128 == 0, "boxes must keep 128-byte alignment");
 };
 
-template <typename Cfg, int NBOX>
-constexpr size_t scan_smem_bytes() {
-  // NBOX boxes + CT floats + mbarrier + ticket, plus 128 B for alignment.
-  return size_t(NBOX) * Cfg::kBoxBytes + Cfg::CT * sizeof(float) + 16 + 128;
-}
+// Shared-memory plan of the forward kernel: two stages of {a, v, q} boxes.
+template <typename Cfg>
+struct FwdSmem {
+  static constexpr size_t kStage = 3 * size_t(Cfg::kBoxBytes);
+  static constexpr size_t kMisc = Cfg::CT * sizeof(float) + 64;
+  static constexpr size_t kBytes = 2 * kStage + kMisc + 128;   // +128 for alignment
+};
+
+// Backward: two stages of {a, v} boxes plus one {q, dy} pair.
+template <typename Cfg>
+struct BwdSmem {
+  static constexpr size_t kStage = 2 * size_t(Cfg::kBoxBytes);
+  static constexpr size_t kQdy = 2 * size_t(Cfg::kBoxBytes);
+  static constexpr size_t kMisc = Cfg::CT * sizeof(float) + 64;
+  static constexpr size_t kBytes = 2 * kStage + kQdy + kMisc + 128;
+};
 
 __device__ __forceinline__ unsigned char *align128(unsigned char *p) {
   return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(p) + 127) & ~uintptr_t(127));
@@ -93,7 +110,7 @@ __device__ __forceinline__ unsigned char *align128(unsigned char *p) {
 template <typename Cfg>
 struct ThreadPos {
   int vec, run, ch, row0;
-  __device__ __forceinline__ ThreadPos(int tid) {
+  __device__ __forceinline__ explicit ThreadPos(int tid) {
     const int warp = tid >> 5, lane = tid & 31;
     const int vseg = warp % Cfg::NVSEG, rgrp = warp / Cfg::NVSEG;
     vec = vseg * Cfg::VW + lane % Cfg::VW;
@@ -103,437 +120,606 @@ struct ThreadPos {
   }
 };
 
-// Decoupled look-back for one channel (called by the first CT threads).
-// `slot` is this tile; its predecessors in processing order are
-// slot + dir, slot + 2 dir, ...  (dir = -1 forward in time, +1 backward).
-// Returns the carry entering this tile.  The walk stops at the nearest
-// predecessor whose inclusive carry is published, then applies the
-// aggregates of the tiles in between oldest first.
-__device__ __forceinline__ float lookback(const unsigned *flags, const float2 *agg, const float *state,
-                                          long slot, int dir, int CT, int c, unsigned *abort_flag,
-                                          unsigned *status) {
-  long j = slot + dir;
-  for (;;) {
-    const unsigned f = wait_flag_bounded(&flags[j], abort_flag, status);
-    if (f == kFlagIncl) break;
-    if (f == 0) return 0.0f;  // gave up; status already records the timeout
-    j += dir;
+// Run-scan scratch: float2 (map P, S) per (run, channel).  A thread's 8
+// channels form a 64-byte block made of four 16-byte chunks; chunk q of vector
+// `vec` is stored at position (q + vec / 2) mod 4 so that the 16-byte accesses
+// of 8 consecutive vectors hit distinct banks, and the serial scan's 8-byte
+// accesses by consecutive channels stay conflict-free as well.
+template <int CT>
+__device__ __forceinline__ int scan_pos(int run, int c) {
+  const int vec = c >> 3, j = c & 7;
+  const int chunk = ((j >> 1) + (vec >> 1)) & 3;
+  return run * CT + vec * 8 + chunk * 2 + (j & 1);
+}
+
+template <int CT>
+__device__ __forceinline__ void scan_store8(float2 *scan, int run, int ch, const float (&p)[8], const float (&s)[8]) {
+  const int vec = ch >> 3;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int chunk = (q + (vec >> 1)) & 3;
+    reinterpret_cast<float4 *>(scan + run * CT + ch + chunk * 2)[0] =
+        make_float4(p[2 * q], s[2 * q], p[2 * q + 1], s[2 * q + 1]);
   }
+}
+
+template <int CT>
+__device__ __forceinline__ void scan_load8(const float2 *scan, int run, int ch, float (&p)[8], float (&s)[8]) {
+  const int vec = ch >> 3;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int chunk = (q + (vec >> 1)) & 3;
+    const float4 u = reinterpret_cast<const float4 *>(scan + run * CT + ch + chunk * 2)[0];
+    p[2 * q] = u.x;
+    s[2 * q] = u.y;
+    p[2 * q + 1] = u.z;
+    s[2 * q + 1] = u.w;
+  }
+}
+
+// Serial scan over the runs of one channel (threads 0..CT-1).  Replaces each
+// entry by the exclusive prefix and returns the tile map (forward order:
+// oldest run first; backward order: latest run first).
+template <int CT, int RUNS, bool kReverse>
+__device__ __forceinline__ float2 scan_runs(float2 *scan, int c) {
+  float cp = 1.0f, cs = 0.0f;
+#pragma unroll 4
+  for (int k = 0; k < RUNS; ++k) {
+    const int r = kReverse ? RUNS - 1 - k : k;
+    const int at = scan_pos<CT>(r, c);
+    const float2 e = scan[at];
+    scan[at] = make_float2(cp, cs);
+    cs = __fmaf_rn(e.x, cs, e.y);
+    cp = cp * e.x;
+  }
+  return make_float2(cp, cs);
+}
+
+// Called by warp LB_WARP: find the nearest predecessor of `slot` (at
+// distance 1..avail, step `dir`) whose inclusive carry is published, with
+// every tile in between at least aggregate-published.  Returns its slot, or
+// -1 if the bounded wait gave up (status recorded).
+__device__ __forceinline__ long find_inclusive(const unsigned *flags, long slot, int dir, int avail,
+                                               unsigned *abort_flag, unsigned *status) {
+  const int lane = threadIdx.x & 31;
+  int base = 1;
+  unsigned ns = 32;
+  for (unsigned it = 0; it < kSpinLimit; ++it) {
+    const int dist = base + lane;
+    const bool in = dist <= avail;
+    const unsigned f = in ? ld_acquire(&flags[slot + static_cast<long>(dir) * dist]) : 0u;
+    const unsigned incl = __ballot_sync(0xffffffffu, in && f == kFlagIncl);
+    const unsigned missing = __ballot_sync(0xffffffffu, in && f == 0u);
+    if (incl) {
+      const int first = __ffs(incl) - 1;
+      if ((missing & ((1u << first) - 1u)) == 0u) return slot + static_cast<long>(dir) * (base + first);
+    } else if (missing == 0u && base + 31 < avail) {
+      base += 32;   // 32 aggregates in a row: keep walking back
+      continue;
+    }
+    if ((it & 63u) == 63u) {
+      const unsigned ab = (lane == 0) ? ld_relaxed(abort_flag) : 0u;
+      if (__shfl_sync(0xffffffffu, ab, 0)) break;
+    }
+    __nanosleep(ns);
+    ns = ns < 256 ? ns * 2 : 256;
+  }
+  if (lane == 0) {
+    atomicOr(status, kStatusTimeout);
+    atomicExch(abort_flag, 1u);
+  }
+  return -1;
+}
+
+// Apply the aggregates of the tiles strictly between `j` (inclusive carry
+// published) and `slot`, oldest first, to j's carry.  Channel c.
+__device__ __forceinline__ float apply_carries(const float2 *agg, const float *state, long j, long slot, int dir,
+                                               int CT, int c) {
   float E = __ldcg(&state[j * CT + c]);
-  for (long m = j - dir; m != slot; m -= dir) {
+  long m = j - dir;
+  for (; (slot - m) * (-dir) >= 4; m -= 4 * dir) {   // four loads in flight
+    const float2 e0 = __ldcg(&agg[m * CT + c]);
+    const float2 e1 = __ldcg(&agg[(m - dir) * CT + c]);
+    const float2 e2 = __ldcg(&agg[(m - 2 * dir) * CT + c]);
+    const float2 e3 = __ldcg(&agg[(m - 3 * dir) * CT + c]);
+    E = __fmaf_rn(e0.x, E, e0.y);
+    E = __fmaf_rn(e1.x, E, e1.y);
+    E = __fmaf_rn(e2.x, E, e2.y);
+    E = __fmaf_rn(e3.x, E, e3.y);
+  }
+  for (; m != slot; m -= dir) {
     const float2 e = __ldcg(&agg[m * CT + c]);
     E = __fmaf_rn(e.x, E, e.y);
   }
   return E;
 }
 
+// The carry entering tile `slot` (threads 0..CT-1; uses named barrier 1).
+// Publishes the tile's aggregate first.  `avail` = number of predecessors.
+template <typename Cfg>
+__device__ __forceinline__ float lookback_carry(const Workspace &ws, unsigned *flags, unsigned *hdr, float *state,
+                                                long slot, int dir, int avail, float2 tile_map, long *bcast) {
+  const int tid = threadIdx.x;
+  ws.agg[slot * Cfg::CT + tid] = tile_map;
+  bar_sync_first(Cfg::CT);
+  if (tid == 0) {
+    fence_acq_rel_gpu();
+    st_relaxed(&flags[slot], kFlagAgg);
+  }
+  if ((tid >> 5) == Cfg::LB_WARP) {
+    const long j = find_inclusive(flags, slot, dir, avail, &hdr[2], ws.status);
+    if ((tid & 31) == 0) *bcast = j;
+  }
+  bar_sync_first(Cfg::CT);
+  const long j = *bcast;
+  if (j < 0) return 0.0f;
+  return apply_carries(ws.agg, state, j, slot, dir, Cfg::CT, tid);
+}
+
+// Gate of one channel in the form the recurrence uses: direct keeps A,
+// controlled keeps 1 - A (no cancellation when A is close to 1).
+template <int MODE>
+__device__ __forceinline__ float gate_coef(const Gate &g) { return MODE == 0 ? g.A : g.Ac; }
+
+// One step of the recurrence with the stored gate coefficient `c`.
+template <int MODE>
+__device__ __forceinline__ float rec_step(float c, float E, float v) {
+  return MODE == 0 ? __fmaf_rn(c, E, v) : __fmaf_rn(c, v - E, E);
+}
+
 // ===========================================================================
-// Forward scan.
+// Forward scan (persistent).
 // ===========================================================================
 template <typename T, int MODE, int LPH, int VPR, int L, int K>
-__global__ void __launch_bounds__(VPR *(L / K))
+__global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
     esa_scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_q, const FwdArgs args) {
   using Cfg = TileCfg<T, LPH, VPR, L, K>;
+  using Sm = FwdSmem<Cfg>;
   constexpr int CT = Cfg::CT, RUNS = Cfg::RUNS;
 
   extern __shared__ unsigned char smem_raw[];
   unsigned char *base = align128(smem_raw);
-  T *a_s = reinterpret_cast<T *>(base);
-  T *v_s = a_s + L * CT;
-  T *q_s = v_s + L * CT;
-  float *es_s = reinterpret_cast<float *>(q_s + L * CT);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(es_s + CT);
-  int *ticket_s = reinterpret_cast<int *>(bar + 1);
-  float2 *scan_s = reinterpret_cast<float2 *>(a_s);  // reused once pass 1 is done
+  float *es_s = reinterpret_cast<float *>(base + 2 * Sm::kStage);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(es_s + CT);     // [2]
+  int *ticket_s = reinterpret_cast<int *>(bar + 2);            // [2]
+  long *bcast = reinterpret_cast<long *>(ticket_s + 2);
 
   const int tid = threadIdx.x;
   const ScanShape &sh = args.s;
   const Workspace &ws = args.ws;
+  unsigned *hdr = ws.fwd_hdr;
+
+  auto box = [&](int stage, int k) -> T * {
+    return reinterpret_cast<T *>(base + stage * Sm::kStage + k * size_t(Cfg::kBoxBytes));
+  };
+  auto issue = [&](int stage, int tile) {
+    const int chain = tile % sh.nchains, chunk = tile / sh.nchains;
+    const int c0 = (chain % sh.nct) * CT, b = chain / sh.nct, t0 = chunk * L;
+    mbar_expect_tx(&bar[stage], 3 * Cfg::kBoxBytes);
+    tma_load_3d(box(stage, 0), &tm_a, c0, t0, b, &bar[stage]);
+    tma_load_3d(box(stage, 1), &tm_v, c0, t0, b, &bar[stage]);
+    tma_load_3d(box(stage, 2), &tm_q, c0, t0, b, &bar[stage]);
+  };
 
   if (tid == 0) {
     prefetch_tensormap(&tm_a);
     prefetch_tensormap(&tm_v);
     prefetch_tensormap(&tm_q);
-    mbar_init(bar, 1);
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
     fence_mbar_init();
     fence_proxy_async_smem();
-    *ticket_s = static_cast<int>(atomicAdd(&ws.fwd_hdr[1], 1u));
+    const int t0 = static_cast<int>(atomicAdd(&hdr[1], 1u));
+    const int t1 = static_cast<int>(atomicAdd(&hdr[1], 1u));
+    ticket_s[0] = t0;
+    ticket_s[1] = t1;
+    if (t0 < sh.ntiles) issue(0, t0);
+    if (t1 < sh.ntiles) issue(1, t1);
   }
   __syncthreads();
-  const int tile = *ticket_s;
-  const int chain = tile % sh.nchains;
-  const int chunk = tile / sh.nchains;
-  const int b = chain / sh.nct;
-  const int c0 = (chain % sh.nct) * CT;
-  const int t0 = chunk * L;
-  const long slot = static_cast<long>(chain) * sh.nchunks + chunk;
-
-  if (tid == 0) {
-    mbar_expect_tx(bar, 3 * Cfg::kBoxBytes);
-    tma_load_3d(a_s, &tm_a, c0, t0, b, bar);
-    tma_load_3d(v_s, &tm_v, c0, t0, b, bar);
-    tma_load_3d(q_s, &tm_q, c0, t0, b, bar);
-  }
 
   const ThreadPos<Cfg> pos(tid);
-  mbar_wait_bounded(bar, 0, ws.status);
+  T *yg = static_cast<T *>(args.y);
+  unsigned phase = 0;   // bit s = parity of stage s
 
-  // ---- pass 1: gates and the run's affine map -----------------------------
-  float Ar[K][8];   // direct: A_t; controlled: 1 - A_t
-  float P[8], S[8];
+  for (int it = 0;; ++it) {
+    const int s = it & 1;
+    const int tile = ticket_s[s];
+    if (tile >= sh.ntiles) break;
+    unsigned next = 0;
+    if (tid == 0) next = atomicAdd(&hdr[1], 1u);   // the tile that will refill this stage
+
+    const int chain = tile % sh.nchains, chunk = tile / sh.nchains;
+    const int b = chain / sh.nct, c0 = (chain % sh.nct) * CT, t0 = chunk * L;
+    const long slot = static_cast<long>(chain) * sh.nchunks + chunk;
+    const T *a_s = box(s, 0);
+    const T *v_s = box(s, 1);
+    const T *q_s = box(s, 2);
+    float2 *scan_s = reinterpret_cast<float2 *>(box(s, 0));   // reused once pass 1 is done
+
+    mbar_wait_bounded(&bar[s], (phase >> s) & 1u, ws.status);
+    phase ^= 1u << s;
+
+    // ---- pass 1: gates and the run's affine map ---------------------------
+    float Ar[K][8];
+    float P[8], S[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) { P[j] = 1.0f; S[j] = 0.0f; }
+    for (int j = 0; j < 8; ++j) { P[j] = 1.0f; S[j] = 0.0f; }
 #pragma unroll
-  for (int i = 0; i < K; ++i) {
-    const int r = pos.row0 + i;
-    const bool valid = (t0 + r) < sh.T;
-    float x[8], vv[8];
-    Io<T>::load8(a_s + r * CT + pos.ch, x);
-    Io<T>::load8(v_s + r * CT + pos.ch, vv);
+    for (int i = 0; i < K; ++i) {
+      const int r = pos.row0 + i;
+      const bool valid = (t0 + r) < sh.T;
+      float x[8], vv[8];
+      Io<T>::load8(a_s + r * CT + pos.ch, x);
+      Io<T>::load8(v_s + r * CT + pos.ch, vv);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const Gate g = gate_of(x[j]);
-      if (MODE == 0) {
-        Ar[i][j] = g.A;
-        if (valid) { P[j] *= g.A; S[j] = __fmaf_rn(g.A, S[j], vv[j]); }
+      for (int j = 0; j < 8; ++j) {
+        const Gate g = gate_of(x[j]);
+        Ar[i][j] = gate_coef<MODE>(g);
+        if (valid) {
+          P[j] *= g.A;
+          S[j] = rec_step<MODE>(Ar[i][j], S[j], vv[j]);
+        }
+      }
+    }
+    __syncthreads();   // the gate box is free from here on
+    scan_store8<CT>(scan_s, pos.run, pos.ch, P, S);
+    __syncthreads();
+
+    // ---- scan over runs, look-back, publish --------------------------------
+    if (tid < CT) {
+      const float2 tmap = scan_runs<CT, RUNS, false>(scan_s, tid);
+      const int cg = c0 + tid;
+      float E_start;
+      if (chunk == 0) {
+        E_start = (args.E_init != nullptr && cg < sh.C) ? args.E_init[static_cast<long>(b) * sh.C + cg] : 0.0f;
       } else {
-        Ar[i][j] = g.Ac;
-        if (valid) { P[j] *= g.A; S[j] = __fmaf_rn(g.Ac, vv[j] - S[j], S[j]); }
+        E_start = lookback_carry<Cfg>(ws, ws.fwd_flags, hdr, ws.fstate, slot, -1, chunk, tmap, bcast);
+      }
+      const float E_end = __fmaf_rn(tmap.x, E_start, tmap.y);
+      ws.fstate[slot * CT + tid] = E_end;
+      if (chunk == sh.nchunks - 1 && args.E_final != nullptr && cg < sh.C)
+        args.E_final[static_cast<long>(b) * sh.C + cg] = E_end;
+      es_s[tid] = E_start;
+    }
+    __syncthreads();
+    if (tid == 0) {   // publish this chunk's end state
+      fence_acq_rel_gpu();
+      st_relaxed(&ws.fwd_flags[slot], kFlagIncl);
+    }
+
+    // ---- pass 2: exact states and the readout ------------------------------
+    float E[8];
+    {
+      float pe[8], se[8];
+      scan_load8<CT>(scan_s, pos.run, pos.ch, pe, se);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) E[j] = __fmaf_rn(pe[j], es_s[pos.ch + j], se[j]);
+    }
+    const bool ch_ok = (c0 + pos.ch) < sh.C;
+    const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+      const int r = pos.row0 + i;
+      const bool valid = (t0 + r) < sh.T;
+      float vv[8], qq[8];
+      Io<T>::load8(v_s + r * CT + pos.ch, vv);
+      Io<T>::load8(q_s + r * CT + pos.ch, qq);
+      float ss = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        E[j] = rec_step<MODE>(Ar[i][j], E[j], vv[j]);
+        ss = __fmaf_rn(E[j], E[j], ss);
+      }
+      ss = head_sum<LPH>(ss);
+      const float rr = rsqrt_approx(__fmaf_rn(ss, sh.inv_D, kEps));
+      float yv[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) yv[j] = qq[j] * (E[j] * rr);
+      if (valid && ch_ok) Io<T>::store8(yg + gbase + static_cast<long>(r) * sh.C, yv);
+    }
+
+    // ---- refill this stage --------------------------------------------------
+    __syncthreads();   // everybody is done with stage s
+    if (tid == 0) {
+      ticket_s[s] = static_cast<int>(next);
+      if (static_cast<int>(next) < sh.ntiles) {
+        fence_proxy_async_smem();   // generic writes (scan scratch) before the async refill
+        issue(s, static_cast<int>(next));
       }
     }
   }
-  __syncthreads();  // the gate box is free from here on
-#pragma unroll
-  for (int j = 0; j < 8; ++j) scan_s[pos.run * CT + pos.ch + j] = make_float2(P[j], S[j]);
-  __syncthreads();
-
-  // ---- scan over runs, look-back, publish --------------------------------
-  if (tid < CT) {
-    float cp = 1.0f, cs = 0.0f;
-#pragma unroll 4
-    for (int r = 0; r < RUNS; ++r) {
-      const float2 e = scan_s[r * CT + tid];
-      scan_s[r * CT + tid] = make_float2(cp, cs);   // exclusive prefix of the runs
-      cs = __fmaf_rn(e.x, cs, e.y);
-      cp = cp * e.x;
-    }
-    const int cg = c0 + tid;
-    float E_start;
-    if (chunk == 0) {
-      E_start = (args.E_init != nullptr && cg < sh.C) ? args.E_init[static_cast<long>(b) * sh.C + cg] : 0.0f;
-    } else {
-      ws.agg[slot * CT + tid] = make_float2(cp, cs);
-      __threadfence();
-      bar_sync_first(CT);
-      if (tid == 0) st_release(&ws.fwd_flags[slot], kFlagAgg);
-      E_start = lookback(ws.fwd_flags, ws.agg, ws.fstate, slot, -1, CT, tid, &ws.fwd_hdr[2], ws.status);
-    }
-    const float E_end = __fmaf_rn(cp, E_start, cs);
-    ws.fstate[slot * CT + tid] = E_end;
-    __threadfence();
-    bar_sync_first(CT);
-    if (tid == 0) st_release(&ws.fwd_flags[slot], kFlagIncl);
-    if (chunk == sh.nchunks - 1 && args.E_final != nullptr && cg < sh.C)
-      args.E_final[static_cast<long>(b) * sh.C + cg] = E_end;
-    es_s[tid] = E_start;
-  }
-  __syncthreads();
-
-  // ---- pass 2: exact states and the readout ------------------------------
-  float E[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float2 pe = scan_s[pos.run * CT + pos.ch + j];
-    E[j] = __fmaf_rn(pe.x, es_s[pos.ch + j], pe.y);
-  }
-  T *yg = static_cast<T *>(args.y);
-  const bool ch_ok = (c0 + pos.ch) < sh.C;
-  const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
-#pragma unroll
-  for (int i = 0; i < K; ++i) {
-    const int r = pos.row0 + i;
-    const bool valid = (t0 + r) < sh.T;
-    float vv[8], qq[8];
-    Io<T>::load8(v_s + r * CT + pos.ch, vv);
-    Io<T>::load8(q_s + r * CT + pos.ch, qq);
-    float ss = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      E[j] = (MODE == 0) ? __fmaf_rn(Ar[i][j], E[j], vv[j]) : __fmaf_rn(Ar[i][j], vv[j] - E[j], E[j]);
-      ss = __fmaf_rn(E[j], E[j], ss);
-    }
-    ss = head_sum<LPH>(ss);
-    const float rr = rsqrtf(__fmaf_rn(ss, sh.inv_D, kEps));
-    float yv[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) yv[j] = qq[j] * (E[j] * rr);
-    if (valid && ch_ok) Io<T>::store8(yg + gbase + static_cast<long>(r) * sh.C, yv);
-  }
 }
 
 // ===========================================================================
-// Backward scan.
+// Backward scan (persistent).
 // ===========================================================================
-template <typename T>
-__device__ __forceinline__ void put_ghat(T *q_slot, T *dy_slot, const float (&g)[8]) {
-  if (sizeof(T) == 2) {
-    reinterpret_cast<float4 *>(q_slot)[0] = make_float4(g[0], g[1], g[2], g[3]);
-    reinterpret_cast<float4 *>(dy_slot)[0] = make_float4(g[4], g[5], g[6], g[7]);
-  } else {
-    reinterpret_cast<float4 *>(q_slot)[0] = make_float4(g[0], g[1], g[2], g[3]);
-    reinterpret_cast<float4 *>(q_slot)[1] = make_float4(g[4], g[5], g[6], g[7]);
-  }
-}
-
-template <typename T>
-__device__ __forceinline__ void get_ghat(const T *q_slot, const T *dy_slot, float (&g)[8]) {
-  float4 u, w;
-  if (sizeof(T) == 2) {
-    u = reinterpret_cast<const float4 *>(q_slot)[0];
-    w = reinterpret_cast<const float4 *>(dy_slot)[0];
-  } else {
-    u = reinterpret_cast<const float4 *>(q_slot)[0];
-    w = reinterpret_cast<const float4 *>(q_slot)[1];
-  }
-  g[0] = u.x; g[1] = u.y; g[2] = u.z; g[3] = u.w;
-  g[4] = w.x; g[5] = w.y; g[6] = w.z; g[7] = w.w;
-}
-
+// Two CTAs per SM when the block has at most 256 threads (the smem plan fits).
 template <typename T, int MODE, int LPH, int VPR, int L, int K>
-__global__ void __launch_bounds__(VPR *(L / K))
+__global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
     esa_scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dy,
                         const BwdArgs args) {
   using Cfg = TileCfg<T, LPH, VPR, L, K>;
+  using Sm = BwdSmem<Cfg>;
   constexpr int CT = Cfg::CT, RUNS = Cfg::RUNS;
 
   extern __shared__ unsigned char smem_raw[];
   unsigned char *base = align128(smem_raw);
-  T *a_s = reinterpret_cast<T *>(base);
-  T *v_s = a_s + L * CT;
-  T *q_s = v_s + L * CT;
+  T *q_s = reinterpret_cast<T *>(base + 2 * Sm::kStage);
   T *dy_s = q_s + L * CT;
-  float *es_s = reinterpret_cast<float *>(dy_s + L * CT);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(es_s + CT);
-  int *ticket_s = reinterpret_cast<int *>(bar + 1);
-  float2 *scan_s = reinterpret_cast<float2 *>(a_s);
+  float *es_s = reinterpret_cast<float *>(base + 2 * Sm::kStage + Sm::kQdy);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(es_s + CT);     // [0..1] a/v stages, [2] q/dy
+  int *ticket_s = reinterpret_cast<int *>(bar + 3);            // [2]
+  long *bcast = reinterpret_cast<long *>(ticket_s + 2);
 
   const int tid = threadIdx.x;
   const ScanShape &sh = args.s;
   const Workspace &ws = args.ws;
+  unsigned *hdr = ws.bwd_hdr;
+
+  auto box = [&](int stage, int k) -> T * {
+    return reinterpret_cast<T *>(base + stage * Sm::kStage + k * size_t(Cfg::kBoxBytes));
+  };
+  auto coords = [&](int tile, int &c0, int &t0, int &b) {
+    const int chain = tile % sh.nchains;
+    const int chunk = sh.nchunks - 1 - tile / sh.nchains;   // latest chunk first
+    c0 = (chain % sh.nct) * CT;
+    b = chain / sh.nct;
+    t0 = chunk * L;
+  };
+  auto issue_av = [&](int stage, int tile) {
+    int c0, t0, b;
+    coords(tile, c0, t0, b);
+    mbar_expect_tx(&bar[stage], 2 * Cfg::kBoxBytes);
+    tma_load_3d(box(stage, 0), &tm_a, c0, t0, b, &bar[stage]);
+    tma_load_3d(box(stage, 1), &tm_v, c0, t0, b, &bar[stage]);
+  };
+  auto issue_qdy = [&](int tile) {
+    int c0, t0, b;
+    coords(tile, c0, t0, b);
+    mbar_expect_tx(&bar[2], 2 * Cfg::kBoxBytes);
+    tma_load_3d(q_s, &tm_q, c0, t0, b, &bar[2]);
+    tma_load_3d(dy_s, &tm_dy, c0, t0, b, &bar[2]);
+  };
 
   if (tid == 0) {
     prefetch_tensormap(&tm_a);
     prefetch_tensormap(&tm_v);
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_dy);
-    mbar_init(bar, 1);
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_init(&bar[2], 1);
     fence_mbar_init();
     fence_proxy_async_smem();
-    *ticket_s = static_cast<int>(atomicAdd(&ws.bwd_hdr[1], 1u));
+    const int t0 = static_cast<int>(atomicAdd(&hdr[1], 1u));
+    const int t1 = static_cast<int>(atomicAdd(&hdr[1], 1u));
+    ticket_s[0] = t0;
+    ticket_s[1] = t1;
+    if (t0 < sh.ntiles) {
+      issue_av(0, t0);
+      issue_qdy(t0);
+    }
+    if (t1 < sh.ntiles) issue_av(1, t1);
   }
   __syncthreads();
-  const int tile = *ticket_s;
-  const int chain = tile % sh.nchains;
-  const int chunk = sh.nchunks - 1 - tile / sh.nchains;   // latest chunk first
-  const int b = chain / sh.nct;
-  const int c0 = (chain % sh.nct) * CT;
-  const int t0 = chunk * L;
-  const long slot = static_cast<long>(chain) * sh.nchunks + chunk;
-
-  if (tid == 0) {
-    mbar_expect_tx(bar, 4 * Cfg::kBoxBytes);
-    tma_load_3d(a_s, &tm_a, c0, t0, b, bar);
-    tma_load_3d(v_s, &tm_v, c0, t0, b, bar);
-    tma_load_3d(q_s, &tm_q, c0, t0, b, bar);
-    tma_load_3d(dy_s, &tm_dy, c0, t0, b, bar);
-  }
-  if (tid < CT) {   // forward state entering the chunk (checkpoint)
-    const int cg = c0 + tid;
-    es_s[tid] = (chunk == 0)
-                    ? ((args.E_init != nullptr && cg < sh.C) ? args.E_init[static_cast<long>(b) * sh.C + cg] : 0.0f)
-                    : __ldcg(&ws.fstate[(slot - 1) * CT + tid]);
-  }
 
   const ThreadPos<Cfg> pos(tid);
-  mbar_wait_bounded(bar, 0, ws.status);
-
-  // ---- F1: gates and the run's forward map --------------------------------
-  float Ar[K][8];
-  float P[8], S[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) { P[j] = 1.0f; S[j] = 0.0f; }
-#pragma unroll
-  for (int i = 0; i < K; ++i) {
-    const int r = pos.row0 + i;
-    const bool valid = (t0 + r) < sh.T;
-    float x[8], vv[8];
-    Io<T>::load8(a_s + r * CT + pos.ch, x);
-    Io<T>::load8(v_s + r * CT + pos.ch, vv);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const Gate g = gate_of(x[j]);
-      if (MODE == 0) {
-        Ar[i][j] = g.A;
-        if (valid) { P[j] *= g.A; S[j] = __fmaf_rn(g.A, S[j], vv[j]); }
-      } else {
-        Ar[i][j] = g.Ac;
-        if (valid) { P[j] *= g.A; S[j] = __fmaf_rn(g.Ac, vv[j] - S[j], S[j]); }
-      }
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int j = 0; j < 8; ++j) scan_s[pos.run * CT + pos.ch + j] = make_float2(P[j], S[j]);
-  __syncthreads();
-  if (tid < CT) {
-    float cp = 1.0f, cs = 0.0f;
-#pragma unroll 4
-    for (int r = 0; r < RUNS; ++r) {
-      const float2 e = scan_s[r * CT + tid];
-      scan_s[r * CT + tid] = make_float2(cp, cs);
-      cs = __fmaf_rn(e.x, cs, e.y);
-      cp = cp * e.x;
-    }
-  }
-  __syncthreads();
-
-  // ---- F2: replay states, readout backward, dq, ghat ----------------------
-  float E[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float2 pe = scan_s[pos.run * CT + pos.ch + j];
-    E[j] = __fmaf_rn(pe.x, es_s[pos.ch + j], pe.y);
-  }
-  float Ep[K][8];   // E_{t-1} of every row of the run
-  const bool ch_ok = (c0 + pos.ch) < sh.C;
-  const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
-  T *dqg = static_cast<T *>(args.dq);
-#pragma unroll
-  for (int i = 0; i < K; ++i) {
-    const int r = pos.row0 + i;
-    const bool valid = (t0 + r) < sh.T;
-    float vv[8], qq[8], gg[8];
-    Io<T>::load8(v_s + r * CT + pos.ch, vv);
-    Io<T>::load8(q_s + r * CT + pos.ch, qq);
-    Io<T>::load8(dy_s + r * CT + pos.ch, gg);
-    float ss = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      Ep[i][j] = E[j];
-      E[j] = (MODE == 0) ? __fmaf_rn(Ar[i][j], E[j], vv[j]) : __fmaf_rn(Ar[i][j], vv[j] - E[j], E[j]);
-      ss = __fmaf_rn(E[j], E[j], ss);
-    }
-    ss = head_sum<LPH>(ss);
-    const float rr = rsqrtf(__fmaf_rn(ss, sh.inv_D, kEps));
-    float nn[8], dn[8], dqv[8];
-    float dot = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      nn[j] = E[j] * rr;
-      dn[j] = gg[j] * qq[j];
-      dqv[j] = gg[j] * nn[j];
-      dot = __fmaf_rn(dn[j], nn[j], dot);
-    }
-    dot = head_sum<LPH>(dot) * sh.inv_D;
-    float gh[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) gh[j] = rr * __fmaf_rn(-nn[j], dot, dn[j]);
-    put_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
-    if (valid && ch_ok) Io<T>::store8(dqg + gbase + static_cast<long>(r) * sh.C, dqv);
-  }
-
-  // ---- R1: the run's reverse map h -> P h + hl ---------------------------
-  float hl[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) hl[j] = 0.0f;
-#pragma unroll
-  for (int i = K - 1; i >= 0; --i) {
-    const int r = pos.row0 + i;
-    if ((t0 + r) < sh.T) {
-      float gh[8];
-      get_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float A = (MODE == 0) ? Ar[i][j] : 1.0f - Ar[i][j];
-        hl[j] = A * (gh[j] + hl[j]);
-      }
-    }
-  }
-  __syncthreads();   // everybody is done with the forward prefixes
-#pragma unroll
-  for (int j = 0; j < 8; ++j) scan_s[pos.run * CT + pos.ch + j] = make_float2(P[j], hl[j]);
-  __syncthreads();
-
-  // ---- reverse scan over runs, look-back towards later chunks -------------
-  if (tid < CT) {
-    float cq = 1.0f, cr = 0.0f;   // run's incoming carry = cq * H_in + cr
-#pragma unroll 4
-    for (int r = RUNS - 1; r >= 0; --r) {
-      const float2 e = scan_s[r * CT + tid];
-      scan_s[r * CT + tid] = make_float2(cq, cr);
-      cr = __fmaf_rn(e.x, cr, e.y);
-      cq = e.x * cq;
-    }
-    const int cg = c0 + tid;
-    float H_in;
-    if (chunk == sh.nchunks - 1) {
-      H_in = (args.dE_final != nullptr && cg < sh.C) ? args.dE_final[static_cast<long>(b) * sh.C + cg] : 0.0f;
-    } else {
-      ws.agg[slot * CT + tid] = make_float2(cq, cr);
-      __threadfence();
-      bar_sync_first(CT);
-      if (tid == 0) st_release(&ws.bwd_flags[slot], kFlagAgg);
-      H_in = lookback(ws.bwd_flags, ws.agg, ws.bstate, slot, +1, CT, tid, &ws.bwd_hdr[2], ws.status);
-    }
-    const float H_out = __fmaf_rn(cq, H_in, cr);
-    ws.bstate[slot * CT + tid] = H_out;
-    __threadfence();
-    bar_sync_first(CT);
-    if (tid == 0) st_release(&ws.bwd_flags[slot], kFlagIncl);
-    if (chunk == 0 && args.dE_init != nullptr && cg < sh.C)
-      args.dE_init[static_cast<long>(b) * sh.C + cg] = H_out;
-    es_s[tid] = H_in;
-  }
-  __syncthreads();
-
-  // ---- B: gradients, latest step first ------------------------------------
-  float h[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float2 qr = scan_s[pos.run * CT + pos.ch + j];
-    h[j] = __fmaf_rn(qr.x, es_s[pos.ch + j], qr.y);
-  }
   T *dag = static_cast<T *>(args.da);
   T *dvg = static_cast<T *>(args.dv);
+  T *dqg = static_cast<T *>(args.dq);
+  unsigned phase = 0;   // bits 0..1: a/v stages, bit 2: q/dy
+
+  for (int it = 0;; ++it) {
+    const int s = it & 1;
+    const int tile = ticket_s[s];
+    if (tile >= sh.ntiles) break;
+    unsigned next = 0;
+    if (tid == 0) next = atomicAdd(&hdr[1], 1u);
+
+    const int chain = tile % sh.nchains;
+    const int chunk = sh.nchunks - 1 - tile / sh.nchains;
+    const int b = chain / sh.nct, c0 = (chain % sh.nct) * CT, t0 = chunk * L;
+    const long slot = static_cast<long>(chain) * sh.nchunks + chunk;
+    const T *a_s = box(s, 0);
+    const T *v_s = box(s, 1);
+    float2 *scan_s = reinterpret_cast<float2 *>(box(s, 0));
+
+    float E_ck = 0.0f;   // forward state entering the chunk, channel tid (checkpoint)
+    if (tid < CT) {
+      const int cg = c0 + tid;
+      E_ck = (chunk == 0) ? ((args.E_init != nullptr && cg < sh.C) ? args.E_init[static_cast<long>(b) * sh.C + cg]
+                                                                   : 0.0f)
+                          : __ldcg(&ws.fstate[(slot - 1) * CT + tid]);
+    }
+
+    mbar_wait_bounded(&bar[s], (phase >> s) & 1u, ws.status);
+    phase ^= 1u << s;
+
+    // ---- F1: gates and the run's forward map ------------------------------
+    float Ar[K][8];
+    float P[8], S[8];
 #pragma unroll
-  for (int i = K - 1; i >= 0; --i) {
-    const int r = pos.row0 + i;
-    if ((t0 + r) < sh.T) {
-      float gh[8], vv[8], dav[8], dvv[8];
-      get_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
-      if (MODE == 1) Io<T>::load8(v_s + r * CT + pos.ch, vv);
+    for (int j = 0; j < 8; ++j) { P[j] = 1.0f; S[j] = 0.0f; }
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+      const int r = pos.row0 + i;
+      const bool valid = (t0 + r) < sh.T;
+      float x[8], vv[8];
+      Io<T>::load8(a_s + r * CT + pos.ch, x);
+      Io<T>::load8(v_s + r * CT + pos.ch, vv);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float G = gh[j] + h[j];
-        if (MODE == 0) {
-          const float A = Ar[i][j];
-          dvv[j] = G;
-          dav[j] = G * Ep[i][j] * (A * (1.0f - A));
-          h[j] = A * G;
-        } else {
-          const float Ac = Ar[i][j];
-          const float A = 1.0f - Ac;
-          dvv[j] = G * Ac;
-          dav[j] = G * (Ep[i][j] - vv[j]) * (A * Ac);
-          h[j] = A * G;
+        const Gate g = gate_of(x[j]);
+        Ar[i][j] = gate_coef<MODE>(g);
+        if (valid) {
+          P[j] *= g.A;
+          S[j] = rec_step<MODE>(Ar[i][j], S[j], vv[j]);
         }
       }
-      if (ch_ok) {
-        const long off = gbase + static_cast<long>(r) * sh.C;
-        Io<T>::store8(dag + off, dav);
-        Io<T>::store8(dvg + off, dvv);
+    }
+    __syncthreads();
+    scan_store8<CT>(scan_s, pos.run, pos.ch, P, S);
+    if (tid < CT) es_s[tid] = E_ck;
+    __syncthreads();
+    if (tid < CT) scan_runs<CT, RUNS, false>(scan_s, tid);
+    __syncthreads();
+
+    // ---- F2: replay states, readout backward, dq, ghat ---------------------
+    float Ec[8];   // the run's forward carry-in
+    {
+      float pe[8], se[8];
+      scan_load8<CT>(scan_s, pos.run, pos.ch, pe, se);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) Ec[j] = __fmaf_rn(pe[j], es_s[pos.ch + j], se[j]);
+    }
+    mbar_wait_bounded(&bar[2], (phase >> 2) & 1u, ws.status);
+    phase ^= 4u;
+    float gh[K][8];
+    const bool ch_ok = (c0 + pos.ch) < sh.C;
+    const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
+    {
+      float E[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) E[j] = Ec[j];
+#pragma unroll
+      for (int i = 0; i < K; ++i) {
+        const int r = pos.row0 + i;
+        const bool valid = (t0 + r) < sh.T;
+        float vv[8], qq[8], gg[8];
+        Io<T>::load8(v_s + r * CT + pos.ch, vv);
+        Io<T>::load8(q_s + r * CT + pos.ch, qq);
+        Io<T>::load8(dy_s + r * CT + pos.ch, gg);
+        float ss = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          E[j] = rec_step<MODE>(Ar[i][j], E[j], vv[j]);
+          ss = __fmaf_rn(E[j], E[j], ss);
+        }
+        ss = head_sum<LPH>(ss);
+        const float rr = rsqrt_approx(__fmaf_rn(ss, sh.inv_D, kEps));
+        float nn[8], dn[8], dqv[8];
+        float dot = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          nn[j] = E[j] * rr;
+          dn[j] = gg[j] * qq[j];
+          dqv[j] = gg[j] * nn[j];
+          dot = __fmaf_rn(dn[j], nn[j], dot);
+        }
+        dot = head_sum<LPH>(dot) * sh.inv_D;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) gh[i][j] = rr * __fmaf_rn(-nn[j], dot, dn[j]);
+        if (valid && ch_ok) Io<T>::store8(dqg + gbase + static_cast<long>(r) * sh.C, dqv);
+      }
+    }
+    __syncthreads();   // q/dy box and the forward prefixes are free
+    if (tid == 0 && ticket_s[s ^ 1] < sh.ntiles) issue_qdy(ticket_s[s ^ 1]);
+
+    // ---- R1: the run's reverse map h -> P h + hl ----------------------------
+    {
+      float hl[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) hl[j] = 0.0f;
+#pragma unroll
+      for (int i = K - 1; i >= 0; --i) {
+        if ((t0 + pos.row0 + i) < sh.T) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float A = (MODE == 0) ? Ar[i][j] : 1.0f - Ar[i][j];
+            hl[j] = A * (gh[i][j] + hl[j]);
+          }
+        }
+      }
+      scan_store8<CT>(scan_s, pos.run, pos.ch, P, hl);
+    }
+    __syncthreads();
+
+    // ---- reverse scan over runs, look-back towards later chunks -------------
+    if (tid < CT) {
+      const float2 tmap = scan_runs<CT, RUNS, true>(scan_s, tid);
+      const int cg = c0 + tid;
+      float H_in;
+      if (chunk == sh.nchunks - 1) {
+        H_in = (args.dE_final != nullptr && cg < sh.C) ? args.dE_final[static_cast<long>(b) * sh.C + cg] : 0.0f;
+      } else {
+        H_in = lookback_carry<Cfg>(ws, ws.bwd_flags, hdr, ws.bstate, slot, +1, sh.nchunks - 1 - chunk, tmap,
+                                   bcast);
+      }
+      const float H_out = __fmaf_rn(tmap.x, H_in, tmap.y);
+      ws.bstate[slot * CT + tid] = H_out;
+      if (chunk == 0 && args.dE_init != nullptr && cg < sh.C)
+        args.dE_init[static_cast<long>(b) * sh.C + cg] = H_out;
+      es_s[tid] = H_in;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      fence_acq_rel_gpu();
+      st_relaxed(&ws.bwd_flags[slot], kFlagIncl);
+    }
+
+    // ---- B1: total gradient G_t, latest step first ---------------------------
+    {
+      float h[8];
+      float pe[8], se[8];
+      scan_load8<CT>(scan_s, pos.run, pos.ch, pe, se);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) h[j] = __fmaf_rn(pe[j], es_s[pos.ch + j], se[j]);
+#pragma unroll
+      for (int i = K - 1; i >= 0; --i) {
+        if ((t0 + pos.row0 + i) < sh.T) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float A = (MODE == 0) ? Ar[i][j] : 1.0f - Ar[i][j];
+            const float G = gh[i][j] + h[j];
+            gh[i][j] = G;
+            h[j] = A * G;
+          }
+        }
+      }
+    }
+
+    // ---- B2: replay states forward, emit da and dv ---------------------------
+    {
+      float E[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) E[j] = Ec[j];
+#pragma unroll
+      for (int i = 0; i < K; ++i) {
+        const int r = pos.row0 + i;
+        float vv[8], dav[8], dvv[8];
+        Io<T>::load8(v_s + r * CT + pos.ch, vv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float G = gh[i][j];
+          if (MODE == 0) {
+            const float A = Ar[i][j];
+            dvv[j] = G;
+            dav[j] = G * E[j] * (A * (1.0f - A));
+          } else {
+            const float Ac = Ar[i][j];
+            dvv[j] = G * Ac;
+            dav[j] = G * (E[j] - vv[j]) * ((1.0f - Ac) * Ac);
+          }
+          E[j] = rec_step<MODE>(Ar[i][j], E[j], vv[j]);
+        }
+        if ((t0 + r) < sh.T && ch_ok) {
+          const long off = gbase + static_cast<long>(r) * sh.C;
+          Io<T>::store8(dag + off, dav);
+          Io<T>::store8(dvg + off, dvv);
+        }
+      }
+    }
+
+    // ---- refill this a/v stage ----------------------------------------------
+    __syncthreads();
+    if (tid == 0) {
+      ticket_s[s] = static_cast<int>(next);
+      if (static_cast<int>(next) < sh.ntiles) {
+        fence_proxy_async_smem();
+        issue_av(s, static_cast<int>(next));
       }
     }
   }
@@ -542,11 +728,6 @@ __global__ void __launch_bounds__(VPR *(L / K))
 // ===========================================================================
 // One-token decode step: one thread per 8 channels of one (b, h).
 // ===========================================================================
-template <typename T>
-__device__ __forceinline__ void load8_global(const T *p, float (&x)[8]) {
-  Io<T>::load8(p, x);
-}
-
 template <typename T, int MODE, int LPH>
 __global__ void __launch_bounds__(256)
     esa_step_kernel(const T *__restrict__ a, const T *__restrict__ v, const T *__restrict__ q,
@@ -555,9 +736,9 @@ __global__ void __launch_bounds__(256)
   const bool act = idx < nvec;
   float x[8], vv[8], qq[8], e[8];
   if (act) {
-    load8_global(a + idx * 8, x);
-    load8_global(v + idx * 8, vv);
-    load8_global(q + idx * 8, qq);
+    Io<T>::load8(a + idx * 8, x);
+    Io<T>::load8(v + idx * 8, vv);
+    Io<T>::load8(q + idx * 8, qq);
     Io<float>::load8(E + idx * 8, e);
   } else {
 #pragma unroll
@@ -567,11 +748,11 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const Gate g = gate_of(x[j]);
-    e[j] = (MODE == 0) ? __fmaf_rn(g.A, e[j], vv[j]) : __fmaf_rn(g.Ac, vv[j] - e[j], e[j]);
+    e[j] = rec_step<MODE>(gate_coef<MODE>(g), e[j], vv[j]);
     ss = __fmaf_rn(e[j], e[j], ss);
   }
   ss = head_sum<LPH>(ss);
-  const float rr = rsqrtf(__fmaf_rn(ss, inv_D, kEps));
+  const float rr = rsqrt_approx(__fmaf_rn(ss, inv_D, kEps));
   float yv[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) yv[j] = qq[j] * (e[j] * rr);
