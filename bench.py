@@ -55,16 +55,20 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="run a smaller batch of the same workload (profiling cases only)")
+    ap.add_argument("--seq", type=int, default=None,
+                    help="run a shorter sequence of the same workload (profiling cases only)")
     return ap.parse_args(argv)
 
 
-def workload(batch=None):
+def workload(batch=None, seq=None):
     import dataclasses
 
     from gated_linear_recurrence_b200 import inputs
     w = inputs.WORKLOADS[WORKLOAD_NAME]
     if batch is not None and batch != w.B:
         w = dataclasses.replace(w, B=int(batch), name=f"{w.name} (batch reduced to {batch})")
+    if seq is not None and seq != w.T:
+        w = dataclasses.replace(w, T=int(seq), name=f"{w.name} (sequence reduced to {seq})")
     return w
 
 
@@ -72,7 +76,8 @@ def config_dict(w):
     return {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "D": w.D, "C": w.C,
             "mode": "controlled" if w.mode == 1 else "direct", "io_dtype": w.dtype, "state_dtype": "f32",
             "gate_logit_mean": w.a_mean, "step": "esa_scan_fwd + esa_scan_bwd",
-            "l2": "inputs larger than L2 (4.3 GB read per step vs 126 MB L2); no flush"}
+            "l2": f"inputs larger than L2 ({4 * w.B * w.T * w.C * 2 / 1e9:.2f} GB read per step vs 126 MB L2); "
+                  "no flush"}
 
 
 def measured_peak():
@@ -207,7 +212,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = workload(args.batch)
+    w = workload(args.batch, args.seq)
     rows, T = 1, 16384
     for i in range(args.warmup):
         oracle_sample_seconds(w, rows, T, seed=1000 + i)
@@ -258,7 +263,7 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    w = workload(args.batch)
+    w = workload(args.batch, args.seq)
     B, T, H, D, mode = w.B, w.T, w.H, w.D, w.mode
     x = inputs.make_scan_inputs(B, T, H, D, w.dtype, w.a_mean, w.seed + 17 * rank, device=dev)
     a, v, q, dy = x["a"], x["v"], x["q"], x["dy"]

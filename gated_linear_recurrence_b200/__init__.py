@@ -16,6 +16,7 @@ from .esa import (  # noqa: F401
     esa_step,
     esa_strerror,
     esa_version,
+    esa_workspace_init,
     esa_workspace_size,
     load_library,
     new_workspace,
@@ -23,5 +24,5 @@ from .esa import (  # noqa: F401
 
 __all__ = [
     "CONTROLLED", "DIRECT", "EsaError", "LIB_PATH", "esa_check", "esa_scan_bwd", "esa_scan_fwd",
-    "esa_step", "esa_strerror", "esa_version", "esa_workspace_size", "load_library", "new_workspace",
+    "esa_step", "esa_strerror", "esa_version", "esa_workspace_init", "esa_workspace_size", "load_library", "new_workspace",
 ]

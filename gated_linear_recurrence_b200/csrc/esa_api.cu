@@ -8,6 +8,7 @@
 #include <atomic>
 #include <climits>
 #include <cstdint>
+#include <cstddef>
 #include <cstring>
 #include <mutex>
 
@@ -32,21 +33,19 @@ size_t elem_bytes(int dtype) { return dtype == ESA_F32 ? 4 : 2; }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Workspace layout (byte offsets from the workspace base):
-//   [0, 4)            device status word (sticky until esa_check)
-//   [16, 32)          forward header: [1] tile ticket, [2] abort flag
-//   [32, 32+4n)       forward per-tile flags
-//   bwd               backward header (16 B) + per-tile flags
-//   agg               n * CT float2   per-tile affine carry maps
-//   fstate            n * CT float    forward state at each chunk end
-//   bstate            n * CT float    backward carry at each chunk start
-// with n = B * ceil(C / CT) * ceil(T / L) tiles.
+//   [0, 256)     header (esa::WsHeader: magic, epoch, status, per-kernel
+//                ticket / done / abort words)
+//   incl_f       n * CT  u64   forward chunk-end states (epoch-tagged)
+//   incl_b       n * CT  u64   backward chunk carries (epoch-tagged)
+//   agg          n * CT  2*u64 chunk maps (P, S), each word epoch-tagged
+// with n = B * ceil(C / CT) * ceil(T / L) chunks.
 struct Layout {
   int L = 0, CT = 0, nct = 0, nchunks = 0, nchains = 0;
   long long ntiles = 0;
-  size_t fwd_bytes = 0;   // bytes cleared before each forward (status + header + flags)
-  size_t bwd_off = 0, bwd_bytes = 0;
-  size_t agg_off = 0, fstate_off = 0, bstate_off = 0, total = 0;
+  size_t incl_f_off = 0, incl_b_off = 0, agg_off = 0, total = 0;
 };
+
+constexpr size_t kHeaderBytes = 256;
 
 bool make_layout(int B, int T, int H, int D, int dtype, Layout *lo) {
   if (B < 0 || T < 0 || H < 1 || D < 1) return false;
@@ -63,18 +62,14 @@ bool make_layout(int B, int T, int H, int D, int dtype, Layout *lo) {
   lo->nchains = static_cast<int>(nchains);
   lo->ntiles = nchains * lo->nchunks;
   if (lo->ntiles > INT_MAX) return false;
-  const size_t n = static_cast<size_t>(lo->ntiles);
-  lo->fwd_bytes = 32 + 4 * n;
-  size_t off = align_up(lo->fwd_bytes, 256);
-  lo->bwd_off = off;
-  lo->bwd_bytes = 16 + 4 * n;
-  off = align_up(off + lo->bwd_bytes, 256);
+  const size_t words = static_cast<size_t>(lo->ntiles) * lo->CT;
+  size_t off = kHeaderBytes;
+  lo->incl_f_off = off;
+  off = align_up(off + words * sizeof(unsigned long long), 256);
+  lo->incl_b_off = off;
+  off = align_up(off + words * sizeof(unsigned long long), 256);
   lo->agg_off = off;
-  off = align_up(off + n * lo->CT * sizeof(float2), 256);
-  lo->fstate_off = off;
-  off = align_up(off + n * lo->CT * sizeof(float), 256);
-  lo->bstate_off = off;
-  off = align_up(off + n * lo->CT * sizeof(float), 256);
+  off = align_up(off + words * sizeof(ulonglong2), 256);
   lo->total = off;
   return true;
 }
@@ -82,14 +77,10 @@ bool make_layout(int B, int T, int H, int D, int dtype, Layout *lo) {
 esa::Workspace workspace_view(void *base, const Layout &lo) {
   unsigned char *p = static_cast<unsigned char *>(base);
   esa::Workspace ws;
-  ws.status = reinterpret_cast<unsigned *>(p);
-  ws.fwd_hdr = reinterpret_cast<unsigned *>(p + 16);
-  ws.fwd_flags = reinterpret_cast<unsigned *>(p + 32);
-  ws.bwd_hdr = reinterpret_cast<unsigned *>(p + lo.bwd_off);
-  ws.bwd_flags = reinterpret_cast<unsigned *>(p + lo.bwd_off + 16);
-  ws.agg = reinterpret_cast<float2 *>(p + lo.agg_off);
-  ws.fstate = reinterpret_cast<float *>(p + lo.fstate_off);
-  ws.bstate = reinterpret_cast<float *>(p + lo.bstate_off);
+  ws.hdr = reinterpret_cast<esa::WsHeader *>(p);
+  ws.incl_f = reinterpret_cast<unsigned long long *>(p + lo.incl_f_off);
+  ws.incl_b = reinterpret_cast<unsigned long long *>(p + lo.incl_b_off);
+  ws.agg = reinterpret_cast<ulonglong2 *>(p + lo.agg_off);
   return ws;
 }
 
@@ -217,7 +208,6 @@ int esa_scan_fwd(const void *a, const void *v, const void *q, void *y, float *E_
   if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo))) return rc;
   if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo))) return rc;
   if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo))) return rc;
-  if ((rc = rt(cudaMemsetAsync(workspace, 0, lo.fwd_bytes, st)))) return rc;
   esa::FwdArgs args;
   args.s = scan_shape(B, T, H, D, lo);
   args.y = y;
@@ -257,8 +247,6 @@ int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy, co
   if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo))) return rc;
   if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo))) return rc;
   if ((rc = make_tmap(&tdy, dy, dtype, B, T, C, lo))) return rc;
-  unsigned char *base = static_cast<unsigned char *>(workspace);
-  if ((rc = rt(cudaMemsetAsync(base + lo.bwd_off, 0, lo.bwd_bytes, st)))) return rc;
   esa::BwdArgs args;
   args.s = scan_shape(B, T, H, D, lo);
   args.da = da;
@@ -291,11 +279,27 @@ int esa_check(void *workspace, void *stream) {
   int rc = check_device();
   if (rc) return rc;
   if ((rc = rt(cudaStreamSynchronize(static_cast<cudaStream_t>(stream))))) return rc;
-  unsigned status = 0;
-  if ((rc = rt(cudaMemcpy(&status, workspace, sizeof(status), cudaMemcpyDeviceToHost)))) return rc;
-  if (status == 0) return ESA_OK;
-  if ((rc = rt(cudaMemset(workspace, 0, sizeof(status))))) return rc;
-  return ESA_ERR_TIMEOUT;
+  esa::WsHeader h;
+  if ((rc = rt(cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost)))) return rc;
+  const unsigned status = h.status;
+  if (status != 0) {
+    unsigned char *st_word = static_cast<unsigned char *>(workspace) + offsetof(esa::WsHeader, status);
+    if ((rc = rt(cudaMemset(st_word, 0, sizeof(unsigned))))) return rc;
+  }
+  if (h.magic != esa::kWorkspaceMagic || (status & esa::kStatusUninit)) return ESA_ERR_WORKSPACE;
+  if (status & esa::kStatusTimeout) return ESA_ERR_TIMEOUT;
+  return ESA_OK;
+}
+
+int esa_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
+  if (!workspace) return ESA_ERR_ARG;
+  if (!aligned16(workspace)) return ESA_ERR_ALIGN;
+  if (workspace_bytes < kHeaderBytes) return ESA_ERR_WORKSPACE;
+  int rc = check_device();
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = rt(cudaMemsetAsync(workspace, 0, workspace_bytes, st)))) return rc;
+  return esa::launch_ws_init(static_cast<esa::WsHeader *>(workspace), st);
 }
 
 const char *esa_strerror(int status) {

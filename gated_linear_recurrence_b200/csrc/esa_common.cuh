@@ -13,31 +13,57 @@
 namespace esa {
 
 constexpr float kEps = 1e-6f;          // RMS-norm epsilon (inside the square root)
-constexpr unsigned kFlagAgg = 1u;      // chunk aggregate published
-constexpr unsigned kFlagIncl = 2u;     // chunk's inclusive carry published
-constexpr unsigned kStatusTimeout = 1u;
+
+// Device status bits (sticky in the workspace header until esa_check).
+constexpr unsigned kStatusTimeout = 1u;    // a bounded wait gave up
+constexpr unsigned kStatusUninit = 2u;     // workspace not initialised (or epochs exhausted)
+
 // Iteration cap of every device-side wait.  With the back-off below this is
 // at most a second or two, far above any legitimate wait (microseconds).
 constexpr unsigned kSpinLimit = 1u << 21;
 
+// Marks an initialised workspace header.
+constexpr unsigned long long kWorkspaceMagic = 0x45534153434e3031ull;
+
 // ---------------------------------------------------------------------------
-// Workspace view.  Every time chunk of every sequence owns one "slot":
+// Workspace.  A 256-byte header followed by per-chunk carry words.  Every
+// time chunk of every sequence owns one "slot":
 //   slot = chain * nchunks + chunk,  chain = b * nct + ct
-// where ct indexes channel tiles of CT channels.  Per slot and channel:
-//   agg   (P, S): the chunk's affine carry map  x -> P x + S
-//   fstate       : forward state at the chunk's end (checkpoint for backward)
-//   bstate       : backward carry leaving the chunk towards earlier time
+// and per slot and channel:
+//   incl_f  (E, tag)          forward state at the chunk's end; also the
+//                             checkpoint the backward replays from
+//   incl_b  (H, tag)          backward carry leaving the chunk (to earlier time)
+//   agg     (P, tag), (S, tag) the chunk's affine carry map x -> P x + S
+// Each word packs a float32 value with the 32-bit epoch of the call that wrote
+// it, and is written with one single-copy-atomic 64-bit store, so a reader
+// that sees the current epoch also sees the matching value: publication needs
+// no fence and a look-back needs one round trip.  The epoch advances by one
+// per scan call (the kernel's last CTA does it) and is never 0; init zeroes
+// every word, so no stale word can carry a current tag.
 // ---------------------------------------------------------------------------
-struct Workspace {
-  unsigned *fwd_hdr;    // [1] tile ticket counter, [2] abort flag
-  unsigned *fwd_flags;
-  unsigned *bwd_hdr;
-  unsigned *bwd_flags;
-  unsigned *status;     // sticky device status (0 = ok)
-  float2 *agg;
-  float *fstate;
-  float *bstate;
+struct WsHeader {
+  unsigned long long magic;   // kWorkspaceMagic once initialised
+  unsigned epoch;             // tag used by the next scan call
+  unsigned status;            // sticky status bits
+  unsigned ticket[2];         // tile ticket counters: [0] forward, [1] backward
+  unsigned done[2];           // CTAs finished, per kernel
+  unsigned abort[2];          // raised by a CTA whose wait gave up
 };
+
+struct Workspace {
+  WsHeader *hdr;
+  unsigned long long *incl_f;
+  unsigned long long *incl_b;
+  ulonglong2 *agg;
+};
+
+__device__ __forceinline__ unsigned long long pack_tag(float v, unsigned tag) {
+  return (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(v);
+}
+__device__ __forceinline__ unsigned tag_of(unsigned long long w) { return static_cast<unsigned>(w >> 32); }
+__device__ __forceinline__ float val_of(unsigned long long w) {
+  return __uint_as_float(static_cast<unsigned>(w));
+}
 
 // ---------------------------------------------------------------------------
 // I/O element traits: 8 consecutive channels per thread.
@@ -201,10 +227,25 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+__device__ __forceinline__ unsigned long long ld_relaxed_b64(const unsigned long long *p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
+}
+
+// Two independent 64-bit words (each single-copy atomic on its own).
+__device__ __forceinline__ ulonglong2 ld_relaxed_v2b64(const ulonglong2 *p) {
+  ulonglong2 v;
+  asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_relaxed_b64(unsigned long long *p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_relaxed_v2b64(ulonglong2 *p, ulonglong2 v) {
+  asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(p), "l"(v.x), "l"(v.y) : "memory");
 }
 
 __device__ __forceinline__ unsigned ld_relaxed(const unsigned *p) {
@@ -213,21 +254,8 @@ __device__ __forceinline__ unsigned ld_relaxed(const unsigned *p) {
   return v;
 }
 
-__device__ __forceinline__ void st_relaxed(unsigned *p, unsigned v) {
-  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 
-// Release fence at GPU scope.  Issued by one thread after a CTA barrier, it
-// orders the barrier participants' earlier writes before the thread's next
-// (flag) store, as seen by any thread that acquires that flag.
-__device__ __forceinline__ void fence_acq_rel_gpu() {
-  asm volatile("fence.acq_rel.gpu;" ::: "memory");
-}
 
-// Named barrier over the first `nthreads` threads of the CTA (id 1; id 0 is __syncthreads).
-__device__ __forceinline__ void bar_sync_first(unsigned nthreads) {
-  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
-}
 
 // Wait for the TMA transaction on `bar` (given phase parity).  Bounded: on
 // giving up it records a timeout in the status word and returns false.

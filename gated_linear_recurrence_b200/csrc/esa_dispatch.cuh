@@ -13,10 +13,10 @@ int dispatch_d(int D, F &&f) {
   constexpr int L = sizeof(T) == 4 ? 32 : 64;
   constexpr int K = kStepsPerThread;
   switch (D) {
-    case 8: return f.template operator()<T, MODE, 1, 16, L, K>();
-    case 16: return f.template operator()<T, MODE, 2, 16, L, K>();
-    case 32: return f.template operator()<T, MODE, 4, 16, L, K>();
-    case 64: return f.template operator()<T, MODE, 8, 16, L, K>();
+    case 8: return f.template operator()<T, MODE, 1, 8, L, K>();
+    case 16: return f.template operator()<T, MODE, 2, 8, L, K>();
+    case 32: return f.template operator()<T, MODE, 4, 8, L, K>();
+    case 64: return f.template operator()<T, MODE, 8, 8, L, K>();
     case 128: return f.template operator()<T, MODE, 16, 16, L, K>();
     case 256: return f.template operator()<T, MODE, 32, 32, L, K>();
     default: return -3;

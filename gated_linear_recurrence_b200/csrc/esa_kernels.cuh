@@ -3,7 +3,7 @@
 //
 // Work decomposition (forward and backward):
 //   * A "chain" is one batch row b and one tile of CT consecutive channels
-//     (CT = 128, or 256 when the head dimension is 256).  Heads never straddle
+//     (CT = 64, or D when the head dimension D is 128 or 256).  Heads never straddle
 //     a channel tile, so the per-head RMS readout stays inside one CTA.
 //   * A chain is cut into time chunks of L steps.  A tile is one (chain,
 //     chunk); its a/v/q(/dy) boxes [L x CT] are staged in shared memory by TMA
@@ -13,9 +13,10 @@
 //     folds its run into an affine map x -> P x + S per channel; the runs of a
 //     tile are combined by a short serial scan per channel in shared memory;
 //     the tile map is chained to earlier tiles by a single-pass decoupled
-//     look-back over per-chunk flags in the workspace, one warp polling a
-//     window of 32 predecessors at a time.  Pass 2 replays the run from its
-//     exact carry-in and emits the readout.
+//     look-back: every channel publishes its chunk map and, once known, its
+//     chunk-end carry as epoch-tagged 64-bit words, and reads those of its
+//     four nearest predecessors in one round trip (no fences, no flags).
+//     Pass 2 replays the run from its exact carry-in and emits the readout.
 //   * The carry is always applied in chunk order, oldest first, with the same
 //     fused multiply-add that the producing tile used for its own inclusive
 //     state, so the result is bitwise independent of how far a look-back
@@ -24,8 +25,10 @@
 //     atomic ticket (taken one tile ahead, chain as the fast index, so a
 //     tile's predecessor always belongs to a running CTA), and the TMA loads
 //     of the next tile are in flight while the current one is processed.
+//     The last CTA to finish resets the ticket counter and advances the
+//     workspace epoch, so a call needs no separate reset launch.
 //     Every wait is bounded (iteration cap, then an error status).
-//   * The forward stores the state at every chunk end (fstate); the backward
+//   * The forward stores the state at every chunk end (incl_f); the backward
 //     replays each chunk from that checkpoint, so nothing of size T x C is
 //     stored besides the outputs.
 #pragma once
@@ -74,7 +77,6 @@ struct TileCfg {
   static constexpr int VW = VW0 < VPR ? VW0 : VPR; // vectors per warp row segment
   static constexpr int RW = 32 / VW;               // runs per warp
   static constexpr int NVSEG = VPR / VW;
-  static constexpr int LB_WARP = CT / 32 - 1;      // the warp that polls look-back flags
   static constexpr unsigned kBoxBytes = L * CT * sizeof(T);
   static_assert(L % K == 0, "K must divide L");
   static_assert(NT % 32 == 0 && NT <= 1024, "bad block size");
@@ -175,85 +177,121 @@ __device__ __forceinline__ float2 scan_runs(float2 *scan, int c) {
   return make_float2(cp, cs);
 }
 
-// Called by warp LB_WARP: find the nearest predecessor of `slot` (at
-// distance 1..avail, step `dir`) whose inclusive carry is published, with
-// every tile in between at least aggregate-published.  Returns its slot, or
-// -1 if the bounded wait gave up (status recorded).
-__device__ __forceinline__ long find_inclusive(const unsigned *flags, long slot, int dir, int avail,
-                                               unsigned *abort_flag, unsigned *status) {
-  const int lane = threadIdx.x & 31;
-  int base = 1;
-  unsigned ns = 32;
+// The carry entering chunk `slot` for channel `c`: the nearest predecessor
+// (distance 1, 2, ... in direction `dir`, at most `avail`) whose chunk-end
+// carry carries the current tag, with the chunk maps of every tile in between
+// applied oldest first -- the same fused multiply-adds those tiles used for
+// their own carries, so the value does not depend on how far the search went.
+// Distances 1..4 are read in one round trip; deeper searches walk one chunk
+// at a time.  Bounded: gives up (returns 0, records a timeout, raises the
+// abort flag) after kSpinLimit polls or when another CTA raised the flag.
+__device__ __forceinline__ float carry_in(const unsigned long long *incl, const ulonglong2 *agg, long slot, int dir,
+                                       int avail, int CT, int c, unsigned tag, unsigned *abort_flag,
+                                       unsigned *status) {
+  const long me = slot * CT + c;
+  const long step = static_cast<long>(dir) * CT;
+  unsigned ns = 16;
   for (unsigned it = 0; it < kSpinLimit; ++it) {
-    const int dist = base + lane;
-    const bool in = dist <= avail;
-    const unsigned f = in ? ld_acquire(&flags[slot + static_cast<long>(dir) * dist]) : 0u;
-    const unsigned incl = __ballot_sync(0xffffffffu, in && f == kFlagIncl);
-    const unsigned missing = __ballot_sync(0xffffffffu, in && f == 0u);
-    if (incl) {
-      const int first = __ffs(incl) - 1;
-      if ((missing & ((1u << first) - 1u)) == 0u) return slot + static_cast<long>(dir) * (base + first);
-    } else if (missing == 0u && base + 31 < avail) {
-      base += 32;   // 32 aggregates in a row: keep walking back
-      continue;
+    unsigned long long iw[4];
+    ulonglong2 aw[4];
+#pragma unroll
+    for (int d = 0; d < 4; ++d) {
+      if (d < avail) {
+        iw[d] = ld_relaxed_b64(&incl[me + (d + 1) * step]);
+        aw[d] = ld_relaxed_v2b64(&agg[me + (d + 1) * step]);
+      } else {
+        iw[d] = 0ull;
+        aw[d] = make_ulonglong2(0ull, 0ull);
+      }
     }
-    if ((it & 63u) == 63u) {
-      const unsigned ab = (lane == 0) ? ld_relaxed(abort_flag) : 0u;
-      if (__shfl_sync(0xffffffffu, ab, 0)) break;
+    int found = -1;
+    bool blocked = false;
+#pragma unroll
+    for (int d = 0; d < 4; ++d) {
+      if (found < 0 && !blocked && d < avail) {
+        if (tag_of(iw[d]) == tag) found = d;
+        else if (tag_of(aw[d].x) != tag || tag_of(aw[d].y) != tag) blocked = true;
+      }
     }
+    if (found >= 0) {
+      float E = val_of(found == 0 ? iw[0] : found == 1 ? iw[1] : found == 2 ? iw[2] : iw[3]);
+#pragma unroll
+      for (int d = 3; d >= 0; --d)
+        if (d < found) E = __fmaf_rn(val_of(aw[d].x), E, val_of(aw[d].y));
+      return E;
+    }
+    if (!blocked && avail > 4) {
+      // Four chunk maps in a row and no carry yet: walk further back.
+      int far = 4;   // distances 1..far have published maps
+      for (; it < kSpinLimit; ++it) {
+        const long at = me + static_cast<long>(far + 1) * step;
+        const unsigned long long w = ld_relaxed_b64(&incl[at]);
+        if (tag_of(w) == tag) {
+          float E = val_of(w);
+          for (int d = far; d >= 1; --d) {
+            const ulonglong2 m = ld_relaxed_v2b64(&agg[me + static_cast<long>(d) * step]);
+            E = __fmaf_rn(val_of(m.x), E, val_of(m.y));
+          }
+          return E;
+        }
+        const ulonglong2 m = ld_relaxed_v2b64(&agg[at]);
+        if (tag_of(m.x) == tag && tag_of(m.y) == tag && far + 1 < avail) {
+          ++far;
+          continue;
+        }
+        if ((it & 63u) == 63u && ld_relaxed(abort_flag)) break;
+        __nanosleep(ns);
+        ns = ns < 256 ? ns * 2 : 256;
+      }
+      break;
+    }
+    if ((it & 63u) == 63u && ld_relaxed(abort_flag)) break;
     __nanosleep(ns);
     ns = ns < 256 ? ns * 2 : 256;
   }
-  if (lane == 0) {
-    atomicOr(status, kStatusTimeout);
-    atomicExch(abort_flag, 1u);
-  }
-  return -1;
+  atomicOr(status, kStatusTimeout);
+  atomicExch(abort_flag, 1u);
+  return 0.0f;
 }
 
-// Apply the aggregates of the tiles strictly between `j` (inclusive carry
-// published) and `slot`, oldest first, to j's carry.  Channel c.
-__device__ __forceinline__ float apply_carries(const float2 *agg, const float *state, long j, long slot, int dir,
-                                               int CT, int c) {
-  float E = __ldcg(&state[j * CT + c]);
-  long m = j - dir;
-  for (; (slot - m) * (-dir) >= 4; m -= 4 * dir) {   // four loads in flight
-    const float2 e0 = __ldcg(&agg[m * CT + c]);
-    const float2 e1 = __ldcg(&agg[(m - dir) * CT + c]);
-    const float2 e2 = __ldcg(&agg[(m - 2 * dir) * CT + c]);
-    const float2 e3 = __ldcg(&agg[(m - 3 * dir) * CT + c]);
-    E = __fmaf_rn(e0.x, E, e0.y);
-    E = __fmaf_rn(e1.x, E, e1.y);
-    E = __fmaf_rn(e2.x, E, e2.y);
-    E = __fmaf_rn(e3.x, E, e3.y);
+// Kernel prologue shared by both scans (thread 0): read the epoch tag and
+// check the workspace is initialised.  Returns the tag, or 0 if not.
+__device__ __forceinline__ unsigned scan_prologue(WsHeader *hdr) {
+  const unsigned long long magic = *reinterpret_cast<volatile unsigned long long *>(&hdr->magic);
+  const unsigned epoch = *reinterpret_cast<volatile unsigned *>(&hdr->epoch);
+  if (magic != kWorkspaceMagic || epoch == 0u) {
+    atomicOr(&hdr->status, kStatusUninit);
+    return 0u;
   }
-  for (; m != slot; m -= dir) {
-    const float2 e = __ldcg(&agg[m * CT + c]);
-    E = __fmaf_rn(e.x, E, e.y);
-  }
-  return E;
+  return epoch;
 }
 
-// The carry entering tile `slot` (threads 0..CT-1; uses named barrier 1).
-// Publishes the tile's aggregate first.  `avail` = number of predecessors.
-template <typename Cfg>
-__device__ __forceinline__ float lookback_carry(const Workspace &ws, unsigned *flags, unsigned *hdr, float *state,
-                                                long slot, int dir, int avail, float2 tile_map, long *bcast) {
-  const int tid = threadIdx.x;
-  ws.agg[slot * Cfg::CT + tid] = tile_map;
-  bar_sync_first(Cfg::CT);
-  if (tid == 0) {
-    fence_acq_rel_gpu();
-    st_relaxed(&flags[slot], kFlagAgg);
+// Kernel epilogue (all threads): the last CTA to finish resets the ticket,
+// done and abort words of kernel `k` and advances the epoch (an exhausted
+// epoch range clears the magic, so the next call reports an uninitialised
+// workspace instead of reusing tags).
+__device__ __forceinline__ void scan_epilogue(WsHeader *hdr, int k, bool ran) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned prev = atomicAdd(&hdr->done[k], 1u);
+    if (prev == gridDim.x - 1) {
+      __threadfence();
+      hdr->ticket[k] = 0u;
+      hdr->done[k] = 0u;
+      hdr->abort[k] = 0u;
+      if (ran) {
+        const unsigned next = hdr->epoch + 1u;
+        if (next == 0u) {
+          hdr->magic = 0ull;
+          hdr->epoch = 0u;
+        } else {
+          hdr->epoch = next;
+        }
+      }
+      __threadfence();
+    }
   }
-  if ((tid >> 5) == Cfg::LB_WARP) {
-    const long j = find_inclusive(flags, slot, dir, avail, &hdr[2], ws.status);
-    if ((tid & 31) == 0) *bcast = j;
-  }
-  bar_sync_first(Cfg::CT);
-  const long j = *bcast;
-  if (j < 0) return 0.0f;
-  return apply_carries(ws.agg, state, j, slot, dir, Cfg::CT, tid);
 }
 
 // Gate of one channel in the form the recurrence uses: direct keeps A,
@@ -271,7 +309,7 @@ __device__ __forceinline__ float rec_step(float c, float E, float v) {
 // Forward scan (persistent).
 // ===========================================================================
 template <typename T, int MODE, int LPH, int VPR, int L, int K>
-__global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
+__global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 128) ? 4 : (VPR * (L / K) <= 256) ? 2 : 1)
     esa_scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_q, const FwdArgs args) {
   using Cfg = TileCfg<T, LPH, VPR, L, K>;
@@ -283,12 +321,12 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
   float *es_s = reinterpret_cast<float *>(base + 2 * Sm::kStage);
   uint64_t *bar = reinterpret_cast<uint64_t *>(es_s + CT);     // [2]
   int *ticket_s = reinterpret_cast<int *>(bar + 2);            // [2]
-  long *bcast = reinterpret_cast<long *>(ticket_s + 2);
+  unsigned *tag_s = reinterpret_cast<unsigned *>(ticket_s + 2);
 
   const int tid = threadIdx.x;
   const ScanShape &sh = args.s;
   const Workspace &ws = args.ws;
-  unsigned *hdr = ws.fwd_hdr;
+  WsHeader *hdr = ws.hdr;
 
   auto box = [&](int stage, int k) -> T * {
     return reinterpret_cast<T *>(base + stage * Sm::kStage + k * size_t(Cfg::kBoxBytes));
@@ -310,8 +348,10 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
     mbar_init(&bar[1], 1);
     fence_mbar_init();
     fence_proxy_async_smem();
-    const int t0 = static_cast<int>(atomicAdd(&hdr[1], 1u));
-    const int t1 = static_cast<int>(atomicAdd(&hdr[1], 1u));
+    const unsigned tag = scan_prologue(hdr);
+    *tag_s = tag;
+    const int t0 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[0], 1u)) : sh.ntiles;
+    const int t1 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[0], 1u)) : sh.ntiles;
     ticket_s[0] = t0;
     ticket_s[1] = t1;
     if (t0 < sh.ntiles) issue(0, t0);
@@ -321,6 +361,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
 
   const ThreadPos<Cfg> pos(tid);
   T *yg = static_cast<T *>(args.y);
+  const unsigned tag = *tag_s;
   unsigned phase = 0;   // bit s = parity of stage s
 
   for (int it = 0;; ++it) {
@@ -328,7 +369,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
     const int tile = ticket_s[s];
     if (tile >= sh.ntiles) break;
     unsigned next = 0;
-    if (tid == 0) next = atomicAdd(&hdr[1], 1u);   // the tile that will refill this stage
+    if (tid == 0) next = atomicAdd(&hdr->ticket[0], 1u);   // the tile that will refill this stage
 
     const int chain = tile % sh.nchains, chunk = tile / sh.nchains;
     const int b = chain / sh.nct, c0 = (chain % sh.nct) * CT, t0 = chunk * L;
@@ -338,7 +379,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
     const T *q_s = box(s, 2);
     float2 *scan_s = reinterpret_cast<float2 *>(box(s, 0));   // reused once pass 1 is done
 
-    mbar_wait_bounded(&bar[s], (phase >> s) & 1u, ws.status);
+    mbar_wait_bounded(&bar[s], (phase >> s) & 1u, &hdr->status);
     phase ^= 1u << s;
 
     // ---- pass 1: gates and the run's affine map ---------------------------
@@ -372,22 +413,20 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
       const float2 tmap = scan_runs<CT, RUNS, false>(scan_s, tid);
       const int cg = c0 + tid;
       float E_start;
+      const long at = slot * CT + tid;
       if (chunk == 0) {
         E_start = (args.E_init != nullptr && cg < sh.C) ? args.E_init[static_cast<long>(b) * sh.C + cg] : 0.0f;
       } else {
-        E_start = lookback_carry<Cfg>(ws, ws.fwd_flags, hdr, ws.fstate, slot, -1, chunk, tmap, bcast);
+        st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tmap.x, tag), pack_tag(tmap.y, tag)));
+        E_start = carry_in(ws.incl_f, ws.agg, slot, -1, chunk, CT, tid, tag, &hdr->abort[0], &hdr->status);
       }
       const float E_end = __fmaf_rn(tmap.x, E_start, tmap.y);
-      ws.fstate[slot * CT + tid] = E_end;
+      st_relaxed_b64(&ws.incl_f[at], pack_tag(E_end, tag));
       if (chunk == sh.nchunks - 1 && args.E_final != nullptr && cg < sh.C)
         args.E_final[static_cast<long>(b) * sh.C + cg] = E_end;
       es_s[tid] = E_start;
     }
     __syncthreads();
-    if (tid == 0) {   // publish this chunk's end state
-      fence_acq_rel_gpu();
-      st_relaxed(&ws.fwd_flags[slot], kFlagIncl);
-    }
 
     // ---- pass 2: exact states and the readout ------------------------------
     float E[8];
@@ -430,14 +469,41 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
       }
     }
   }
+  scan_epilogue(hdr, 0, tag != 0u);
+}
+
+// ghat (8 float32) of one thread's row, kept in that row's q and dy slots:
+// 16-bit I/O splits it over both 16-byte slots; float32 I/O uses the q slot.
+template <typename T>
+__device__ __forceinline__ void put_ghat(T *q_slot, T *dy_slot, const float (&g)[8]) {
+  if (sizeof(T) == 2) {
+    reinterpret_cast<float4 *>(q_slot)[0] = make_float4(g[0], g[1], g[2], g[3]);
+    reinterpret_cast<float4 *>(dy_slot)[0] = make_float4(g[4], g[5], g[6], g[7]);
+  } else {
+    reinterpret_cast<float4 *>(q_slot)[0] = make_float4(g[0], g[1], g[2], g[3]);
+    reinterpret_cast<float4 *>(q_slot)[1] = make_float4(g[4], g[5], g[6], g[7]);
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void get_ghat(const T *q_slot, const T *dy_slot, float (&g)[8]) {
+  float4 u, w;
+  if (sizeof(T) == 2) {
+    u = reinterpret_cast<const float4 *>(q_slot)[0];
+    w = reinterpret_cast<const float4 *>(dy_slot)[0];
+  } else {
+    u = reinterpret_cast<const float4 *>(q_slot)[0];
+    w = reinterpret_cast<const float4 *>(q_slot)[1];
+  }
+  g[0] = u.x; g[1] = u.y; g[2] = u.z; g[3] = u.w;
+  g[4] = w.x; g[5] = w.y; g[6] = w.z; g[7] = w.w;
 }
 
 // ===========================================================================
 // Backward scan (persistent).
 // ===========================================================================
-// Two CTAs per SM when the block has at most 256 threads (the smem plan fits).
 template <typename T, int MODE, int LPH, int VPR, int L, int K>
-__global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
+__global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 128) ? 4 : (VPR * (L / K) <= 256) ? 2 : 1)
     esa_scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dy,
                         const BwdArgs args) {
@@ -452,12 +518,12 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
   float *es_s = reinterpret_cast<float *>(base + 2 * Sm::kStage + Sm::kQdy);
   uint64_t *bar = reinterpret_cast<uint64_t *>(es_s + CT);     // [0..1] a/v stages, [2] q/dy
   int *ticket_s = reinterpret_cast<int *>(bar + 3);            // [2]
-  long *bcast = reinterpret_cast<long *>(ticket_s + 2);
+  unsigned *tag_s = reinterpret_cast<unsigned *>(ticket_s + 2);
 
   const int tid = threadIdx.x;
   const ScanShape &sh = args.s;
   const Workspace &ws = args.ws;
-  unsigned *hdr = ws.bwd_hdr;
+  WsHeader *hdr = ws.hdr;
 
   auto box = [&](int stage, int k) -> T * {
     return reinterpret_cast<T *>(base + stage * Sm::kStage + k * size_t(Cfg::kBoxBytes));
@@ -494,8 +560,10 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
     mbar_init(&bar[2], 1);
     fence_mbar_init();
     fence_proxy_async_smem();
-    const int t0 = static_cast<int>(atomicAdd(&hdr[1], 1u));
-    const int t1 = static_cast<int>(atomicAdd(&hdr[1], 1u));
+    const unsigned tag = scan_prologue(hdr);
+    *tag_s = tag;
+    const int t0 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[1], 1u)) : sh.ntiles;
+    const int t1 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[1], 1u)) : sh.ntiles;
     ticket_s[0] = t0;
     ticket_s[1] = t1;
     if (t0 < sh.ntiles) {
@@ -510,6 +578,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
   T *dag = static_cast<T *>(args.da);
   T *dvg = static_cast<T *>(args.dv);
   T *dqg = static_cast<T *>(args.dq);
+  const unsigned tag = *tag_s;
   unsigned phase = 0;   // bits 0..1: a/v stages, bit 2: q/dy
 
   for (int it = 0;; ++it) {
@@ -517,7 +586,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
     const int tile = ticket_s[s];
     if (tile >= sh.ntiles) break;
     unsigned next = 0;
-    if (tid == 0) next = atomicAdd(&hdr[1], 1u);
+    if (tid == 0) next = atomicAdd(&hdr->ticket[1], 1u);
 
     const int chain = tile % sh.nchains;
     const int chunk = sh.nchunks - 1 - tile / sh.nchains;
@@ -532,10 +601,10 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
       const int cg = c0 + tid;
       E_ck = (chunk == 0) ? ((args.E_init != nullptr && cg < sh.C) ? args.E_init[static_cast<long>(b) * sh.C + cg]
                                                                    : 0.0f)
-                          : __ldcg(&ws.fstate[(slot - 1) * CT + tid]);
+                          : val_of(__ldcg(&ws.incl_f[(slot - 1) * CT + tid]));
     }
 
-    mbar_wait_bounded(&bar[s], (phase >> s) & 1u, ws.status);
+    mbar_wait_bounded(&bar[s], (phase >> s) & 1u, &hdr->status);
     phase ^= 1u << s;
 
     // ---- F1: gates and the run's forward map ------------------------------
@@ -568,22 +637,19 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
     __syncthreads();
 
     // ---- F2: replay states, readout backward, dq, ghat ---------------------
-    float Ec[8];   // the run's forward carry-in
-    {
-      float pe[8], se[8];
-      scan_load8<CT>(scan_s, pos.run, pos.ch, pe, se);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) Ec[j] = __fmaf_rn(pe[j], es_s[pos.ch + j], se[j]);
-    }
-    mbar_wait_bounded(&bar[2], (phase >> 2) & 1u, ws.status);
-    phase ^= 4u;
-    float gh[K][8];
-    const bool ch_ok = (c0 + pos.ch) < sh.C;
-    const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
+    // ghat of each row overwrites that row's q/dy slots (only this thread
+    // reads them); w keeps what da needs of the previous state.
+    float w[K][8];   // direct: E_{t-1}; controlled: E_{t-1} - v_t
     {
       float E[8];
+      {
+        float pe[8], se[8];
+        scan_load8<CT>(scan_s, pos.run, pos.ch, pe, se);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) E[j] = Ec[j];
+        for (int j = 0; j < 8; ++j) E[j] = __fmaf_rn(pe[j], es_s[pos.ch + j], se[j]);
+      }
+      mbar_wait_bounded(&bar[2], (phase >> 2) & 1u, &hdr->status);
+      phase ^= 4u;
 #pragma unroll
       for (int i = 0; i < K; ++i) {
         const int r = pos.row0 + i;
@@ -595,6 +661,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
         float ss = 0.0f;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
+          w[i][j] = (MODE == 0) ? E[j] : E[j] - vv[j];
           E[j] = rec_step<MODE>(Ar[i][j], E[j], vv[j]);
           ss = __fmaf_rn(E[j], E[j], ss);
         }
@@ -610,13 +677,14 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
           dot = __fmaf_rn(dn[j], nn[j], dot);
         }
         dot = head_sum<LPH>(dot) * sh.inv_D;
+        float gh[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) gh[i][j] = rr * __fmaf_rn(-nn[j], dot, dn[j]);
-        if (valid && ch_ok) Io<T>::store8(dqg + gbase + static_cast<long>(r) * sh.C, dqv);
+        for (int j = 0; j < 8; ++j) gh[j] = rr * __fmaf_rn(-nn[j], dot, dn[j]);
+        put_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
+        if (valid && (c0 + pos.ch) < sh.C)
+          Io<T>::store8(dqg + (static_cast<long>(b) * sh.T + t0 + r) * sh.C + c0 + pos.ch, dqv);
       }
     }
-    __syncthreads();   // q/dy box and the forward prefixes are free
-    if (tid == 0 && ticket_s[s ^ 1] < sh.ntiles) issue_qdy(ticket_s[s ^ 1]);
 
     // ---- R1: the run's reverse map h -> P h + hl ----------------------------
     {
@@ -625,14 +693,18 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
       for (int j = 0; j < 8; ++j) hl[j] = 0.0f;
 #pragma unroll
       for (int i = K - 1; i >= 0; --i) {
-        if ((t0 + pos.row0 + i) < sh.T) {
+        const int r = pos.row0 + i;
+        if ((t0 + r) < sh.T) {
+          float gh[8];
+          get_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const float A = (MODE == 0) ? Ar[i][j] : 1.0f - Ar[i][j];
-            hl[j] = A * (gh[i][j] + hl[j]);
+            hl[j] = A * (gh[j] + hl[j]);
           }
         }
       }
+      __syncthreads();   // every thread has read its forward prefixes
       scan_store8<CT>(scan_s, pos.run, pos.ch, P, hl);
     }
     __syncthreads();
@@ -642,87 +714,74 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 256) ? 2 : 1)
       const float2 tmap = scan_runs<CT, RUNS, true>(scan_s, tid);
       const int cg = c0 + tid;
       float H_in;
+      const long at = slot * CT + tid;
       if (chunk == sh.nchunks - 1) {
         H_in = (args.dE_final != nullptr && cg < sh.C) ? args.dE_final[static_cast<long>(b) * sh.C + cg] : 0.0f;
       } else {
-        H_in = lookback_carry<Cfg>(ws, ws.bwd_flags, hdr, ws.bstate, slot, +1, sh.nchunks - 1 - chunk, tmap,
-                                   bcast);
+        st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tmap.x, tag), pack_tag(tmap.y, tag)));
+        H_in = carry_in(ws.incl_b, ws.agg, slot, +1, sh.nchunks - 1 - chunk, CT, tid, tag, &hdr->abort[1],
+                        &hdr->status);
       }
       const float H_out = __fmaf_rn(tmap.x, H_in, tmap.y);
-      ws.bstate[slot * CT + tid] = H_out;
+      st_relaxed_b64(&ws.incl_b[at], pack_tag(H_out, tag));
       if (chunk == 0 && args.dE_init != nullptr && cg < sh.C)
         args.dE_init[static_cast<long>(b) * sh.C + cg] = H_out;
       es_s[tid] = H_in;
     }
     __syncthreads();
-    if (tid == 0) {
-      fence_acq_rel_gpu();
-      st_relaxed(&ws.bwd_flags[slot], kFlagIncl);
-    }
 
-    // ---- B1: total gradient G_t, latest step first ---------------------------
+    // ---- B: total gradient G_t and da, dv, latest step first -----------------
     {
       float h[8];
-      float pe[8], se[8];
-      scan_load8<CT>(scan_s, pos.run, pos.ch, pe, se);
+      {
+        float pe[8], se[8];
+        scan_load8<CT>(scan_s, pos.run, pos.ch, pe, se);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) h[j] = __fmaf_rn(pe[j], es_s[pos.ch + j], se[j]);
+        for (int j = 0; j < 8; ++j) h[j] = __fmaf_rn(pe[j], es_s[pos.ch + j], se[j]);
+      }
+      const bool ch_ok = (c0 + pos.ch) < sh.C;
+      const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
 #pragma unroll
       for (int i = K - 1; i >= 0; --i) {
-        if ((t0 + pos.row0 + i) < sh.T) {
+        const int r = pos.row0 + i;
+        if ((t0 + r) < sh.T) {
+          float gh[8], dav[8], dvv[8];
+          get_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const float A = (MODE == 0) ? Ar[i][j] : 1.0f - Ar[i][j];
-            const float G = gh[i][j] + h[j];
-            gh[i][j] = G;
-            h[j] = A * G;
+            const float G = gh[j] + h[j];
+            if (MODE == 0) {
+              const float A = Ar[i][j];
+              dvv[j] = G;
+              dav[j] = G * w[i][j] * (A * (1.0f - A));
+              h[j] = A * G;
+            } else {
+              const float Ac = Ar[i][j];
+              const float A = 1.0f - Ac;
+              dvv[j] = G * Ac;
+              dav[j] = G * w[i][j] * (A * Ac);
+              h[j] = A * G;
+            }
+          }
+          if (ch_ok) {
+            const long off = gbase + static_cast<long>(r) * sh.C;
+            Io<T>::store8(dag + off, dav);
+            Io<T>::store8(dvg + off, dvv);
           }
         }
       }
     }
 
-    // ---- B2: replay states forward, emit da and dv ---------------------------
-    {
-      float E[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) E[j] = Ec[j];
-#pragma unroll
-      for (int i = 0; i < K; ++i) {
-        const int r = pos.row0 + i;
-        float vv[8], dav[8], dvv[8];
-        Io<T>::load8(v_s + r * CT + pos.ch, vv);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float G = gh[i][j];
-          if (MODE == 0) {
-            const float A = Ar[i][j];
-            dvv[j] = G;
-            dav[j] = G * E[j] * (A * (1.0f - A));
-          } else {
-            const float Ac = Ar[i][j];
-            dvv[j] = G * Ac;
-            dav[j] = G * (E[j] - vv[j]) * ((1.0f - Ac) * Ac);
-          }
-          E[j] = rec_step<MODE>(Ar[i][j], E[j], vv[j]);
-        }
-        if ((t0 + r) < sh.T && ch_ok) {
-          const long off = gbase + static_cast<long>(r) * sh.C;
-          Io<T>::store8(dag + off, dav);
-          Io<T>::store8(dvg + off, dvv);
-        }
-      }
-    }
-
-    // ---- refill this a/v stage ----------------------------------------------
+    // ---- refill: next tile's q/dy, and this a/v stage -------------------------
     __syncthreads();
     if (tid == 0) {
+      fence_proxy_async_smem();   // generic smem writes before the async refills
+      if (ticket_s[s ^ 1] < sh.ntiles) issue_qdy(ticket_s[s ^ 1]);
       ticket_s[s] = static_cast<int>(next);
-      if (static_cast<int>(next) < sh.ntiles) {
-        fence_proxy_async_smem();
-        issue_av(s, static_cast<int>(next));
-      }
+      if (static_cast<int>(next) < sh.ntiles) issue_av(s, static_cast<int>(next));
     }
   }
+  scan_epilogue(hdr, 1, tag != 0u);
 }
 
 // ===========================================================================

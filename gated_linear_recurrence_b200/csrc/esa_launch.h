@@ -12,7 +12,7 @@ namespace esa {
 // Tile rows per chunk and channels per tile, as chosen for each I/O dtype and
 // head dimension.  The workspace layout and the kernels both follow these.
 inline int tile_rows(int dtype) { return dtype == 0 ? 32 : 64; }   // f32 : 16-bit
-inline int tile_cols(int D) { return D <= 128 ? 128 : 256; }
+inline int tile_cols(int D) { return D <= 64 ? 64 : D; }
 constexpr int kStepsPerThread = 4;
 
 // Launch the forward / backward scan for (dtype, mode, D).  The tensor maps
@@ -23,6 +23,8 @@ int launch_fwd(int dtype, int mode, int D, const CUtensorMap &ta, const CUtensor
 int launch_bwd(int dtype, int mode, int D, const CUtensorMap &ta, const CUtensorMap &tv,
                const CUtensorMap &tq, const CUtensorMap &tdy, const BwdArgs &args, int ntiles,
                cudaStream_t stream);
+// Write the header of a freshly zeroed workspace (magic, epoch 1).
+int launch_ws_init(WsHeader *hdr, cudaStream_t stream);
 int launch_step(int dtype, int mode, int D, const void *a, const void *v, const void *q, float *E,
                 void *y, long nvec, float inv_D, cudaStream_t stream);
 

@@ -24,6 +24,18 @@ struct StepLauncher {
 };
 }  // namespace
 
+namespace {
+__global__ void esa_ws_init_kernel(WsHeader *hdr) {
+  hdr->magic = kWorkspaceMagic;
+  hdr->epoch = 1u;
+}
+}  // namespace
+
+int launch_ws_init(WsHeader *hdr, cudaStream_t stream) {
+  esa_ws_init_kernel<<<1, 1, 0, stream>>>(hdr);
+  return launch_status(cudaGetLastError());
+}
+
 int launch_step(int dtype, int mode, int D, const void *a, const void *v, const void *q, float *E,
                 void *y, long nvec, float inv_D, cudaStream_t stream) {
   return dispatch(dtype, mode, D, StepLauncher{a, v, q, E, y, nvec, inv_D, stream});

@@ -11,6 +11,7 @@ The functions carry the C names:
 * :func:`esa_scan_bwd`  -- backward scan (da, dv, dq, dE_init)
 * :func:`esa_step`      -- one-token decode update (in place on E)
 * :func:`esa_check`     -- synchronise and read the device status of a workspace
+* :func:`esa_workspace_init` -- zero a new workspace and write its header
 * :func:`esa_workspace_size`, :func:`esa_strerror`, :func:`esa_version`
 """
 from __future__ import annotations
@@ -71,6 +72,8 @@ def load_library():
         lib.esa_step.restype = I
         lib.esa_check.argtypes = [P, P]
         lib.esa_check.restype = I
+        lib.esa_workspace_init.argtypes = [P, S, P]
+        lib.esa_workspace_init.restype = I
         lib.esa_strerror.argtypes = [I]
         lib.esa_strerror.restype = ctypes.c_char_p
         lib.esa_version.argtypes = []
@@ -132,12 +135,25 @@ def _dims(a):
     return tuple(int(s) for s in a.shape)
 
 
-def new_workspace(B, T, H, D, dtype, device):
-    """Allocate a workspace of the size the C ABI asks for (torch memory, caller-owned)."""
+def esa_workspace_init(workspace, stream=None):
+    """Zero a workspace and write its header (once, after allocation)."""
+    lib = load_library()
+    with torch.cuda.device(workspace.device):
+        rc = lib.esa_workspace_init(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(workspace.device, stream))
+    if rc != 0:
+        raise EsaError("esa_workspace_init", rc)
+    return workspace
+
+
+def new_workspace(B, T, H, D, dtype, device, stream=None):
+    """Allocate and initialise a workspace of the size the C ABI asks for
+    (torch memory, caller-owned)."""
     n = esa_workspace_size(B, T, H, D, dtype)
     if n == 0:
         raise ValueError("unsupported shape for the ESA scan")
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    return esa_workspace_init(ws, stream)
 
 
 def esa_scan_fwd(a, v, q, y=None, E_final=None, mode=CONTROLLED, E_init=None, workspace=None,

@@ -60,7 +60,7 @@ typedef enum {
     ESA_ERR_ARG = -1,         /* bad size, mode, dtype or a required NULL pointer */
     ESA_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned */
     ESA_ERR_UNSUPPORTED = -3, /* head dimension D outside {8,16,32,64,128,256} */
-    ESA_ERR_WORKSPACE = -4,   /* workspace NULL or smaller than esa_workspace_size() */
+    ESA_ERR_WORKSPACE = -4,   /* workspace NULL, too small, or not initialised (esa_workspace_init) */
     ESA_ERR_LAUNCH = -5,      /* the CUDA runtime rejected a launch or copy */
     ESA_ERR_TIMEOUT = -6,     /* a bounded device-side wait gave up (see esa_check) */
     ESA_ERR_DEVICE = -7       /* no CUDA device, or the current device is not sm_100 */
@@ -69,24 +69,41 @@ typedef enum {
 /*
  * Bytes of device workspace that esa_scan_fwd / esa_scan_bwd need for a
  * problem of this shape and dtype (0 on a bad argument).  The workspace
- * holds the float32 state at the end of every time chunk of every sequence
- * (written by the forward, read by the backward) plus the per-chunk carry
- * descriptors and status words of the single-pass scan.  About
- * 16 * B * C * ceil(T / L) bytes, L = 64 for 16-bit I/O and 32 for float32.
+ * holds a 256-byte header, the float32 state at the end of every time chunk
+ * of every sequence (written by the forward, read by the backward as its
+ * replay checkpoints) and the per-chunk carry words of the single-pass scan,
+ * each tagged with the epoch of the call that wrote it.  That is
+ * 256 + 32 * B * ceil(C / CT) * CT * ceil(T / L) bytes (rounded up to 256 B
+ * per array), with L = 64 time steps per chunk for 16-bit I/O and 32 for
+ * float32, and CT = 64 channels per tile (CT = D when D is 128 or 256).
  */
 size_t esa_workspace_size(int B, int T, int H, int D, int dtype);
 
 /*
- * Forward scan (prefill / training forward).
+ * Prepare a workspace for use: zero all `workspace_bytes` and write its
+ * header (enqueued on `stream`).  Call once after allocating the buffer,
+ * before its first scan; the buffer can then be reused by any number of scan
+ * calls of any shape whose esa_workspace_size() fits in it.  Scans advance a
+ * 32-bit epoch stored in the header; after 2^32 - 1 scan calls the header is
+ * invalidated and esa_check() reports ESA_ERR_WORKSPACE until the workspace
+ * is initialised again.  A scan given a workspace that was never initialised
+ * does no work and esa_check() reports ESA_ERR_WORKSPACE.
+ */
+int esa_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Forward scan (prefill / training forward).  The stages of the scan:
+ * gate sigmoid, chunk-local scan, carry between chunks, readout -- all in
+ * one kernel launch, without a separate reset launch.
  *   a, v, q   [B,T,H,D] inputs: gate logits, values, queries (required).
  *   y         [B,T,H,D] output: q (.) E_t / rms(E_t) (required).
  *   E_final   [B,H,D] float32 output: E_T, the state to continue decoding
  *             from (NULL = not written).  With T = 0 it equals E_init.
  *   E_init    [B,H,D] float32 initial state E_0 (NULL = zeros).
- *   workspace device buffer of at least esa_workspace_size() bytes; its
- *             previous contents are irrelevant.  After the call it holds the
- *             chunk-boundary states that esa_scan_bwd needs, so keep it
- *             unchanged until the matching backward has run.
+ *   workspace device buffer of at least esa_workspace_size() bytes,
+ *             initialised once with esa_workspace_init.  After the call it
+ *             holds the chunk-boundary states that esa_scan_bwd needs, so
+ *             run no other forward on it before the matching backward.
  * Sources: state recurrence and modes ("entangled-state-attention 0.1.0",
  * "Core idea"); prefill returning the state (mlbricks-web.pages.dev/esa,
  * Quick start: prefill returns (out, state)).
@@ -132,9 +149,11 @@ int esa_step(const void *a_t, const void *v_t, const void *q_t, float *E, void *
 
 /*
  * Synchronise `stream`, then read and clear the device status word in
- * `workspace`.  Returns ESA_OK, ESA_ERR_TIMEOUT if a bounded wait inside a
- * scan kernel gave up since the last check (the outputs of that call are
- * then invalid), or ESA_ERR_LAUNCH if the stream reports a CUDA error.
+ * `workspace`.  Returns ESA_OK; ESA_ERR_WORKSPACE if the workspace is not
+ * initialised (a scan on it did nothing); ESA_ERR_TIMEOUT if a bounded wait
+ * inside a scan kernel gave up since the last check (the outputs of that
+ * call are then invalid); or ESA_ERR_LAUNCH if the stream reports a CUDA
+ * error.
  */
 int esa_check(void *workspace, void *stream);
 

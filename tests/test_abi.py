@@ -33,8 +33,8 @@ def declared_functions():
 
 def test_header_declares_the_three_entry_points():
     names = declared_functions()
-    for n in ("esa_scan_fwd", "esa_scan_bwd", "esa_step", "esa_workspace_size", "esa_check",
-              "esa_strerror", "esa_version"):
+    for n in ("esa_scan_fwd", "esa_scan_bwd", "esa_step", "esa_workspace_size", "esa_workspace_init",
+              "esa_check", "esa_strerror", "esa_version"):
         assert n in names
 
 
@@ -61,18 +61,19 @@ def test_version_and_strerror(lib):
 
 @pytest.mark.parametrize("dtype,L", [(0, 32), (1, 64), (2, 64)])
 def test_workspace_size_layout(lib, dtype, L):
-    B, T, H, D = 3, 1000, 5, 64          # C = 320 -> 3 channel tiles of 128
-    n = B * 3 * -(-T // L)
-    expect = 0
+    B, T, H, D = 3, 1000, 5, 64          # C = 320 -> 5 channel tiles of 64
+    words = B * 5 * -(-T // L) * 64
 
     def up(x):
         return -(-x // 256) * 256
-    expect = up(32 + 4 * n)
-    expect = up(expect + 16 + 4 * n)
-    expect = up(expect + n * 128 * 8)
-    expect = up(expect + n * 128 * 4)
-    expect = up(expect + n * 128 * 4)
+    expect = 256
+    expect = up(expect + 8 * words)      # forward chunk-end states
+    expect = up(expect + 8 * words)      # backward chunk carries
+    expect = up(expect + 16 * words)     # chunk maps
     assert lib.esa_workspace_size(B, T, H, D, dtype) == expect
+    assert lib.esa_workspace_size(B, T, H, 256, dtype) == up(up(up(256 + 8 * B * -(-T // L) * 5 * 256)
+                                                                 + 8 * B * -(-T // L) * 5 * 256)
+                                                              + 16 * B * -(-T // L) * 5 * 256)
 
 
 def test_workspace_size_rejects_bad_shapes(lib):
@@ -129,6 +130,9 @@ def test_no_device_is_an_error_not_a_fallback(lib):
         pytest.skip("a CUDA device is present; this checks the device-less path")
     from gated_linear_recurrence_b200 import esa
     assert _fwd(lib) == esa.ESA_ERR_DEVICE
+    assert lib.esa_workspace_init(_fake(0x10000), 4096, None) == esa.ESA_ERR_DEVICE
+    assert lib.esa_workspace_init(None, 4096, None) == esa.ESA_ERR_ARG
+    assert lib.esa_workspace_init(_fake(0x10004), 4096, None) == esa.ESA_ERR_ALIGN
     assert lib.esa_step(_fake(0x1000), _fake(0x2000), _fake(0x3000), _fake(0x4000), _fake(0x5000),
                         2, 2, 32, 1, 1, None) == esa.ESA_ERR_DEVICE
 
