@@ -66,62 +66,84 @@ __device__ __forceinline__ float val_of(unsigned long long w) {
 }
 
 // ---------------------------------------------------------------------------
-// I/O element traits: 8 consecutive channels per thread.
+// Packed float32 pairs.  sm_100 executes FADD2 / FMUL2 / FFMA2 on two fp32
+// lanes per instruction, each lane rounded to nearest exactly like the
+// scalar instruction, so packing halves the float32 instruction count without
+// changing a single result bit.  A thread's 8 channels are 4 pairs (2i, 2i+1).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float2 splat(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+// ---------------------------------------------------------------------------
+// I/O element traits: 8 consecutive channels per thread, as 4 float2 pairs.
+// load8_gate also clamps the gate logit at -80 (in the I/O type, one packed
+// min/max per pair) so that exp(-x) stays finite.
 // ---------------------------------------------------------------------------
 template <typename T> struct Io;
 
 template <> struct Io<float> {
-  static constexpr int kBytes = 4;
-  static __device__ __forceinline__ void load8(const float *p, float (&x)[8]) {
+  static __device__ __forceinline__ void load8(const float *p, float2 (&x)[4]) {
     const float4 u = reinterpret_cast<const float4 *>(p)[0];
     const float4 w = reinterpret_cast<const float4 *>(p)[1];
-    x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
-    x[4] = w.x; x[5] = w.y; x[6] = w.z; x[7] = w.w;
+    x[0] = make_float2(u.x, u.y); x[1] = make_float2(u.z, u.w);
+    x[2] = make_float2(w.x, w.y); x[3] = make_float2(w.z, w.w);
   }
-  static __device__ __forceinline__ void store8(float *p, const float (&x)[8]) {
-    reinterpret_cast<float4 *>(p)[0] = make_float4(x[0], x[1], x[2], x[3]);
-    reinterpret_cast<float4 *>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
+  static __device__ __forceinline__ void load8_gate(const float *p, float2 (&x)[4]) {
+    load8(p, x);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = make_float2(fmaxf(x[i].x, -80.0f), fmaxf(x[i].y, -80.0f));
+  }
+  static __device__ __forceinline__ void store8(float *p, const float2 (&x)[4]) {
+    reinterpret_cast<float4 *>(p)[0] = make_float4(x[0].x, x[0].y, x[1].x, x[1].y);
+    reinterpret_cast<float4 *>(p)[1] = make_float4(x[2].x, x[2].y, x[3].x, x[3].y);
   }
 };
 
 template <> struct Io<__half> {
-  static constexpr int kBytes = 2;
-  static __device__ __forceinline__ void load8(const __half *p, float (&x)[8]) {
+  static __device__ __forceinline__ void load8(const __half *p, float2 (&x)[4]) {
     const uint4 u = *reinterpret_cast<const uint4 *>(p);
     const __half2 *h = reinterpret_cast<const __half2 *>(&u);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(h[i]);
-      x[2 * i] = f.x;
-      x[2 * i + 1] = f.y;
-    }
+    for (int i = 0; i < 4; ++i) x[i] = __half22float2(h[i]);
   }
-  static __device__ __forceinline__ void store8(__half *p, const float (&x)[8]) {
+  static __device__ __forceinline__ void load8_gate(const __half *p, float2 (&x)[4]) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+    const __half2 lo = __float2half2_rn(-80.0f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = __half22float2(__hmax2(h[i], lo));
+  }
+  static __device__ __forceinline__ void store8(__half *p, const float2 (&x)[4]) {
     uint4 u;
     __half2 *h = reinterpret_cast<__half2 *>(&u);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(x[2 * i], x[2 * i + 1]);
+    for (int i = 0; i < 4; ++i) h[i] = __float22half2_rn(x[i]);
     *reinterpret_cast<uint4 *>(p) = u;
   }
 };
 
 template <> struct Io<__nv_bfloat16> {
-  static constexpr int kBytes = 2;
-  static __device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&x)[8]) {
+  static __device__ __forceinline__ void load8(const __nv_bfloat16 *p, float2 (&x)[4]) {
     const uint4 u = *reinterpret_cast<const uint4 *>(p);
     const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __bfloat1622float2(h[i]);
-      x[2 * i] = f.x;
-      x[2 * i + 1] = f.y;
-    }
+    for (int i = 0; i < 4; ++i) x[i] = __bfloat1622float2(h[i]);
   }
-  static __device__ __forceinline__ void store8(__nv_bfloat16 *p, const float (&x)[8]) {
+  static __device__ __forceinline__ void load8_gate(const __nv_bfloat16 *p, float2 (&x)[4]) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+    const __nv_bfloat162 lo = __float2bfloat162_rn(-80.0f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = __bfloat1622float2(__hmax2(h[i], lo));
+  }
+  static __device__ __forceinline__ void store8(__nv_bfloat16 *p, const float2 (&x)[4]) {
     uint4 u;
     __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    for (int i = 0; i < 4; ++i) h[i] = __float22bfloat162_rn(x[i]);
     *reinterpret_cast<uint4 *>(p) = u;
   }
 };
@@ -148,22 +170,24 @@ __device__ __forceinline__ float rsqrt_approx(float x) {
 }
 
 // ---------------------------------------------------------------------------
-// Gate.  With u = exp(-x) = 2^(-x log2 e) (x clamped at -80 so u stays
-// finite):
+// Gate of a channel pair.  With u = exp(-x) = 2^(-x log2 e) (x already
+// clamped at -80 so u stays finite):
 //   A = 1 / (1 + u)      (the logistic sigmoid)
 //   1 - A = u * A        (no cancellation when A is close to 1)
 // ---------------------------------------------------------------------------
-struct Gate {
-  float A;    // sigmoid(x)
-  float Ac;   // 1 - sigmoid(x)
+struct Gate2 {
+  float2 A;    // sigmoid(x)
+  float2 Ac;   // 1 - sigmoid(x)
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-__device__ __forceinline__ Gate gate_of(float x) {
-  const float u = ex2_approx(fmaxf(x, -80.0f) * -kLog2e);
-  const float A = rcp_approx(1.0f + u);
-  return Gate{A, u * A};
+__device__ __forceinline__ Gate2 gate2(float2 x) {
+  const float2 t = mul2(x, splat(-kLog2e));
+  const float2 u = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+  const float2 d = add2(u, splat(1.0f));
+  const float2 A = make_float2(rcp_approx(d.x), rcp_approx(d.y));
+  return Gate2{A, mul2(u, A)};
 }
 
 // Sum over the `LPH` adjacent lanes that hold one head (LPH a power of two).

@@ -3,8 +3,9 @@
 //
 // Work decomposition (forward and backward):
 //   * A "chain" is one batch row b and one tile of CT consecutive channels
-//     (CT = 64, or D when the head dimension D is 128 or 256).  Heads never straddle
-//     a channel tile, so the per-head RMS readout stays inside one CTA.
+//     (CT = 64, or D when the head dimension D is 128 or 256).  Heads never
+//     straddle a channel tile, so the per-head RMS readout stays inside one
+//     CTA.
 //   * A chain is cut into time chunks of L steps.  A tile is one (chain,
 //     chunk); its a/v/q(/dy) boxes [L x CT] are staged in shared memory by TMA
 //     tensor loads (cp.async.bulk.tensor, no multicast).
@@ -81,7 +82,7 @@ struct TileCfg {
   static_assert(L % K == 0, "K must divide L");
   static_assert(NT % 32 == 0 && NT <= 1024, "bad block size");
   static_assert(RUNS % RW == 0, "runs must fill warps");
-  static_assert(CT % 32 == 0 && NT >= CT && CT >= 64, "look-back needs CT threads");
+  static_assert(CT % 32 == 0 && NT >= CT, "look-back needs CT threads");
   static_assert(RUNS * CT * sizeof(float2) <= kBoxBytes, "scan scratch must fit in the gate box");
   static_assert(VW % LPH == 0, "a head must stay inside a warp");
   static_assert(kBoxBytes % 128 == 0, "boxes must keep 128-byte alignment");
@@ -126,7 +127,8 @@ struct ThreadPos {
 // channels form a 64-byte block made of four 16-byte chunks; chunk q of vector
 // `vec` is stored at position (q + vec / 2) mod 4 so that the 16-byte accesses
 // of 8 consecutive vectors hit distinct banks, and the serial scan's 8-byte
-// accesses by consecutive channels stay conflict-free as well.
+// accesses by consecutive channels stay conflict-free as well.  Chunk q holds
+// channels 2q and 2q+1: (P, S) of the first, then (P, S) of the second.
 template <int CT>
 __device__ __forceinline__ int scan_pos(int run, int c) {
   const int vec = c >> 3, j = c & 7;
@@ -135,27 +137,25 @@ __device__ __forceinline__ int scan_pos(int run, int c) {
 }
 
 template <int CT>
-__device__ __forceinline__ void scan_store8(float2 *scan, int run, int ch, const float (&p)[8], const float (&s)[8]) {
+__device__ __forceinline__ void scan_store8(float2 *scan, int run, int ch, const float2 (&p)[4],
+                                            const float2 (&s)[4]) {
   const int vec = ch >> 3;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int chunk = (q + (vec >> 1)) & 3;
-    reinterpret_cast<float4 *>(scan + run * CT + ch + chunk * 2)[0] =
-        make_float4(p[2 * q], s[2 * q], p[2 * q + 1], s[2 * q + 1]);
+    reinterpret_cast<float4 *>(scan + run * CT + ch + chunk * 2)[0] = make_float4(p[q].x, s[q].x, p[q].y, s[q].y);
   }
 }
 
 template <int CT>
-__device__ __forceinline__ void scan_load8(const float2 *scan, int run, int ch, float (&p)[8], float (&s)[8]) {
+__device__ __forceinline__ void scan_load8(const float2 *scan, int run, int ch, float2 (&p)[4], float2 (&s)[4]) {
   const int vec = ch >> 3;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int chunk = (q + (vec >> 1)) & 3;
     const float4 u = reinterpret_cast<const float4 *>(scan + run * CT + ch + chunk * 2)[0];
-    p[2 * q] = u.x;
-    s[2 * q] = u.y;
-    p[2 * q + 1] = u.z;
-    s[2 * q + 1] = u.w;
+    p[q] = make_float2(u.x, u.z);
+    s[q] = make_float2(u.y, u.w);
   }
 }
 
@@ -164,18 +164,32 @@ __device__ __forceinline__ void scan_load8(const float2 *scan, int run, int ch, 
 // oldest run first; backward order: latest run first).
 template <int CT, int RUNS, bool kReverse>
 __device__ __forceinline__ float2 scan_runs(float2 *scan, int c) {
+  float2 *col = scan + scan_pos<CT>(0, c);
   float cp = 1.0f, cs = 0.0f;
-#pragma unroll 4
+#pragma unroll
   for (int k = 0; k < RUNS; ++k) {
     const int r = kReverse ? RUNS - 1 - k : k;
-    const int at = scan_pos<CT>(r, c);
-    const float2 e = scan[at];
-    scan[at] = make_float2(cp, cs);
+    const float2 e = col[r * CT];
+    col[r * CT] = make_float2(cp, cs);
     cs = __fmaf_rn(e.x, cs, e.y);
     cp = cp * e.x;
   }
   return make_float2(cp, cs);
 }
+
+// The run's carry-in for its 8 channels: prefix map (from the scratch)
+// applied to the tile's carry (es_s, one float per channel).
+template <int CT>
+__device__ __forceinline__ void run_carry(const float2 *scan, const float *es_s, int run, int ch, float2 (&E)[4]) {
+  float2 pe[4], se[4];
+  scan_load8<CT>(scan, run, ch, pe, se);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) E[q] = fma2(pe[q], reinterpret_cast<const float2 *>(es_s + ch)[q], se[q]);
+}
+
+// Sum of a channel-pair accumulator over the LPH lanes of one head.
+template <int LPH>
+__device__ __forceinline__ float head_sum2(float2 s) { return head_sum<LPH>(s.x + s.y); }
 
 // The carry entering chunk `slot` for channel `c`: the nearest predecessor
 // (distance 1, 2, ... in direction `dir`, at most `avail`) whose chunk-end
@@ -246,8 +260,10 @@ __device__ __forceinline__ float carry_in(const unsigned long long *incl, const 
       break;
     }
     if ((it & 63u) == 63u && ld_relaxed(abort_flag)) break;
-    __nanosleep(ns);
-    ns = ns < 256 ? ns * 2 : 256;
+    if (it >= 2) {   // the first re-polls go straight out: a round trip is already ~1 us
+      __nanosleep(ns);
+      ns = ns < 256 ? ns * 2 : 256;
+    }
   }
   atomicOr(status, kStatusTimeout);
   atomicExch(abort_flag, 1u);
@@ -294,22 +310,27 @@ __device__ __forceinline__ void scan_epilogue(WsHeader *hdr, int k, bool ran) {
   }
 }
 
-// Gate of one channel in the form the recurrence uses: direct keeps A,
-// controlled keeps 1 - A (no cancellation when A is close to 1).
+// Gate coefficients of a channel pair in the form the recurrence uses:
+// direct keeps A, controlled keeps 1 - A (no cancellation when A is near 1).
 template <int MODE>
-__device__ __forceinline__ float gate_coef(const Gate &g) { return MODE == 0 ? g.A : g.Ac; }
+__device__ __forceinline__ float2 gate_coef(const Gate2 &g) { return MODE == 0 ? g.A : g.Ac; }
 
-// One step of the recurrence with the stored gate coefficient `c`.
+// One step of the recurrence for a channel pair with stored coefficient c:
+// direct E' = c E + v; controlled E' = E + c (v - E).
 template <int MODE>
-__device__ __forceinline__ float rec_step(float c, float E, float v) {
-  return MODE == 0 ? __fmaf_rn(c, E, v) : __fmaf_rn(c, v - E, E);
+__device__ __forceinline__ float2 rec_step(float2 c, float2 E, float2 v) {
+  return MODE == 0 ? fma2(c, E, v) : fma2(c, sub2(v, E), E);
 }
+
+// A of the pair from its stored coefficient.
+template <int MODE>
+__device__ __forceinline__ float2 gate_A(float2 c) { return MODE == 0 ? c : sub2(splat(1.0f), c); }
 
 // ===========================================================================
 // Forward scan (persistent).
 // ===========================================================================
 template <typename T, int MODE, int LPH, int VPR, int L, int K>
-__global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 128) ? 4 : (VPR * (L / K) <= 256) ? 2 : 1)
+__global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR * (L / K) <= 128) ? 4 : (VPR * (L / K) <= 256) ? 2 : 1)
     esa_scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_q, const FwdArgs args) {
   using Cfg = TileCfg<T, LPH, VPR, L, K>;
@@ -383,24 +404,24 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 128) ? 4 : (VP
     phase ^= 1u << s;
 
     // ---- pass 1: gates and the run's affine map ---------------------------
-    float Ar[K][8];
-    float P[8], S[8];
+    float2 Ar[K][4];   // direct: A_t; controlled: 1 - A_t  (channel pairs)
+    float2 P[4], S[4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) { P[j] = 1.0f; S[j] = 0.0f; }
+    for (int q = 0; q < 4; ++q) { P[q] = splat(1.0f); S[q] = splat(0.0f); }
 #pragma unroll
     for (int i = 0; i < K; ++i) {
       const int r = pos.row0 + i;
       const bool valid = (t0 + r) < sh.T;
-      float x[8], vv[8];
-      Io<T>::load8(a_s + r * CT + pos.ch, x);
+      float2 x[4], vv[4];
+      Io<T>::load8_gate(a_s + r * CT + pos.ch, x);
       Io<T>::load8(v_s + r * CT + pos.ch, vv);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const Gate g = gate_of(x[j]);
-        Ar[i][j] = gate_coef<MODE>(g);
+      for (int q = 0; q < 4; ++q) {
+        const Gate2 g = gate2(x[q]);
+        Ar[i][q] = gate_coef<MODE>(g);
         if (valid) {
-          P[j] *= g.A;
-          S[j] = rec_step<MODE>(Ar[i][j], S[j], vv[j]);
+          P[q] = mul2(P[q], g.A);
+          S[q] = rec_step<MODE>(Ar[i][q], S[q], vv[q]);
         }
       }
     }
@@ -429,33 +450,27 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 128) ? 4 : (VP
     __syncthreads();
 
     // ---- pass 2: exact states and the readout ------------------------------
-    float E[8];
-    {
-      float pe[8], se[8];
-      scan_load8<CT>(scan_s, pos.run, pos.ch, pe, se);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) E[j] = __fmaf_rn(pe[j], es_s[pos.ch + j], se[j]);
-    }
+    float2 E[4];
+    run_carry<CT>(scan_s, es_s, pos.run, pos.ch, E);
     const bool ch_ok = (c0 + pos.ch) < sh.C;
     const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
 #pragma unroll
     for (int i = 0; i < K; ++i) {
       const int r = pos.row0 + i;
       const bool valid = (t0 + r) < sh.T;
-      float vv[8], qq[8];
+      float2 vv[4], qq[4];
       Io<T>::load8(v_s + r * CT + pos.ch, vv);
       Io<T>::load8(q_s + r * CT + pos.ch, qq);
-      float ss = 0.0f;
+      float2 ss = splat(0.0f);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        E[j] = rec_step<MODE>(Ar[i][j], E[j], vv[j]);
-        ss = __fmaf_rn(E[j], E[j], ss);
+      for (int q = 0; q < 4; ++q) {
+        E[q] = rec_step<MODE>(Ar[i][q], E[q], vv[q]);
+        ss = fma2(E[q], E[q], ss);
       }
-      ss = head_sum<LPH>(ss);
-      const float rr = rsqrt_approx(__fmaf_rn(ss, sh.inv_D, kEps));
-      float yv[8];
+      const float rr = rsqrt_approx(__fmaf_rn(head_sum2<LPH>(ss), sh.inv_D, kEps));
+      float2 yv[4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) yv[j] = qq[j] * (E[j] * rr);
+      for (int q = 0; q < 4; ++q) yv[q] = mul2(qq[q], mul2(E[q], splat(rr)));
       if (valid && ch_ok) Io<T>::store8(yg + gbase + static_cast<long>(r) * sh.C, yv);
     }
 
@@ -475,35 +490,27 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 128) ? 4 : (VP
 // ghat (8 float32) of one thread's row, kept in that row's q and dy slots:
 // 16-bit I/O splits it over both 16-byte slots; float32 I/O uses the q slot.
 template <typename T>
-__device__ __forceinline__ void put_ghat(T *q_slot, T *dy_slot, const float (&g)[8]) {
-  if (sizeof(T) == 2) {
-    reinterpret_cast<float4 *>(q_slot)[0] = make_float4(g[0], g[1], g[2], g[3]);
-    reinterpret_cast<float4 *>(dy_slot)[0] = make_float4(g[4], g[5], g[6], g[7]);
-  } else {
-    reinterpret_cast<float4 *>(q_slot)[0] = make_float4(g[0], g[1], g[2], g[3]);
-    reinterpret_cast<float4 *>(q_slot)[1] = make_float4(g[4], g[5], g[6], g[7]);
-  }
+__device__ __forceinline__ void put_ghat(T *q_slot, T *dy_slot, const float2 (&g)[4]) {
+  float4 *lo = reinterpret_cast<float4 *>(q_slot);
+  float4 *hi = sizeof(T) == 2 ? reinterpret_cast<float4 *>(dy_slot) : lo + 1;
+  lo[0] = make_float4(g[0].x, g[0].y, g[1].x, g[1].y);
+  hi[0] = make_float4(g[2].x, g[2].y, g[3].x, g[3].y);
 }
 
 template <typename T>
-__device__ __forceinline__ void get_ghat(const T *q_slot, const T *dy_slot, float (&g)[8]) {
-  float4 u, w;
-  if (sizeof(T) == 2) {
-    u = reinterpret_cast<const float4 *>(q_slot)[0];
-    w = reinterpret_cast<const float4 *>(dy_slot)[0];
-  } else {
-    u = reinterpret_cast<const float4 *>(q_slot)[0];
-    w = reinterpret_cast<const float4 *>(q_slot)[1];
-  }
-  g[0] = u.x; g[1] = u.y; g[2] = u.z; g[3] = u.w;
-  g[4] = w.x; g[5] = w.y; g[6] = w.z; g[7] = w.w;
+__device__ __forceinline__ void get_ghat(const T *q_slot, const T *dy_slot, float2 (&g)[4]) {
+  const float4 *lo = reinterpret_cast<const float4 *>(q_slot);
+  const float4 *hi = sizeof(T) == 2 ? reinterpret_cast<const float4 *>(dy_slot) : lo + 1;
+  const float4 u = lo[0], w = hi[0];
+  g[0] = make_float2(u.x, u.y); g[1] = make_float2(u.z, u.w);
+  g[2] = make_float2(w.x, w.y); g[3] = make_float2(w.z, w.w);
 }
 
 // ===========================================================================
 // Backward scan (persistent).
 // ===========================================================================
 template <typename T, int MODE, int LPH, int VPR, int L, int K>
-__global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 128) ? 4 : (VPR * (L / K) <= 256) ? 2 : 1)
+__global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR * (L / K) <= 128) ? 4 : (VPR * (L / K) <= 256) ? 2 : 1)
     esa_scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dy,
                         const BwdArgs args) {
@@ -608,24 +615,24 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 128) ? 4 : (VP
     phase ^= 1u << s;
 
     // ---- F1: gates and the run's forward map ------------------------------
-    float Ar[K][8];
-    float P[8], S[8];
+    float2 Ar[K][4];
+    float2 P[4], S[4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) { P[j] = 1.0f; S[j] = 0.0f; }
+    for (int q = 0; q < 4; ++q) { P[q] = splat(1.0f); S[q] = splat(0.0f); }
 #pragma unroll
     for (int i = 0; i < K; ++i) {
       const int r = pos.row0 + i;
       const bool valid = (t0 + r) < sh.T;
-      float x[8], vv[8];
-      Io<T>::load8(a_s + r * CT + pos.ch, x);
+      float2 x[4], vv[4];
+      Io<T>::load8_gate(a_s + r * CT + pos.ch, x);
       Io<T>::load8(v_s + r * CT + pos.ch, vv);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const Gate g = gate_of(x[j]);
-        Ar[i][j] = gate_coef<MODE>(g);
+      for (int q = 0; q < 4; ++q) {
+        const Gate2 g = gate2(x[q]);
+        Ar[i][q] = gate_coef<MODE>(g);
         if (valid) {
-          P[j] *= g.A;
-          S[j] = rec_step<MODE>(Ar[i][j], S[j], vv[j]);
+          P[q] = mul2(P[q], g.A);
+          S[q] = rec_step<MODE>(Ar[i][q], S[q], vv[q]);
         }
       }
     }
@@ -638,48 +645,43 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 128) ? 4 : (VP
 
     // ---- F2: replay states, readout backward, dq, ghat ---------------------
     // ghat of each row overwrites that row's q/dy slots (only this thread
-    // reads them); w keeps what da needs of the previous state.
-    float w[K][8];   // direct: E_{t-1}; controlled: E_{t-1} - v_t
+    // reads them again).
+    float2 Ec[4];   // the run's forward carry-in, kept for the da sweep
+    run_carry<CT>(scan_s, es_s, pos.run, pos.ch, Ec);
+    mbar_wait_bounded(&bar[2], (phase >> 2) & 1u, &hdr->status);
+    phase ^= 4u;
     {
-      float E[8];
-      {
-        float pe[8], se[8];
-        scan_load8<CT>(scan_s, pos.run, pos.ch, pe, se);
+      float2 E[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) E[j] = __fmaf_rn(pe[j], es_s[pos.ch + j], se[j]);
-      }
-      mbar_wait_bounded(&bar[2], (phase >> 2) & 1u, &hdr->status);
-      phase ^= 4u;
+      for (int q = 0; q < 4; ++q) E[q] = Ec[q];
 #pragma unroll
       for (int i = 0; i < K; ++i) {
         const int r = pos.row0 + i;
         const bool valid = (t0 + r) < sh.T;
-        float vv[8], qq[8], gg[8];
+        float2 vv[4], qq[4], gg[4];
         Io<T>::load8(v_s + r * CT + pos.ch, vv);
         Io<T>::load8(q_s + r * CT + pos.ch, qq);
         Io<T>::load8(dy_s + r * CT + pos.ch, gg);
-        float ss = 0.0f;
+        float2 ss = splat(0.0f);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          w[i][j] = (MODE == 0) ? E[j] : E[j] - vv[j];
-          E[j] = rec_step<MODE>(Ar[i][j], E[j], vv[j]);
-          ss = __fmaf_rn(E[j], E[j], ss);
+        for (int q = 0; q < 4; ++q) {
+          E[q] = rec_step<MODE>(Ar[i][q], E[q], vv[q]);
+          ss = fma2(E[q], E[q], ss);
         }
-        ss = head_sum<LPH>(ss);
-        const float rr = rsqrt_approx(__fmaf_rn(ss, sh.inv_D, kEps));
-        float nn[8], dn[8], dqv[8];
-        float dot = 0.0f;
+        const float rr = rsqrt_approx(__fmaf_rn(head_sum2<LPH>(ss), sh.inv_D, kEps));
+        float2 nn[4], dn[4], dqv[4];
+        float2 dot2 = splat(0.0f);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          nn[j] = E[j] * rr;
-          dn[j] = gg[j] * qq[j];
-          dqv[j] = gg[j] * nn[j];
-          dot = __fmaf_rn(dn[j], nn[j], dot);
+        for (int q = 0; q < 4; ++q) {
+          nn[q] = mul2(E[q], splat(rr));
+          dn[q] = mul2(gg[q], qq[q]);
+          dqv[q] = mul2(gg[q], nn[q]);
+          dot2 = fma2(dn[q], nn[q], dot2);
         }
-        dot = head_sum<LPH>(dot) * sh.inv_D;
-        float gh[8];
+        const float dot = head_sum2<LPH>(dot2) * sh.inv_D;
+        float2 gh[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) gh[j] = rr * __fmaf_rn(-nn[j], dot, dn[j]);
+        for (int q = 0; q < 4; ++q) gh[q] = mul2(splat(rr), fma2(nn[q], splat(-dot), dn[q]));
         put_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
         if (valid && (c0 + pos.ch) < sh.C)
           Io<T>::store8(dqg + (static_cast<long>(b) * sh.T + t0 + r) * sh.C + c0 + pos.ch, dqv);
@@ -688,20 +690,17 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 128) ? 4 : (VP
 
     // ---- R1: the run's reverse map h -> P h + hl ----------------------------
     {
-      float hl[8];
+      float2 hl[4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) hl[j] = 0.0f;
+      for (int q = 0; q < 4; ++q) hl[q] = splat(0.0f);
 #pragma unroll
       for (int i = K - 1; i >= 0; --i) {
         const int r = pos.row0 + i;
         if ((t0 + r) < sh.T) {
-          float gh[8];
+          float2 gh[4];
           get_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float A = (MODE == 0) ? Ar[i][j] : 1.0f - Ar[i][j];
-            hl[j] = A * (gh[j] + hl[j]);
-          }
+          for (int q = 0; q < 4; ++q) hl[q] = mul2(gate_A<MODE>(Ar[i][q]), add2(gh[q], hl[q]));
         }
       }
       __syncthreads();   // every thread has read its forward prefixes
@@ -730,45 +729,52 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 128) ? 4 : (VP
     }
     __syncthreads();
 
-    // ---- B: total gradient G_t and da, dv, latest step first -----------------
+    // ---- B1: total gradient G_t (latest step first): dv, and the da factor -
+    // G A (1 - A) replaces ghat in the row's slots.
+    const bool ch_ok = (c0 + pos.ch) < sh.C;
+    const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
     {
-      float h[8];
-      {
-        float pe[8], se[8];
-        scan_load8<CT>(scan_s, pos.run, pos.ch, pe, se);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) h[j] = __fmaf_rn(pe[j], es_s[pos.ch + j], se[j]);
-      }
-      const bool ch_ok = (c0 + pos.ch) < sh.C;
-      const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
+      float2 h[4];
+      run_carry<CT>(scan_s, es_s, pos.run, pos.ch, h);
 #pragma unroll
       for (int i = K - 1; i >= 0; --i) {
         const int r = pos.row0 + i;
         if ((t0 + r) < sh.T) {
-          float gh[8], dav[8], dvv[8];
+          float2 gh[4], dvv[4];
           get_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float G = gh[j] + h[j];
-            if (MODE == 0) {
-              const float A = Ar[i][j];
-              dvv[j] = G;
-              dav[j] = G * w[i][j] * (A * (1.0f - A));
-              h[j] = A * G;
-            } else {
-              const float Ac = Ar[i][j];
-              const float A = 1.0f - Ac;
-              dvv[j] = G * Ac;
-              dav[j] = G * w[i][j] * (A * Ac);
-              h[j] = A * G;
-            }
+          for (int q = 0; q < 4; ++q) {
+            const float2 G = add2(gh[q], h[q]);
+            const float2 A = gate_A<MODE>(Ar[i][q]);
+            const float2 Ac = (MODE == 0) ? sub2(splat(1.0f), A) : Ar[i][q];
+            dvv[q] = (MODE == 0) ? G : mul2(G, Ac);
+            gh[q] = mul2(G, mul2(A, Ac));
+            h[q] = mul2(A, G);
           }
-          if (ch_ok) {
-            const long off = gbase + static_cast<long>(r) * sh.C;
-            Io<T>::store8(dag + off, dav);
-            Io<T>::store8(dvg + off, dvv);
-          }
+          put_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
+          if (ch_ok) Io<T>::store8(dvg + gbase + static_cast<long>(r) * sh.C, dvv);
         }
+      }
+    }
+
+    // ---- B2: replay states forward: da = G A (1 - A) (E_{t-1} - v_t) --------
+    //      (direct mode: times E_{t-1})
+    {
+      float2 E[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) E[q] = Ec[q];
+#pragma unroll
+      for (int i = 0; i < K; ++i) {
+        const int r = pos.row0 + i;
+        float2 vv[4], ga[4], dav[4];
+        Io<T>::load8(v_s + r * CT + pos.ch, vv);
+        get_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, ga);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          dav[q] = mul2(ga[q], (MODE == 0) ? E[q] : sub2(E[q], vv[q]));
+          E[q] = rec_step<MODE>(Ar[i][q], E[q], vv[q]);
+        }
+        if ((t0 + r) < sh.T && ch_ok) Io<T>::store8(dag + gbase + static_cast<long>(r) * sh.C, dav);
       }
     }
 
@@ -793,28 +799,26 @@ __global__ void __launch_bounds__(256)
                     float *__restrict__ E, T *__restrict__ y, long nvec, float inv_D) {
   const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const bool act = idx < nvec;
-  float x[8], vv[8], qq[8], e[8];
+  float2 x[4], vv[4], qq[4], e[4];
   if (act) {
-    Io<T>::load8(a + idx * 8, x);
+    Io<T>::load8_gate(a + idx * 8, x);
     Io<T>::load8(v + idx * 8, vv);
     Io<T>::load8(q + idx * 8, qq);
     Io<float>::load8(E + idx * 8, e);
   } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) { x[j] = 0.0f; vv[j] = 0.0f; qq[j] = 0.0f; e[j] = 0.0f; }
+    for (int i = 0; i < 4; ++i) { x[i] = splat(0.0f); vv[i] = splat(0.0f); qq[i] = splat(0.0f); e[i] = splat(0.0f); }
   }
-  float ss = 0.0f;
+  float2 ss = splat(0.0f);
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const Gate g = gate_of(x[j]);
-    e[j] = rec_step<MODE>(gate_coef<MODE>(g), e[j], vv[j]);
-    ss = __fmaf_rn(e[j], e[j], ss);
+  for (int i = 0; i < 4; ++i) {
+    e[i] = rec_step<MODE>(gate_coef<MODE>(gate2(x[i])), e[i], vv[i]);
+    ss = fma2(e[i], e[i], ss);
   }
-  ss = head_sum<LPH>(ss);
-  const float rr = rsqrt_approx(__fmaf_rn(ss, inv_D, kEps));
-  float yv[8];
+  const float rr = rsqrt_approx(__fmaf_rn(head_sum2<LPH>(ss), inv_D, kEps));
+  float2 yv[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) yv[j] = qq[j] * (e[j] * rr);
+  for (int i = 0; i < 4; ++i) yv[i] = mul2(qq[i], mul2(e[i], splat(rr)));
   if (act) {
     Io<float>::store8(E + idx * 8, e);
     Io<T>::store8(y + idx * 8, yv);
