@@ -124,7 +124,7 @@ int esa_scan_fwd(const void *a, const void *v, const void *q, void *y, float *E_
  *             the chunk-boundary states in it are read, the rest is scratch.
  * The pages do not print the backward; it is the chain rule of the forward
  * (training through the layer with loss.backward(), "Entangled State
- * Attention v2.1", Trainer section):
+ * Attention v2.1", section 9 "Continue training a loaded model"):
  *   G_t = ghat_t + A_{t+1} G_{t+1}, G_T = ghat_T + dE_final,
  *   ghat_t = r (dn - n mean_d(dn n)), n = E r, dn = dy q, dq = dy n,
  *   direct: dv = G, da = G E_{t-1} A(1-A);

@@ -34,7 +34,8 @@
  *   - State shape [B, H, D], prompt length not a dimension of it:
  *     mlbricks-web.pages.dev/esa, "Generation / memory", "State shape".
  *   - The backward pass is not printed on any page; training through the
- *     layer (loss.backward() in the v2.1 Trainer section) implies it.  It is
+ *     layer (loss.backward() in "Entangled State Attention v2.1", section 9
+ *     "Continue training a loaded model") implies it.  It is
  *     derived here by the chain rule from the forward definition above:
  *       n = E r,  dq = dy n,  dn = dy q,
  *       ghat_t = r (dn - n * mean_d(dn n))          (gradient into E_t via y_t)
