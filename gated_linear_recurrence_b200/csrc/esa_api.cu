@@ -312,6 +312,8 @@ const char *esa_strerror(int status) {
     case ESA_ERR_LAUNCH: return "the CUDA runtime rejected a launch, copy or tensor map";
     case ESA_ERR_TIMEOUT: return "a bounded device-side wait gave up; outputs of the call are invalid";
     case ESA_ERR_DEVICE: return "no CUDA device, or the current device is not sm_100 (B200)";
+    case ESA_ERR_NOALLOC_LIMIT:
+      return "esa_scan_fwd_noalloc: the shape needs more scratch than the built-in 64 MiB array";
     default: return "unknown esa status";
   }
 }

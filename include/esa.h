@@ -63,7 +63,9 @@ typedef enum {
     ESA_ERR_WORKSPACE = -4,   /* workspace NULL, too small, or not initialised (esa_workspace_init) */
     ESA_ERR_LAUNCH = -5,      /* the CUDA runtime rejected a launch or copy */
     ESA_ERR_TIMEOUT = -6,     /* a bounded device-side wait gave up (see esa_check) */
-    ESA_ERR_DEVICE = -7       /* no CUDA device, or the current device is not sm_100 */
+    ESA_ERR_DEVICE = -7,      /* no CUDA device, or the current device is not sm_100 */
+    ESA_ERR_NOALLOC_LIMIT = -8 /* esa_scan_fwd_noalloc: the shape needs more scratch than
+                                  ESA_NOALLOC_SCRATCH_BYTES */
 } esa_status;
 
 /*
@@ -134,6 +136,35 @@ int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy,
                  const float *dE_final, void *da, void *dv, void *dq, float *dE_init,
                  int B, int T, int H, int D, int mode, const float *E_init,
                  int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Forward scan that allocates nothing.  The pages have no counterpart of this
+ * entry point; it exists for callers that cannot allocate device memory at
+ * the point where they run the scan -- serving loops whose device-memory
+ * budget is fixed at start-up, latency-critical paths where cudaMalloc may
+ * implicitly synchronise the device, and foreign-language callers that are
+ * only handed tensor pointers and own no device allocator.
+ *
+ * Same arguments and results as esa_scan_fwd, minus the workspace: the
+ * scratch lives in a static device array of ESA_NOALLOC_SCRATCH_BYTES
+ * (64 MiB) inside the library, which every GPU that loads this part of the
+ * library holds until the process exits.
+ *   - A shape whose esa_workspace_size() exceeds ESA_NOALLOC_SCRATCH_BYTES is
+ *     rejected with ESA_ERR_NOALLOC_LIMIT before anything is enqueued (for
+ *     example B=64, T=8192, C=128 in 16-bit I/O needs 33.6 MB and fits).
+ *   - The first call on a device sets the array up with that device current
+ *     (looks up its device address, zeroes it) and synchronises `stream`
+ *     once; make that first call before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents
+ *     (the chunk carries are tagged with a per-call epoch, so nothing needs
+ *     clearing between calls).  Calls whose executions overlap on the GPU,
+ *     from any stream or thread, race on it: order them.  The chunk-end
+ *     states it holds are not kept for a backward pass.
+ */
+#define ESA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int esa_scan_fwd_noalloc(const void *a, const void *v, const void *q, void *y, float *E_final,
+                         int B, int T, int H, int D, int mode, const float *E_init,
+                         int dtype, void *stream);
 
 /*
  * One-token recurrent update (decode): E <- A (.) E + B in place, then
