@@ -177,6 +177,32 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# Multi-rank helpers (weak scaling: every rank runs its own batch).
+# ---------------------------------------------------------------------------
+
+def rank_seed(w, rank):
+    """Seed of rank `rank`'s independent batch of workload `w`."""
+    return w.seed + 17 * rank
+
+
+def max_over_ranks(x, world, device):
+    """Max of a per-rank float over all ranks (identity when world == 1)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def tokens_per_second(world, B, T, steps, elapsed_ms):
+    """Whole-job throughput: every rank processed steps * B * T tokens in the
+    slowest rank's elapsed time."""
+    return world * B * T * steps / (elapsed_ms / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle legs (the oracle is test infrastructure; only these legs use it).
 # ---------------------------------------------------------------------------
 
@@ -256,16 +282,9 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     w = workload(args.batch, args.seq)
     B, T, H, D, mode = w.B, w.T, w.H, w.D, w.mode
-    x = inputs.make_scan_inputs(B, T, H, D, w.dtype, w.a_mean, w.seed + 17 * rank, device=dev)
+    x = inputs.make_scan_inputs(B, T, H, D, w.dtype, w.a_mean, rank_seed(w, rank), device=dev)
     a, v, q, dy = x["a"], x["v"], x["q"], x["dy"]
     y = torch.empty_like(a)
     da, dv, dq = torch.empty_like(a), torch.empty_like(a), torch.empty_like(a)
@@ -302,10 +321,10 @@ def run_ours(args):
     barrier()
     clk = clocks.stop()
     esa.esa_check(ws)
-    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    value = world * B * T * K / (elapsed_ms / 1e3)
+    value = tokens_per_second(world, B, T, K, elapsed_ms)
 
     s = a.element_size()
     C = H * D
@@ -356,11 +375,11 @@ def run_ours(args):
         torch.cuda.synchronize()
         barrier()
         esa.esa_check(ws)
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         h2d = sum(t.numel() * t.element_size() for t in h_in.values())
         d2h = sum(t.numel() * t.element_size() for t in h_out.values()) + \
             sum(t.numel() * t.element_size() for t in h_st.values())
-        e2e = {"value": world * tokens * K2 / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": tokens_per_second(world, B, T, K2, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": K2,
                "path": "pinned host -> esa_scan_fwd -> esa_scan_bwd -> pinned host, one stream, device-timed"}
         del h_in, h_out, h_st, d_in
