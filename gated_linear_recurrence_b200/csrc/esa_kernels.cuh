@@ -64,6 +64,39 @@ struct BwdArgs {
   Workspace ws;
 };
 
+// Coordinates of one tile, decoded once by the thread that takes its ticket
+// and published to the CTA in shared memory next to the tile's stage.
+struct TileInfo {
+  int tile;     // ticket (>= ntiles: no more work)
+  int chunk;    // time chunk
+  int b;        // batch row
+  int c0;       // first channel of the tile
+  int t0;       // first time step of the tile
+  int pad;
+  long slot;    // chain * nchunks + chunk
+};
+
+// kReverse: chunks in processing order run from the last to the first.
+template <bool kReverse>
+__device__ __forceinline__ TileInfo decode_tile(int tile, const ScanShape &sh, int CT, int L) {
+  TileInfo t;
+  t.tile = tile;
+  t.pad = 0;
+  if (tile >= sh.ntiles) {
+    t.chunk = t.b = t.c0 = t.t0 = 0;
+    t.slot = 0;
+    return t;
+  }
+  const int chain = tile % sh.nchains;
+  const int k = tile / sh.nchains;
+  t.chunk = kReverse ? sh.nchunks - 1 - k : k;
+  t.b = chain / sh.nct;
+  t.c0 = (chain % sh.nct) * CT;
+  t.t0 = t.chunk * L;
+  t.slot = static_cast<long>(chain) * sh.nchunks + t.chunk;
+  return t;
+}
+
 // Compile-time tile geometry.
 template <typename T, int LPH_, int VPR_, int L_, int K_>
 struct TileCfg {
@@ -92,7 +125,7 @@ struct TileCfg {
 template <typename Cfg>
 struct FwdSmem {
   static constexpr size_t kStage = 3 * size_t(Cfg::kBoxBytes);
-  static constexpr size_t kMisc = Cfg::CT * sizeof(float) + 64;
+  static constexpr size_t kMisc = Cfg::CT * sizeof(float) + 128;
   static constexpr size_t kBytes = 2 * kStage + kMisc + 128;   // +128 for alignment
 };
 
@@ -101,12 +134,18 @@ template <typename Cfg>
 struct BwdSmem {
   static constexpr size_t kStage = 2 * size_t(Cfg::kBoxBytes);
   static constexpr size_t kQdy = 2 * size_t(Cfg::kBoxBytes);
-  static constexpr size_t kMisc = Cfg::CT * sizeof(float) + 64;
+  static constexpr size_t kMisc = Cfg::CT * sizeof(float) + 128;
   static constexpr size_t kBytes = 2 * kStage + kQdy + kMisc + 128;
 };
 
-__device__ __forceinline__ unsigned char *align128(unsigned char *p) {
-  return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(p) + 127) & ~uintptr_t(127));
+// The first 128-byte-aligned byte of the dynamic shared memory.  The offset
+// is computed on the 32-bit shared-window address and applied to the
+// __shared__ array itself, so the compiler keeps shared-space addressing
+// (a round trip through a generic integer address would turn every later
+// access into a generic one).
+__device__ __forceinline__ unsigned char *smem_aligned128(unsigned char *smem) {
+  const uint32_t a = smem_u32(smem);
+  return smem + (((a + 127u) & ~127u) - a);
 }
 
 // Per-thread coordinates inside a tile.
@@ -123,39 +162,40 @@ struct ThreadPos {
   }
 };
 
-// Run-scan scratch: float2 (map P, S) per (run, channel).  A thread's 8
-// channels form a 64-byte block made of four 16-byte chunks; chunk q of vector
-// `vec` is stored at position (q + vec / 2) mod 4 so that the 16-byte accesses
-// of 8 consecutive vectors hit distinct banks, and the serial scan's 8-byte
-// accesses by consecutive channels stay conflict-free as well.  Chunk q holds
-// channels 2q and 2q+1: (P, S) of the first, then (P, S) of the second.
+// Run-scan scratch: the map (P, S) per (run, channel), as floats.  A
+// thread's 8 channels form a 64-byte block of four 16-byte chunks; chunk q
+// holds (P, P, S, S) of channels 2q and 2q+1 (register-adjacent pairs for the
+// packed instructions) and is stored at position (q + vec / 2) mod 4 of its
+// vector's block, so the 16-byte accesses of 8 consecutive vectors hit
+// distinct banks.
 template <int CT>
-__device__ __forceinline__ int scan_pos(int run, int c) {
+__device__ __forceinline__ int scan_pos(int run, int c) {   // float index of P; S is 2 floats on
   const int vec = c >> 3, j = c & 7;
   const int chunk = ((j >> 1) + (vec >> 1)) & 3;
-  return run * CT + vec * 8 + chunk * 2 + (j & 1);
+  return run * CT * 2 + vec * 16 + chunk * 4 + (j & 1);
 }
 
 template <int CT>
-__device__ __forceinline__ void scan_store8(float2 *scan, int run, int ch, const float2 (&p)[4],
+__device__ __forceinline__ void scan_store8(float *scan, int run, int ch, const float2 (&p)[4],
                                             const float2 (&s)[4]) {
   const int vec = ch >> 3;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int chunk = (q + (vec >> 1)) & 3;
-    reinterpret_cast<float4 *>(scan + run * CT + ch + chunk * 2)[0] = make_float4(p[q].x, s[q].x, p[q].y, s[q].y);
+    reinterpret_cast<float4 *>(scan + run * CT * 2 + vec * 16 + chunk * 4)[0] =
+        make_float4(p[q].x, p[q].y, s[q].x, s[q].y);
   }
 }
 
 template <int CT>
-__device__ __forceinline__ void scan_load8(const float2 *scan, int run, int ch, float2 (&p)[4], float2 (&s)[4]) {
+__device__ __forceinline__ void scan_load8(const float *scan, int run, int ch, float2 (&p)[4], float2 (&s)[4]) {
   const int vec = ch >> 3;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int chunk = (q + (vec >> 1)) & 3;
-    const float4 u = reinterpret_cast<const float4 *>(scan + run * CT + ch + chunk * 2)[0];
-    p[q] = make_float2(u.x, u.z);
-    s[q] = make_float2(u.y, u.w);
+    const float4 u = reinterpret_cast<const float4 *>(scan + run * CT * 2 + vec * 16 + chunk * 4)[0];
+    p[q] = make_float2(u.x, u.y);
+    s[q] = make_float2(u.z, u.w);
   }
 }
 
@@ -163,16 +203,17 @@ __device__ __forceinline__ void scan_load8(const float2 *scan, int run, int ch, 
 // entry by the exclusive prefix and returns the tile map (forward order:
 // oldest run first; backward order: latest run first).
 template <int CT, int RUNS, bool kReverse>
-__device__ __forceinline__ float2 scan_runs(float2 *scan, int c) {
-  float2 *col = scan + scan_pos<CT>(0, c);
+__device__ __forceinline__ float2 scan_runs(float *scan, int c) {
+  float *col = scan + scan_pos<CT>(0, c);
   float cp = 1.0f, cs = 0.0f;
 #pragma unroll
   for (int k = 0; k < RUNS; ++k) {
     const int r = kReverse ? RUNS - 1 - k : k;
-    const float2 e = col[r * CT];
-    col[r * CT] = make_float2(cp, cs);
-    cs = __fmaf_rn(e.x, cs, e.y);
-    cp = cp * e.x;
+    const float ep = col[r * CT * 2], es = col[r * CT * 2 + 2];
+    col[r * CT * 2] = cp;
+    col[r * CT * 2 + 2] = cs;
+    cs = __fmaf_rn(ep, cs, es);
+    cp = cp * ep;
   }
   return make_float2(cp, cs);
 }
@@ -180,7 +221,7 @@ __device__ __forceinline__ float2 scan_runs(float2 *scan, int c) {
 // The run's carry-in for its 8 channels: prefix map (from the scratch)
 // applied to the tile's carry (es_s, one float per channel).
 template <int CT>
-__device__ __forceinline__ void run_carry(const float2 *scan, const float *es_s, int run, int ch, float2 (&E)[4]) {
+__device__ __forceinline__ void run_carry(const float *scan, const float *es_s, int run, int ch, float2 (&E)[4]) {
   float2 pe[4], se[4];
   scan_load8<CT>(scan, run, ch, pe, se);
 #pragma unroll
@@ -338,11 +379,11 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
   constexpr int CT = Cfg::CT, RUNS = Cfg::RUNS;
 
   extern __shared__ unsigned char smem_raw[];
-  unsigned char *base = align128(smem_raw);
+  unsigned char *base = smem_aligned128(smem_raw);
   float *es_s = reinterpret_cast<float *>(base + 2 * Sm::kStage);
   uint64_t *bar = reinterpret_cast<uint64_t *>(es_s + CT);     // [2]
-  int *ticket_s = reinterpret_cast<int *>(bar + 2);            // [2]
-  unsigned *tag_s = reinterpret_cast<unsigned *>(ticket_s + 2);
+  TileInfo *info_s = reinterpret_cast<TileInfo *>(bar + 2);    // [2], per stage
+  unsigned *tag_s = reinterpret_cast<unsigned *>(info_s + 2);
 
   const int tid = threadIdx.x;
   const ScanShape &sh = args.s;
@@ -352,13 +393,15 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
   auto box = [&](int stage, int k) -> T * {
     return reinterpret_cast<T *>(base + stage * Sm::kStage + k * size_t(Cfg::kBoxBytes));
   };
+  // Thread 0: decode a ticket into the stage's tile info and start its loads.
   auto issue = [&](int stage, int tile) {
-    const int chain = tile % sh.nchains, chunk = tile / sh.nchains;
-    const int c0 = (chain % sh.nct) * CT, b = chain / sh.nct, t0 = chunk * L;
+    const TileInfo ti = decode_tile<false>(tile, sh, CT, L);
+    info_s[stage] = ti;
+    if (tile >= sh.ntiles) return;
     mbar_expect_tx(&bar[stage], 3 * Cfg::kBoxBytes);
-    tma_load_3d(box(stage, 0), &tm_a, c0, t0, b, &bar[stage]);
-    tma_load_3d(box(stage, 1), &tm_v, c0, t0, b, &bar[stage]);
-    tma_load_3d(box(stage, 2), &tm_q, c0, t0, b, &bar[stage]);
+    tma_load_3d(box(stage, 0), &tm_a, ti.c0, ti.t0, ti.b, &bar[stage]);
+    tma_load_3d(box(stage, 1), &tm_v, ti.c0, ti.t0, ti.b, &bar[stage]);
+    tma_load_3d(box(stage, 2), &tm_q, ti.c0, ti.t0, ti.b, &bar[stage]);
   };
 
   if (tid == 0) {
@@ -373,10 +416,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     *tag_s = tag;
     const int t0 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[0], 1u)) : sh.ntiles;
     const int t1 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[0], 1u)) : sh.ntiles;
-    ticket_s[0] = t0;
-    ticket_s[1] = t1;
-    if (t0 < sh.ntiles) issue(0, t0);
-    if (t1 < sh.ntiles) issue(1, t1);
+    issue(0, t0);
+    issue(1, t1);
   }
   __syncthreads();
 
@@ -387,18 +428,16 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
 
   for (int it = 0;; ++it) {
     const int s = it & 1;
-    const int tile = ticket_s[s];
-    if (tile >= sh.ntiles) break;
+    const TileInfo ti = info_s[s];
+    if (ti.tile >= sh.ntiles) break;
     unsigned next = 0;
     if (tid == 0) next = atomicAdd(&hdr->ticket[0], 1u);   // the tile that will refill this stage
-
-    const int chain = tile % sh.nchains, chunk = tile / sh.nchains;
-    const int b = chain / sh.nct, c0 = (chain % sh.nct) * CT, t0 = chunk * L;
-    const long slot = static_cast<long>(chain) * sh.nchunks + chunk;
+    const int chunk = ti.chunk, b = ti.b, c0 = ti.c0, t0 = ti.t0;
+    const long slot = ti.slot;
     const T *a_s = box(s, 0);
     const T *v_s = box(s, 1);
     const T *q_s = box(s, 2);
-    float2 *scan_s = reinterpret_cast<float2 *>(box(s, 0));   // reused once pass 1 is done
+    float *scan_s = reinterpret_cast<float *>(box(s, 0));   // reused once pass 1 is done
 
     mbar_wait_bounded(&bar[s], (phase >> s) & 1u, &hdr->status);
     phase ^= 1u << s;
@@ -477,11 +516,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     // ---- refill this stage --------------------------------------------------
     __syncthreads();   // everybody is done with stage s
     if (tid == 0) {
-      ticket_s[s] = static_cast<int>(next);
-      if (static_cast<int>(next) < sh.ntiles) {
-        fence_proxy_async_smem();   // generic writes (scan scratch) before the async refill
-        issue(s, static_cast<int>(next));
-      }
+      fence_proxy_async_smem();   // generic writes (scan scratch) before the async refill
+      issue(s, static_cast<int>(next));
     }
   }
   scan_epilogue(hdr, 0, tag != 0u);
@@ -519,13 +555,13 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
   constexpr int CT = Cfg::CT, RUNS = Cfg::RUNS;
 
   extern __shared__ unsigned char smem_raw[];
-  unsigned char *base = align128(smem_raw);
+  unsigned char *base = smem_aligned128(smem_raw);
   T *q_s = reinterpret_cast<T *>(base + 2 * Sm::kStage);
   T *dy_s = q_s + L * CT;
   float *es_s = reinterpret_cast<float *>(base + 2 * Sm::kStage + Sm::kQdy);
   uint64_t *bar = reinterpret_cast<uint64_t *>(es_s + CT);     // [0..1] a/v stages, [2] q/dy
-  int *ticket_s = reinterpret_cast<int *>(bar + 3);            // [2]
-  unsigned *tag_s = reinterpret_cast<unsigned *>(ticket_s + 2);
+  TileInfo *info_s = reinterpret_cast<TileInfo *>(bar + 4);    // [2], per a/v stage
+  unsigned *tag_s = reinterpret_cast<unsigned *>(info_s + 2);
 
   const int tid = threadIdx.x;
   const ScanShape &sh = args.s;
@@ -535,26 +571,19 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
   auto box = [&](int stage, int k) -> T * {
     return reinterpret_cast<T *>(base + stage * Sm::kStage + k * size_t(Cfg::kBoxBytes));
   };
-  auto coords = [&](int tile, int &c0, int &t0, int &b) {
-    const int chain = tile % sh.nchains;
-    const int chunk = sh.nchunks - 1 - tile / sh.nchains;   // latest chunk first
-    c0 = (chain % sh.nct) * CT;
-    b = chain / sh.nct;
-    t0 = chunk * L;
-  };
+  // Thread 0: decode a ticket into the stage's tile info and start its a/v loads.
   auto issue_av = [&](int stage, int tile) {
-    int c0, t0, b;
-    coords(tile, c0, t0, b);
+    const TileInfo ti = decode_tile<true>(tile, sh, CT, L);
+    info_s[stage] = ti;
+    if (tile >= sh.ntiles) return;
     mbar_expect_tx(&bar[stage], 2 * Cfg::kBoxBytes);
-    tma_load_3d(box(stage, 0), &tm_a, c0, t0, b, &bar[stage]);
-    tma_load_3d(box(stage, 1), &tm_v, c0, t0, b, &bar[stage]);
+    tma_load_3d(box(stage, 0), &tm_a, ti.c0, ti.t0, ti.b, &bar[stage]);
+    tma_load_3d(box(stage, 1), &tm_v, ti.c0, ti.t0, ti.b, &bar[stage]);
   };
-  auto issue_qdy = [&](int tile) {
-    int c0, t0, b;
-    coords(tile, c0, t0, b);
+  auto issue_qdy = [&](const TileInfo &ti) {
     mbar_expect_tx(&bar[2], 2 * Cfg::kBoxBytes);
-    tma_load_3d(q_s, &tm_q, c0, t0, b, &bar[2]);
-    tma_load_3d(dy_s, &tm_dy, c0, t0, b, &bar[2]);
+    tma_load_3d(q_s, &tm_q, ti.c0, ti.t0, ti.b, &bar[2]);
+    tma_load_3d(dy_s, &tm_dy, ti.c0, ti.t0, ti.b, &bar[2]);
   };
 
   if (tid == 0) {
@@ -571,13 +600,9 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     *tag_s = tag;
     const int t0 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[1], 1u)) : sh.ntiles;
     const int t1 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[1], 1u)) : sh.ntiles;
-    ticket_s[0] = t0;
-    ticket_s[1] = t1;
-    if (t0 < sh.ntiles) {
-      issue_av(0, t0);
-      issue_qdy(t0);
-    }
-    if (t1 < sh.ntiles) issue_av(1, t1);
+    issue_av(0, t0);
+    if (t0 < sh.ntiles) issue_qdy(info_s[0]);
+    issue_av(1, t1);
   }
   __syncthreads();
 
@@ -590,18 +615,15 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
 
   for (int it = 0;; ++it) {
     const int s = it & 1;
-    const int tile = ticket_s[s];
-    if (tile >= sh.ntiles) break;
+    const TileInfo ti = info_s[s];
+    if (ti.tile >= sh.ntiles) break;
     unsigned next = 0;
     if (tid == 0) next = atomicAdd(&hdr->ticket[1], 1u);
-
-    const int chain = tile % sh.nchains;
-    const int chunk = sh.nchunks - 1 - tile / sh.nchains;
-    const int b = chain / sh.nct, c0 = (chain % sh.nct) * CT, t0 = chunk * L;
-    const long slot = static_cast<long>(chain) * sh.nchunks + chunk;
+    const int chunk = ti.chunk, b = ti.b, c0 = ti.c0, t0 = ti.t0;
+    const long slot = ti.slot;
     const T *a_s = box(s, 0);
     const T *v_s = box(s, 1);
-    float2 *scan_s = reinterpret_cast<float2 *>(box(s, 0));
+    float *scan_s = reinterpret_cast<float *>(box(s, 0));
 
     float E_ck = 0.0f;   // forward state entering the chunk, channel tid (checkpoint)
     if (tid < CT) {
@@ -782,9 +804,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     __syncthreads();
     if (tid == 0) {
       fence_proxy_async_smem();   // generic smem writes before the async refills
-      if (ticket_s[s ^ 1] < sh.ntiles) issue_qdy(ticket_s[s ^ 1]);
-      ticket_s[s] = static_cast<int>(next);
-      if (static_cast<int>(next) < sh.ntiles) issue_av(s, static_cast<int>(next));
+      if (info_s[s ^ 1].tile < sh.ntiles) issue_qdy(info_s[s ^ 1]);
+      issue_av(s, static_cast<int>(next));
     }
   }
   scan_epilogue(hdr, 1, tag != 0u);
