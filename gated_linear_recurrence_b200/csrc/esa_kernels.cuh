@@ -112,6 +112,11 @@ struct TileCfg {
   static constexpr int RW = 32 / VW;               // runs per warp
   static constexpr int NVSEG = VPR / VW;
   static constexpr unsigned kBoxBytes = L * CT * sizeof(T);
+  // Threads [0, CT/2) scan the runs of channel pairs; threads [LB0, LB0 + CT)
+  // poll the look-back, one channel each -- concurrently with the scan when
+  // the block has room for both, else after it (LB0 = 0).
+  static constexpr int NSCAN = CT / 2;
+  static constexpr int LB0 = (NT >= ((NSCAN + 31) / 32) * 32 + CT) ? ((NSCAN + 31) / 32) * 32 : 0;
   static_assert(L % K == 0, "K must divide L");
   static_assert(NT % 32 == 0 && NT <= 1024, "bad block size");
   static_assert(RUNS % RW == 0, "runs must fill warps");
@@ -199,23 +204,26 @@ __device__ __forceinline__ void scan_load8(const float *scan, int run, int ch, f
   }
 }
 
-// Serial scan over the runs of one channel (threads 0..CT-1).  Replaces each
-// entry by the exclusive prefix and returns the tile map (forward order:
-// oldest run first; backward order: latest run first).
+// Serial scan over the runs of the channel pair (2 c2, 2 c2 + 1), packed
+// (threads 0..CT/2-1).  Replaces each entry by the exclusive prefix and
+// returns the pair's tile map (forward order: oldest run first; backward
+// order: latest run first).
 template <int CT, int RUNS, bool kReverse>
-__device__ __forceinline__ float2 scan_runs(float *scan, int c) {
-  float *col = scan + scan_pos<CT>(0, c);
-  float cp = 1.0f, cs = 0.0f;
+__device__ __forceinline__ void scan_runs2(float *scan, int c2, float2 &tP, float2 &tS) {
+  float *col = scan + scan_pos<CT>(0, 2 * c2);   // P pair at col[0..1], S pair at col[2..3]
+  float2 cp = splat(1.0f), cs = splat(0.0f);
 #pragma unroll
   for (int k = 0; k < RUNS; ++k) {
     const int r = kReverse ? RUNS - 1 - k : k;
-    const float ep = col[r * CT * 2], es = col[r * CT * 2 + 2];
-    col[r * CT * 2] = cp;
-    col[r * CT * 2 + 2] = cs;
-    cs = __fmaf_rn(ep, cs, es);
-    cp = cp * ep;
+    float2 *pp = reinterpret_cast<float2 *>(col + r * CT * 2);
+    const float2 ep = pp[0], es = pp[1];
+    pp[0] = cp;
+    pp[1] = cs;
+    cs = fma2(ep, cs, es);
+    cp = mul2(cp, ep);
   }
-  return make_float2(cp, cs);
+  tP = cp;
+  tS = cs;
 }
 
 // The run's carry-in for its 8 channels: prefix map (from the scratch)
@@ -469,24 +477,36 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     __syncthreads();
 
     // ---- scan over runs, look-back, publish --------------------------------
-    if (tid < CT) {
-      const float2 tmap = scan_runs<CT, RUNS, false>(scan_s, tid);
-      const int cg = c0 + tid;
+    float2 tP = splat(1.0f), tS = splat(0.0f);   // tile map of channel pair tid (scan threads)
+    if (tid < Cfg::NSCAN) {
+      scan_runs2<CT, RUNS, false>(scan_s, tid, tP, tS);
+      if (chunk > 0) {   // publish the pair's chunk map for successors' look-backs
+        const long at = slot * CT + 2 * tid;
+        st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tP.x, tag), pack_tag(tS.x, tag)));
+        st_relaxed_v2b64(&ws.agg[at + 1], make_ulonglong2(pack_tag(tP.y, tag), pack_tag(tS.y, tag)));
+      }
+    }
+    if (tid >= Cfg::LB0 && tid < Cfg::LB0 + CT) {   // carry entering the chunk, one channel each
+      const int c = tid - Cfg::LB0;
+      const int cg = c0 + c;
       float E_start;
-      const long at = slot * CT + tid;
       if (chunk == 0) {
         E_start = (args.E_init != nullptr && cg < sh.C) ? args.E_init[static_cast<long>(b) * sh.C + cg] : 0.0f;
       } else {
-        st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tmap.x, tag), pack_tag(tmap.y, tag)));
-        E_start = carry_in(ws.incl_f, ws.agg, slot, -1, chunk, CT, tid, tag, &hdr->abort[0], &hdr->status);
+        E_start = carry_in(ws.incl_f, ws.agg, slot, -1, chunk, CT, c, tag, &hdr->abort[0], &hdr->status);
       }
-      const float E_end = __fmaf_rn(tmap.x, E_start, tmap.y);
-      st_relaxed_b64(&ws.incl_f[at], pack_tag(E_end, tag));
-      if (chunk == sh.nchunks - 1 && args.E_final != nullptr && cg < sh.C)
-        args.E_final[static_cast<long>(b) * sh.C + cg] = E_end;
-      es_s[tid] = E_start;
+      es_s[c] = E_start;
     }
     __syncthreads();
+    if (tid < Cfg::NSCAN) {   // publish the chunk-end state of the pair
+      const float2 E_end = fma2(tP, reinterpret_cast<const float2 *>(es_s)[tid], tS);
+      const long at = slot * CT + 2 * tid;
+      st_relaxed_v2b64(reinterpret_cast<ulonglong2 *>(&ws.incl_f[at]),
+                       make_ulonglong2(pack_tag(E_end.x, tag), pack_tag(E_end.y, tag)));
+      const int cg = c0 + 2 * tid;
+      if (chunk == sh.nchunks - 1 && args.E_final != nullptr && cg < sh.C)
+        *reinterpret_cast<float2 *>(&args.E_final[static_cast<long>(b) * sh.C + cg]) = E_end;
+    }
 
     // ---- pass 2: exact states and the readout ------------------------------
     float2 E[4];
@@ -662,7 +682,10 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     scan_store8<CT>(scan_s, pos.run, pos.ch, P, S);
     if (tid < CT) es_s[tid] = E_ck;
     __syncthreads();
-    if (tid < CT) scan_runs<CT, RUNS, false>(scan_s, tid);
+    if (tid < Cfg::NSCAN) {
+      float2 tP, tS;
+      scan_runs2<CT, RUNS, false>(scan_s, tid, tP, tS);
+    }
     __syncthreads();
 
     // ---- F2: replay states, readout backward, dq, ghat ---------------------
@@ -731,25 +754,39 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     __syncthreads();
 
     // ---- reverse scan over runs, look-back towards later chunks -------------
-    if (tid < CT) {
-      const float2 tmap = scan_runs<CT, RUNS, true>(scan_s, tid);
-      const int cg = c0 + tid;
-      float H_in;
-      const long at = slot * CT + tid;
-      if (chunk == sh.nchunks - 1) {
-        H_in = (args.dE_final != nullptr && cg < sh.C) ? args.dE_final[static_cast<long>(b) * sh.C + cg] : 0.0f;
-      } else {
-        st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tmap.x, tag), pack_tag(tmap.y, tag)));
-        H_in = carry_in(ws.incl_b, ws.agg, slot, +1, sh.nchunks - 1 - chunk, CT, tid, tag, &hdr->abort[1],
-                        &hdr->status);
+    {
+      float2 tP = splat(1.0f), tS = splat(0.0f);
+      if (tid < Cfg::NSCAN) {
+        scan_runs2<CT, RUNS, true>(scan_s, tid, tP, tS);
+        if (chunk < sh.nchunks - 1) {
+          const long at = slot * CT + 2 * tid;
+          st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tP.x, tag), pack_tag(tS.x, tag)));
+          st_relaxed_v2b64(&ws.agg[at + 1], make_ulonglong2(pack_tag(tP.y, tag), pack_tag(tS.y, tag)));
+        }
       }
-      const float H_out = __fmaf_rn(tmap.x, H_in, tmap.y);
-      st_relaxed_b64(&ws.incl_b[at], pack_tag(H_out, tag));
-      if (chunk == 0 && args.dE_init != nullptr && cg < sh.C)
-        args.dE_init[static_cast<long>(b) * sh.C + cg] = H_out;
-      es_s[tid] = H_in;
+      if (tid >= Cfg::LB0 && tid < Cfg::LB0 + CT) {
+        const int c = tid - Cfg::LB0;
+        const int cg = c0 + c;
+        float H_in;
+        if (chunk == sh.nchunks - 1) {
+          H_in = (args.dE_final != nullptr && cg < sh.C) ? args.dE_final[static_cast<long>(b) * sh.C + cg] : 0.0f;
+        } else {
+          H_in = carry_in(ws.incl_b, ws.agg, slot, +1, sh.nchunks - 1 - chunk, CT, c, tag, &hdr->abort[1],
+                          &hdr->status);
+        }
+        es_s[c] = H_in;
+      }
+      __syncthreads();
+      if (tid < Cfg::NSCAN) {
+        const float2 H_out = fma2(tP, reinterpret_cast<const float2 *>(es_s)[tid], tS);
+        const long at = slot * CT + 2 * tid;
+        st_relaxed_v2b64(reinterpret_cast<ulonglong2 *>(&ws.incl_b[at]),
+                         make_ulonglong2(pack_tag(H_out.x, tag), pack_tag(H_out.y, tag)));
+        const int cg = c0 + 2 * tid;
+        if (chunk == 0 && args.dE_init != nullptr && cg < sh.C)
+          *reinterpret_cast<float2 *>(&args.dE_init[static_cast<long>(b) * sh.C + cg]) = H_out;
+      }
     }
-    __syncthreads();
 
     // ---- B1: total gradient G_t (latest step first): dv, and the da factor -
     // G A (1 - A) replaces ghat in the row's slots.
