@@ -17,6 +17,7 @@
 
 namespace {
 
+using esa::fwd_slots_per_tile;
 using esa::tile_cols;
 using esa::tile_rows;
 
@@ -38,10 +39,11 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 //   incl_f       n * CT  u64   forward chunk-end states (epoch-tagged)
 //   incl_b       n * CT  u64   backward chunk carries (epoch-tagged)
 //   agg          n * CT  2*u64 chunk maps (P, S), each word epoch-tagged
-// with n = B * ceil(C / CT) * ceil(T / L) chunks.
+// with n = B * ceil(C / CT) * ceil(T / L) slots of L rows (L = tile_rows).
+// The backward's tiles are one slot tall; a forward tile may span several.
 struct Layout {
-  int L = 0, CT = 0, nct = 0, nchunks = 0, nchains = 0;
-  long long ntiles = 0;
+  int L = 0, CT = 0, nct = 0, nslots = 0, nchains = 0;
+  long long ntiles = 0;   // nchains * nslots
   size_t incl_f_off = 0, incl_b_off = 0, agg_off = 0, total = 0;
 };
 
@@ -56,11 +58,11 @@ bool make_layout(int B, int T, int H, int D, int dtype, Layout *lo) {
   lo->L = tile_rows(dtype);
   lo->CT = tile_cols(D);
   lo->nct = static_cast<int>((C + lo->CT - 1) / lo->CT);
-  lo->nchunks = (T + lo->L - 1) / lo->L;
+  lo->nslots = (T + lo->L - 1) / lo->L;
   const long long nchains = static_cast<long long>(B) * lo->nct;
   if (nchains > INT_MAX) return false;
   lo->nchains = static_cast<int>(nchains);
-  lo->ntiles = nchains * lo->nchunks;
+  lo->ntiles = nchains * lo->nslots;
   if (lo->ntiles > INT_MAX) return false;
   const size_t words = static_cast<size_t>(lo->ntiles) * lo->CT;
   size_t off = kHeaderBytes;
@@ -122,8 +124,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [B][T][C] tensor in the I/O dtype, read in boxes of [L rows][CT channels].
-int make_tmap(CUtensorMap *map, const void *ptr, int dtype, int B, int T, int C, const Layout &lo) {
+// [B][T][C] tensor in the I/O dtype, read in boxes of [rows][CT channels].
+int make_tmap(CUtensorMap *map, const void *ptr, int dtype, int B, int T, int C, const Layout &lo, int rows) {
   auto fn = encode_fn();
   if (fn == nullptr) return ESA_ERR_LAUNCH;
   const CUtensorMapDataType dt = dtype == ESA_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
@@ -134,7 +136,7 @@ int make_tmap(CUtensorMap *map, const void *ptr, int dtype, int B, int T, int C,
                               static_cast<cuuint64_t>(B)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(C) * s,
                                  static_cast<cuuint64_t>(T) * static_cast<cuuint64_t>(C) * s};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(lo.CT), static_cast<cuuint32_t>(lo.L), 1};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(lo.CT), static_cast<cuuint32_t>(rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   std::memset(map, 0, sizeof(*map));
   const CUresult r = fn(map, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr,
@@ -152,15 +154,17 @@ int check_shape(int B, int T, int H, int D, int mode, int dtype) {
   return ESA_OK;
 }
 
-esa::ScanShape scan_shape(int B, int T, int H, int D, const Layout &lo) {
+// Shape of a scan whose tiles span `sub` slots each.
+esa::ScanShape scan_shape(int B, int T, int H, int D, const Layout &lo, int sub) {
   esa::ScanShape s;
   s.B = B;
   s.T = T;
   s.C = H * D;
-  s.nchunks = lo.nchunks;
+  s.nslots = lo.nslots;
+  s.nchunks = (lo.nslots + sub - 1) / sub;
   s.nct = lo.nct;
   s.nchains = lo.nchains;
-  s.ntiles = static_cast<int>(lo.ntiles);
+  s.ntiles = lo.nchains * s.nchunks;   // <= lo.ntiles, checked to fit an int
   s.inv_D = 1.0f / static_cast<float>(D);
   return s;
 }
@@ -204,17 +208,18 @@ int esa_scan_fwd(const void *a, const void *v, const void *q, void *y, float *E_
     return E_init ? rt(cudaMemcpyAsync(E_final, E_init, bytes, cudaMemcpyDeviceToDevice, st))
                   : rt(cudaMemsetAsync(E_final, 0, bytes, st));
   }
+  const int sub = fwd_slots_per_tile(dtype, D);
   CUtensorMap ta, tv, tq;
-  if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo))) return rc;
-  if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo))) return rc;
-  if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo))) return rc;
+  if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo, lo.L * sub))) return rc;
+  if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo, lo.L * sub))) return rc;
+  if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo, lo.L * sub))) return rc;
   esa::FwdArgs args;
-  args.s = scan_shape(B, T, H, D, lo);
+  args.s = scan_shape(B, T, H, D, lo, sub);
   args.y = y;
   args.E_final = E_final;
   args.E_init = E_init;
   args.ws = workspace_view(workspace, lo);
-  return esa::launch_fwd(dtype, mode, D, ta, tv, tq, args, static_cast<int>(lo.ntiles), st);
+  return esa::launch_fwd(dtype, mode, D, ta, tv, tq, args, args.s.ntiles, st);
 }
 
 int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy, const float *dE_final,
@@ -243,12 +248,12 @@ int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy, co
                     : rt(cudaMemsetAsync(dE_init, 0, bytes, st));
   }
   CUtensorMap ta, tv, tq, tdy;
-  if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo))) return rc;
-  if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo))) return rc;
-  if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo))) return rc;
-  if ((rc = make_tmap(&tdy, dy, dtype, B, T, C, lo))) return rc;
+  if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo, lo.L))) return rc;
+  if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo, lo.L))) return rc;
+  if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo, lo.L))) return rc;
+  if ((rc = make_tmap(&tdy, dy, dtype, B, T, C, lo, lo.L))) return rc;
   esa::BwdArgs args;
-  args.s = scan_shape(B, T, H, D, lo);
+  args.s = scan_shape(B, T, H, D, lo, 1);
   args.da = da;
   args.dv = dv;
   args.dq = dq;
@@ -256,7 +261,7 @@ int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy, co
   args.dE_init = dE_init;
   args.E_init = E_init;
   args.ws = workspace_view(workspace, lo);
-  return esa::launch_bwd(dtype, mode, D, ta, tv, tq, tdy, args, static_cast<int>(lo.ntiles), st);
+  return esa::launch_bwd(dtype, mode, D, ta, tv, tq, tdy, args, args.s.ntiles, st);
 }
 
 int esa_step(const void *a_t, const void *v_t, const void *q_t, float *E, void *y_t, int B, int H, int D,

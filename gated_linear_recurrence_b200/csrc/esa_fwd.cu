@@ -12,9 +12,13 @@ struct FwdLauncher {
 
   template <typename T, int MODE, int LPH, int VPR, int L, int K>
   int operator()() const {
-    using Cfg = TileCfg<T, LPH, VPR, L, K>;
+    constexpr int SUB = fwd_sub<T, VPR>();
+    constexpr int SEG = 1;     // lanes per channel pair in the run scan (one: fewest bank conflicts)
+    using Cfg = TileCfg<T, LPH, VPR, L * SUB, K, SEG>;
+    // The host sized the tile grid with the same slots-per-tile rule.
+    if (args.s.nchunks != (args.s.nslots + SUB - 1) / SUB) return -5;
     const size_t smem = FwdSmem<Cfg>::kBytes;
-    auto kern = esa_scan_fwd_kernel<T, MODE, LPH, VPR, L, K>;
+    auto kern = esa_scan_fwd_kernel<T, MODE, LPH, VPR, L * SUB, K, SUB, SEG>;
     int grid = 0;
     const int rc = persistent_grid(kern, Cfg::NT, smem, ntiles, &grid);
     if (rc) return rc;

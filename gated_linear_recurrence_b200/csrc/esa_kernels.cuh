@@ -40,7 +40,8 @@ namespace esa {
 
 struct ScanShape {
   int B, T, C;          // C = H * D
-  int nchunks;          // ceil(T / L)
+  int nslots;           // workspace slots per chain: ceil(T / G), G = slot rows
+  int nchunks;          // tiles per chain of this kernel: ceil(nslots / SUB)
   int nct;              // channel tiles per batch row
   int nchains;          // B * nct
   int ntiles;           // nchains * nchunks
@@ -73,11 +74,12 @@ struct TileInfo {
   int c0;       // first channel of the tile
   int t0;       // first time step of the tile
   int pad;
-  long slot;    // chain * nchunks + chunk
+  long slot;    // first workspace slot of the tile: chain * nslots + chunk * SUB
 };
 
-// kReverse: chunks in processing order run from the last to the first.
-template <bool kReverse>
+// kReverse: chunks in processing order run from the last to the first.  A
+// tile of L rows spans SUB workspace slots of L / SUB rows each.
+template <bool kReverse, int SUB>
 __device__ __forceinline__ TileInfo decode_tile(int tile, const ScanShape &sh, int CT, int L) {
   TileInfo t;
   t.tile = tile;
@@ -93,12 +95,13 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const ScanShape &sh, i
   t.b = chain / sh.nct;
   t.c0 = (chain % sh.nct) * CT;
   t.t0 = t.chunk * L;
-  t.slot = static_cast<long>(chain) * sh.nchunks + t.chunk;
+  t.slot = static_cast<long>(chain) * sh.nslots + static_cast<long>(t.chunk) * SUB;
   return t;
 }
 
-// Compile-time tile geometry.
-template <typename T, int LPH_, int VPR_, int L_, int K_>
+// Compile-time tile geometry.  SEG_ lanes share the run scan of a channel
+// pair (each scans RUNS / SEG_ runs, then the segments are combined).
+template <typename T, int LPH_, int VPR_, int L_, int K_, int SEG_ = 1>
 struct TileCfg {
   static constexpr int LPH = LPH_;                 // lanes per head = D / 8
   static constexpr int VPR = VPR_;                 // 8-channel vectors per tile row
@@ -111,13 +114,16 @@ struct TileCfg {
   static constexpr int VW = VW0 < VPR ? VW0 : VPR; // vectors per warp row segment
   static constexpr int RW = 32 / VW;               // runs per warp
   static constexpr int NVSEG = VPR / VW;
+  static constexpr int SEG = SEG_;
   static constexpr unsigned kBoxBytes = L * CT * sizeof(T);
-  // Threads [0, CT/2) scan the runs of channel pairs; threads [LB0, LB0 + CT)
-  // poll the look-back, one channel each -- concurrently with the scan when
-  // the block has room for both, else after it (LB0 = 0).
-  static constexpr int NSCAN = CT / 2;
+  // Threads [0, SEG CT/2) scan the runs of channel pairs; threads
+  // [LB0, LB0 + CT) poll the look-back, one channel each -- concurrently with
+  // the scan when the block has room for both, else after it (LB0 = 0).
+  static constexpr int NSCAN = SEG * CT / 2;
   static constexpr int LB0 = (NT >= ((NSCAN + 31) / 32) * 32 + CT) ? ((NSCAN + 31) / 32) * 32 : 0;
   static_assert(L % K == 0, "K must divide L");
+  static_assert(SEG == 1 || SEG == 2 || SEG == 4, "1, 2 or 4 lanes per channel pair");
+  static_assert(RUNS % SEG == 0, "segments must split the runs evenly");
   static_assert(NT % 32 == 0 && NT <= 1024, "bad block size");
   static_assert(RUNS % RW == 0, "runs must fill warps");
   static_assert(CT % 32 == 0 && NT >= CT, "look-back needs CT threads");
@@ -204,26 +210,68 @@ __device__ __forceinline__ void scan_load8(const float *scan, int run, int ch, f
   }
 }
 
-// Serial scan over the runs of the channel pair (2 c2, 2 c2 + 1), packed
-// (threads 0..CT/2-1).  Replaces each entry by the exclusive prefix and
-// returns the pair's tile map (forward order: oldest run first; backward
-// order: latest run first).
-template <int CT, int RUNS, bool kReverse>
-__device__ __forceinline__ void scan_runs2(float *scan, int c2, float2 &tP, float2 &tS) {
+// Scan over the runs of the channel pair (2 c2, 2 c2 + 1), packed, by SEG
+// consecutive lanes: lane `seg` serially scans the runs [seg RS, (seg+1) RS)
+// of the processing order (RS = RUNS / SEG; oldest run first, or latest first
+// for kReverse), the segment maps are combined across the lanes by shuffles,
+// and each lane folds its segment's prefix into its runs.  Every entry is
+// replaced by its exclusive prefix over the tile.  Returns in each lane the
+// prefix at the start of its own segment (sP, sS) and the tile map (tP, tS).
+template <int CT, int RUNS, int SEG, bool kReverse>
+__device__ __forceinline__ void scan_runs(float *scan, int c2, int seg, float2 &sP, float2 &sS, float2 &tP,
+                                          float2 &tS) {
+  constexpr int RS = RUNS / SEG;
   float *col = scan + scan_pos<CT>(0, 2 * c2);   // P pair at col[0..1], S pair at col[2..3]
+  auto entry = [&](int j) -> float2 * {
+    const int r = kReverse ? RUNS - 1 - j : j;
+    return reinterpret_cast<float2 *>(col + r * CT * 2);
+  };
   float2 cp = splat(1.0f), cs = splat(0.0f);
 #pragma unroll
-  for (int k = 0; k < RUNS; ++k) {
-    const int r = kReverse ? RUNS - 1 - k : k;
-    float2 *pp = reinterpret_cast<float2 *>(col + r * CT * 2);
+  for (int k = 0; k < RS; ++k) {
+    float2 *pp = entry(seg * RS + k);
     const float2 ep = pp[0], es = pp[1];
     pp[0] = cp;
     pp[1] = cs;
     cs = fma2(ep, cs, es);
     cp = mul2(cp, ep);
   }
-  tP = cp;
-  tS = cs;
+  if constexpr (SEG == 1) {
+    sP = splat(1.0f);
+    sS = splat(0.0f);
+    tP = cp;
+    tS = cs;
+  } else {
+    // Inclusive composition of the segment maps over lanes 0..seg (a later
+    // map applied after the earlier ones), then shifted to exclusive.
+    float2 iP = cp, iS = cs;
+#pragma unroll
+    for (int o = 1; o < SEG; o <<= 1) {
+      const float2 oP = shfl_up2(iP, o, SEG), oS = shfl_up2(iS, o, SEG);
+      if (seg >= o) {
+        iS = fma2(iP, oS, iS);
+        iP = mul2(iP, oP);
+      }
+    }
+    float2 eP = shfl_up2(iP, 1, SEG), eS = shfl_up2(iS, 1, SEG);
+    if (seg == 0) {
+      eP = splat(1.0f);
+      eS = splat(0.0f);
+    }
+    tP = shfl_idx2(iP, SEG - 1, SEG);
+    tS = shfl_idx2(iS, SEG - 1, SEG);
+    if (seg > 0) {
+#pragma unroll
+      for (int k = 0; k < RS; ++k) {
+        float2 *pp = entry(seg * RS + k);
+        const float2 lp = pp[0], ls = pp[1];
+        pp[0] = mul2(lp, eP);
+        pp[1] = fma2(lp, eS, ls);
+      }
+    }
+    sP = eP;
+    sS = eS;
+  }
 }
 
 // The run's carry-in for its 8 channels: prefix map (from the scratch)
@@ -240,19 +288,17 @@ __device__ __forceinline__ void run_carry(const float *scan, const float *es_s, 
 template <int LPH>
 __device__ __forceinline__ float head_sum2(float2 s) { return head_sum<LPH>(s.x + s.y); }
 
-// The carry entering chunk `slot` for channel `c`: the nearest predecessor
-// (distance 1, 2, ... in direction `dir`, at most `avail`) whose chunk-end
-// carry carries the current tag, with the chunk maps of every tile in between
-// applied oldest first -- the same fused multiply-adds those tiles used for
-// their own carries, so the value does not depend on how far the search went.
-// Distances 1..4 are read in one round trip; deeper searches walk one chunk
-// at a time.  Bounded: gives up (returns 0, records a timeout, raises the
-// abort flag) after kSpinLimit polls or when another CTA raised the flag.
-__device__ __forceinline__ float carry_in(const unsigned long long *incl, const ulonglong2 *agg, long slot, int dir,
-                                       int avail, int CT, int c, unsigned tag, unsigned *abort_flag,
-                                       unsigned *status) {
-  const long me = slot * CT + c;
-  const long step = static_cast<long>(dir) * CT;
+// The carry entering a tile for one channel: the nearest predecessor tile
+// (distance d = 1, 2, ..., at most `avail`; its words sit at me + d * step in
+// `incl` and `agg`) whose chunk-end carry carries the current tag, with the
+// chunk maps of every tile in between applied oldest first -- the same fused
+// multiply-adds those tiles used for their own carries, so the value does not
+// depend on how far the search went.  Distances 1..4 are read in one round
+// trip; deeper searches walk one tile at a time.  Bounded: gives up (returns
+// 0, records a timeout, raises the abort flag) after kSpinLimit polls or when
+// another CTA raised the flag.
+__device__ __forceinline__ float carry_in(const unsigned long long *incl, const ulonglong2 *agg, long me, long step,
+                                       int avail, unsigned tag, unsigned *abort_flag, unsigned *status) {
   unsigned ns = 16;
   for (unsigned it = 0; it < kSpinLimit; ++it) {
     unsigned long long iw[4];
@@ -376,13 +422,17 @@ template <int MODE>
 __device__ __forceinline__ float2 gate_A(float2 c) { return MODE == 0 ? c : sub2(splat(1.0f), c); }
 
 // ===========================================================================
-// Forward scan (persistent).
+// Forward scan (persistent).  A tile of L rows covers SUB workspace slots:
+// it publishes its chunk map and reads its predecessors' at its last slot,
+// and stores the chunk-end state of every slot it covers (the backward's
+// checkpoints), so taller forward tiles leave the workspace layout alone.
 // ===========================================================================
-template <typename T, int MODE, int LPH, int VPR, int L, int K>
+template <typename T, int MODE, int LPH, int VPR, int L, int K, int SUB, int SEG>
 __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR * (L / K) <= 128) ? 4 : (VPR * (L / K) <= 256) ? 2 : 1)
     esa_scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_q, const FwdArgs args) {
-  using Cfg = TileCfg<T, LPH, VPR, L, K>;
+  static_assert(SUB == 1 || SUB == 2, "a forward tile spans one or two slots");
+  using Cfg = TileCfg<T, LPH, VPR, L, K, SEG>;
   using Sm = FwdSmem<Cfg>;
   constexpr int CT = Cfg::CT, RUNS = Cfg::RUNS;
 
@@ -403,7 +453,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
   };
   // Thread 0: decode a ticket into the stage's tile info and start its loads.
   auto issue = [&](int stage, int tile) {
-    const TileInfo ti = decode_tile<false>(tile, sh, CT, L);
+    const TileInfo ti = decode_tile<false, SUB>(tile, sh, CT, L);
     info_s[stage] = ti;
     if (tile >= sh.ntiles) return;
     mbar_expect_tx(&bar[stage], 3 * Cfg::kBoxBytes);
@@ -438,14 +488,21 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     const int s = it & 1;
     const TileInfo ti = info_s[s];
     if (ti.tile >= sh.ntiles) break;
-    unsigned next = 0;
-    if (tid == 0) next = atomicAdd(&hdr->ticket[0], 1u);   // the tile that will refill this stage
+    unsigned next = 0;   // ticket of the tile that will refill this stage
     const int chunk = ti.chunk, b = ti.b, c0 = ti.c0, t0 = ti.t0;
-    const long slot = ti.slot;
+    const long slot = ti.slot;                 // first slot of the tile
+    const long slot_end = slot + SUB - 1;      // the slot its look-back words live in
     const T *a_s = box(s, 0);
     const T *v_s = box(s, 1);
     const T *q_s = box(s, 2);
     float *scan_s = reinterpret_cast<float *>(box(s, 0));   // reused once pass 1 is done
+
+    // Look-back threads read the nearest predecessor's chunk-end carry now, a
+    // pass ahead of the look-back: when that tile has already finished, the
+    // look-back needs no further round trip.
+    const bool lb_thread = tid >= Cfg::LB0 && tid < Cfg::LB0 + CT;
+    unsigned long long early = 0ull;
+    if (lb_thread && chunk > 0) early = ld_relaxed_b64(&ws.incl_f[(slot_end - SUB) * CT + (tid - Cfg::LB0)]);
 
     mbar_wait_bounded(&bar[s], (phase >> s) & 1u, &hdr->status);
     phase ^= 1u << s;
@@ -477,33 +534,60 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     __syncthreads();
 
     // ---- scan over runs, look-back, publish --------------------------------
-    float2 tP = splat(1.0f), tS = splat(0.0f);   // tile map of channel pair tid (scan threads)
+    // Scan lanes: SEG lanes per channel pair c2; the last one publishes.
+    const int c2 = tid / SEG, seg = tid % SEG;
+    const bool publisher = tid < Cfg::NSCAN && seg == SEG - 1;
+    float2 sP = splat(1.0f), sS = splat(0.0f), tP = splat(1.0f), tS = splat(0.0f);
+    float2 mP = splat(1.0f), mS = splat(0.0f);   // prefix at the middle run (SUB == 2)
     if (tid < Cfg::NSCAN) {
-      scan_runs2<CT, RUNS, false>(scan_s, tid, tP, tS);
-      if (chunk > 0) {   // publish the pair's chunk map for successors' look-backs
-        const long at = slot * CT + 2 * tid;
+      scan_runs<CT, RUNS, SEG, false>(scan_s, c2, seg, sP, sS, tP, tS);
+      if constexpr (SUB == 2) {
+        if constexpr (SEG == 1) {   // this lane wrote the entry itself
+          const float2 *pm = reinterpret_cast<const float2 *>(scan_s + scan_pos<CT>(RUNS / 2, 2 * c2));
+          mP = pm[0];
+          mS = pm[1];
+        } else {                    // the middle run starts segment SEG / 2
+          mP = shfl_idx2(sP, SEG / 2, SEG);
+          mS = shfl_idx2(sS, SEG / 2, SEG);
+        }
+      }
+      if (chunk > 0 && publisher) {   // the pair's chunk map, for successors' look-backs
+        const long at = slot_end * CT + 2 * c2;
         st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tP.x, tag), pack_tag(tS.x, tag)));
         st_relaxed_v2b64(&ws.agg[at + 1], make_ulonglong2(pack_tag(tP.y, tag), pack_tag(tS.y, tag)));
       }
     }
-    if (tid >= Cfg::LB0 && tid < Cfg::LB0 + CT) {   // carry entering the chunk, one channel each
+    if (lb_thread) {   // carry entering the chunk, one channel each
       const int c = tid - Cfg::LB0;
       const int cg = c0 + c;
       float E_start;
       if (chunk == 0) {
         E_start = (args.E_init != nullptr && cg < sh.C) ? args.E_init[static_cast<long>(b) * sh.C + cg] : 0.0f;
+      } else if (tag_of(early) == tag) {   // what the look-back returns at distance 1
+        E_start = val_of(early);
       } else {
-        E_start = carry_in(ws.incl_f, ws.agg, slot, -1, chunk, CT, c, tag, &hdr->abort[0], &hdr->status);
+        E_start = carry_in(ws.incl_f, ws.agg, slot_end * CT + c, -static_cast<long>(SUB) * CT, chunk, tag,
+                           &hdr->abort[0], &hdr->status);
       }
       es_s[c] = E_start;
     }
     __syncthreads();
-    if (tid < Cfg::NSCAN) {   // publish the chunk-end state of the pair
-      const float2 E_end = fma2(tP, reinterpret_cast<const float2 *>(es_s)[tid], tS);
-      const long at = slot * CT + 2 * tid;
-      st_relaxed_v2b64(reinterpret_cast<ulonglong2 *>(&ws.incl_f[at]),
-                       make_ulonglong2(pack_tag(E_end.x, tag), pack_tag(E_end.y, tag)));
-      const int cg = c0 + 2 * tid;
+    // The ticket of the tile after next is taken only now: tickets then follow
+    // the order in which CTAs really reach their tiles more closely, so a
+    // tile's predecessors are rarely behind it.  Pass 2 hides the round trip.
+    if (tid == 0) next = atomicAdd(&hdr->ticket[0], 1u);
+    if (publisher) {   // chunk-end states of the pair at every slot the tile covers
+      const float2 E_in = reinterpret_cast<const float2 *>(es_s)[c2];
+      const float2 E_end = fma2(tP, E_in, tS);
+      if constexpr (SUB == 2) {   // the slot ending halfway through the tile
+        const float2 E_mid = fma2(mP, E_in, mS);
+        st_relaxed_v2b64(reinterpret_cast<ulonglong2 *>(&ws.incl_f[slot * CT + 2 * c2]),
+                         make_ulonglong2(pack_tag(E_mid.x, tag), pack_tag(E_mid.y, tag)));
+      }
+      if (chunk * SUB + SUB - 1 < sh.nslots)   // a ragged last tile may cover fewer slots
+        st_relaxed_v2b64(reinterpret_cast<ulonglong2 *>(&ws.incl_f[slot_end * CT + 2 * c2]),
+                         make_ulonglong2(pack_tag(E_end.x, tag), pack_tag(E_end.y, tag)));
+      const int cg = c0 + 2 * c2;
       if (chunk == sh.nchunks - 1 && args.E_final != nullptr && cg < sh.C)
         *reinterpret_cast<float2 *>(&args.E_final[static_cast<long>(b) * sh.C + cg]) = E_end;
     }
@@ -593,7 +677,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
   };
   // Thread 0: decode a ticket into the stage's tile info and start its a/v loads.
   auto issue_av = [&](int stage, int tile) {
-    const TileInfo ti = decode_tile<true>(tile, sh, CT, L);
+    const TileInfo ti = decode_tile<true, 1>(tile, sh, CT, L);
     info_s[stage] = ti;
     if (tile >= sh.ntiles) return;
     mbar_expect_tx(&bar[stage], 2 * Cfg::kBoxBytes);
@@ -637,8 +721,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     const int s = it & 1;
     const TileInfo ti = info_s[s];
     if (ti.tile >= sh.ntiles) break;
-    unsigned next = 0;
-    if (tid == 0) next = atomicAdd(&hdr->ticket[1], 1u);
+    unsigned next = 0;   // ticket of the tile that will refill this a/v stage
     const int chunk = ti.chunk, b = ti.b, c0 = ti.c0, t0 = ti.t0;
     const long slot = ti.slot;
     const T *a_s = box(s, 0);
@@ -683,8 +766,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     if (tid < CT) es_s[tid] = E_ck;
     __syncthreads();
     if (tid < Cfg::NSCAN) {
-      float2 tP, tS;
-      scan_runs2<CT, RUNS, false>(scan_s, tid, tP, tS);
+      float2 sP, sS, tP, tS;
+      scan_runs<CT, RUNS, 1, false>(scan_s, tid, 0, sP, sS, tP, tS);
     }
     __syncthreads();
 
@@ -733,6 +816,12 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
       }
     }
 
+    // Look-back threads read the nearest later chunk's carry now, a pass ahead
+    // of the look-back (see the forward).
+    const bool lb_thread = tid >= Cfg::LB0 && tid < Cfg::LB0 + CT;
+    unsigned long long early = 0ull;
+    if (lb_thread && chunk < sh.nchunks - 1) early = ld_relaxed_b64(&ws.incl_b[(slot + 1) * CT + (tid - Cfg::LB0)]);
+
     // ---- R1: the run's reverse map h -> P h + hl ----------------------------
     {
       float2 hl[4];
@@ -755,23 +844,25 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
 
     // ---- reverse scan over runs, look-back towards later chunks -------------
     {
-      float2 tP = splat(1.0f), tS = splat(0.0f);
+      float2 sP, sS, tP = splat(1.0f), tS = splat(0.0f);
       if (tid < Cfg::NSCAN) {
-        scan_runs2<CT, RUNS, true>(scan_s, tid, tP, tS);
+        scan_runs<CT, RUNS, 1, true>(scan_s, tid, 0, sP, sS, tP, tS);
         if (chunk < sh.nchunks - 1) {
           const long at = slot * CT + 2 * tid;
           st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tP.x, tag), pack_tag(tS.x, tag)));
           st_relaxed_v2b64(&ws.agg[at + 1], make_ulonglong2(pack_tag(tP.y, tag), pack_tag(tS.y, tag)));
         }
       }
-      if (tid >= Cfg::LB0 && tid < Cfg::LB0 + CT) {
+      if (lb_thread) {
         const int c = tid - Cfg::LB0;
         const int cg = c0 + c;
         float H_in;
         if (chunk == sh.nchunks - 1) {
           H_in = (args.dE_final != nullptr && cg < sh.C) ? args.dE_final[static_cast<long>(b) * sh.C + cg] : 0.0f;
+        } else if (tag_of(early) == tag) {
+          H_in = val_of(early);
         } else {
-          H_in = carry_in(ws.incl_b, ws.agg, slot, +1, sh.nchunks - 1 - chunk, CT, c, tag, &hdr->abort[1],
+          H_in = carry_in(ws.incl_b, ws.agg, slot * CT + c, CT, sh.nchunks - 1 - chunk, tag, &hdr->abort[1],
                           &hdr->status);
         }
         es_s[c] = H_in;
@@ -787,6 +878,10 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
           *reinterpret_cast<float2 *>(&args.dE_init[static_cast<long>(b) * sh.C + cg]) = H_out;
       }
     }
+
+    // Ticket of the tile after next, taken once the look-back is resolved (as
+    // in the forward): B1 and B2 hide its round trip.
+    if (tid == 0) next = atomicAdd(&hdr->ticket[1], 1u);
 
     // ---- B1: total gradient G_t (latest step first): dv, and the da factor -
     // G A (1 - A) replaces ghat in the row's slots.

@@ -9,11 +9,19 @@
 
 namespace esa {
 
-// Tile rows per chunk and channels per tile, as chosen for each I/O dtype and
-// head dimension.  The workspace layout and the kernels both follow these.
+// Rows per workspace slot (the backward's tile height) and channels per tile,
+// as chosen for each I/O dtype and head dimension.  The workspace layout and
+// the kernels both follow these.
 inline int tile_rows(int dtype) { return dtype == 0 ? 32 : 64; }   // f32 : 16-bit
 inline int tile_cols(int D) { return D <= 64 ? 64 : D; }
 constexpr int kStepsPerThread = 4;
+
+// Slots per forward tile: 64-channel tiles of 16-bit data run the forward
+// two slots (128 rows) tall -- twice the time between consecutive chunks of a
+// chain, so a tile's predecessors are further ahead when it looks back.
+template <typename T, int VPR>
+constexpr int fwd_sub() { return (sizeof(T) == 2 && VPR == 8) ? 2 : 1; }
+inline int fwd_slots_per_tile(int dtype, int D) { return (dtype != 0 && tile_cols(D) == 64) ? 2 : 1; }
 
 // Launch the forward / backward scan for (dtype, mode, D).  The tensor maps
 // describe a, v, q (and dy) as [B][T][C] boxes of [L][CT].  Return 0 or a
