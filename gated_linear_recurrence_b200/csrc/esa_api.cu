@@ -247,13 +247,14 @@ int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy, co
     return dE_final ? rt(cudaMemcpyAsync(dE_init, dE_final, bytes, cudaMemcpyDeviceToDevice, st))
                     : rt(cudaMemsetAsync(dE_init, 0, bytes, st));
   }
+  const int sub = esa::bwd_slots_per_tile(dtype, D);
   CUtensorMap ta, tv, tq, tdy;
-  if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo, lo.L))) return rc;
-  if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo, lo.L))) return rc;
-  if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo, lo.L))) return rc;
-  if ((rc = make_tmap(&tdy, dy, dtype, B, T, C, lo, lo.L))) return rc;
+  if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo, lo.L * sub))) return rc;
+  if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo, lo.L * sub))) return rc;
+  if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo, lo.L * sub))) return rc;
+  if ((rc = make_tmap(&tdy, dy, dtype, B, T, C, lo, lo.L * sub))) return rc;
   esa::BwdArgs args;
-  args.s = scan_shape(B, T, H, D, lo, 1);
+  args.s = scan_shape(B, T, H, D, lo, sub);
   args.da = da;
   args.dv = dv;
   args.dq = dq;

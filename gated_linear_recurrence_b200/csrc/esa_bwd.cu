@@ -12,9 +12,13 @@ struct BwdLauncher {
 
   template <typename T, int MODE, int LPH, int VPR, int L, int K>
   int operator()() const {
-    using Cfg = TileCfg<T, LPH, VPR, L, K>;
+    constexpr int SUB = bwd_sub<T, VPR>();
+    constexpr int SW = scan_segments<L * SUB / K, VPR * (L * SUB / K), VPR * 8>();
+    using Cfg = TileCfg<T, LPH, VPR, L * SUB, K, SW>;
+    // The host sized the tile grid with the same slots-per-tile rule.
+    if (args.s.nchunks != (args.s.nslots + SUB - 1) / SUB) return -5;
     const size_t smem = BwdSmem<Cfg>::kBytes;
-    auto kern = esa_scan_bwd_kernel<T, MODE, LPH, VPR, L, K>;
+    auto kern = esa_scan_bwd_kernel<T, MODE, LPH, VPR, L * SUB, K, SW, SUB>;
     int grid = 0;
     const int rc = persistent_grid(kern, Cfg::NT, smem, ntiles, &grid);
     if (rc) return rc;

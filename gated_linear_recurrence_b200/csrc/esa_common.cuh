@@ -73,13 +73,6 @@ __device__ __forceinline__ float val_of(unsigned long long w) {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float2 splat(float a) { return make_float2(a, a); }
 
-// Shuffles of a float2 within aligned groups of `width` lanes (full warp).
-__device__ __forceinline__ float2 shfl_up2(float2 v, int d, int width) {
-  return make_float2(__shfl_up_sync(0xffffffffu, v.x, d, width), __shfl_up_sync(0xffffffffu, v.y, d, width));
-}
-__device__ __forceinline__ float2 shfl_idx2(float2 v, int src, int width) {
-  return make_float2(__shfl_sync(0xffffffffu, v.x, src, width), __shfl_sync(0xffffffffu, v.y, src, width));
-}
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {   // a - b, one packed instruction
   unsigned long long ua, ub, ud;

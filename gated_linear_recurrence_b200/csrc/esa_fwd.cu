@@ -13,12 +13,12 @@ struct FwdLauncher {
   template <typename T, int MODE, int LPH, int VPR, int L, int K>
   int operator()() const {
     constexpr int SUB = fwd_sub<T, VPR>();
-    constexpr int SEG = 1;     // lanes per channel pair in the run scan (one: fewest bank conflicts)
-    using Cfg = TileCfg<T, LPH, VPR, L * SUB, K, SEG>;
+    constexpr int SW = scan_segments<L * SUB / K, VPR * (L * SUB / K), VPR * 8>();
+    using Cfg = TileCfg<T, LPH, VPR, L * SUB, K, SW>;
     // The host sized the tile grid with the same slots-per-tile rule.
     if (args.s.nchunks != (args.s.nslots + SUB - 1) / SUB) return -5;
     const size_t smem = FwdSmem<Cfg>::kBytes;
-    auto kern = esa_scan_fwd_kernel<T, MODE, LPH, VPR, L * SUB, K, SUB, SEG>;
+    auto kern = esa_scan_fwd_kernel<T, MODE, LPH, VPR, L * SUB, K, SUB, SW>;
     int grid = 0;
     const int rc = persistent_grid(kern, Cfg::NT, smem, ntiles, &grid);
     if (rc) return rc;

@@ -99,9 +99,10 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const ScanShape &sh, i
   return t;
 }
 
-// Compile-time tile geometry.  SEG_ lanes share the run scan of a channel
-// pair (each scans RUNS / SEG_ runs, then the segments are combined).
-template <typename T, int LPH_, int VPR_, int L_, int K_, int SEG_ = 1>
+// Compile-time tile geometry.  The run scan of a tile is split into SW_
+// segments of RUNS / SW_ consecutive runs; each segment is scanned by its own
+// group of CT / 2 lanes (one lane per channel pair).
+template <typename T, int LPH_, int VPR_, int L_, int K_, int SW_ = 1>
 struct TileCfg {
   static constexpr int LPH = LPH_;                 // lanes per head = D / 8
   static constexpr int VPR = VPR_;                 // 8-channel vectors per tile row
@@ -114,16 +115,19 @@ struct TileCfg {
   static constexpr int VW = VW0 < VPR ? VW0 : VPR; // vectors per warp row segment
   static constexpr int RW = 32 / VW;               // runs per warp
   static constexpr int NVSEG = VPR / VW;
-  static constexpr int SEG = SEG_;
+  static constexpr int SW = SW_;                   // run-scan segments
+  static constexpr int NP = CT / 2;                // channel pairs per tile
   static constexpr unsigned kBoxBytes = L * CT * sizeof(T);
-  // Threads [0, SEG CT/2) scan the runs of channel pairs; threads
+  // Threads [0, SW CT/2) scan the runs of channel pairs; threads
   // [LB0, LB0 + CT) poll the look-back, one channel each -- concurrently with
   // the scan when the block has room for both, else after it (LB0 = 0).
-  static constexpr int NSCAN = SEG * CT / 2;
+  static constexpr int NSCAN = SW * NP;
   static constexpr int LB0 = (NT >= ((NSCAN + 31) / 32) * 32 + CT) ? ((NSCAN + 31) / 32) * 32 : 0;
   static_assert(L % K == 0, "K must divide L");
-  static_assert(SEG == 1 || SEG == 2 || SEG == 4, "1, 2 or 4 lanes per channel pair");
-  static_assert(RUNS % SEG == 0, "segments must split the runs evenly");
+  static_assert(SW == 1 || SW == 2 || SW == 4 || SW == 8, "1, 2, 4 or 8 scan segments");
+  static_assert(RUNS % SW == 0, "segments must split the runs evenly");
+  static_assert(SW == 1 || NSCAN % 32 == 0, "scan groups must fill warps");
+  static_assert(NSCAN <= NT, "not enough threads for the scan groups");
   static_assert(NT % 32 == 0 && NT <= 1024, "bad block size");
   static_assert(RUNS % RW == 0, "runs must fill warps");
   static_assert(CT % 32 == 0 && NT >= CT, "look-back needs CT threads");
@@ -132,11 +136,31 @@ struct TileCfg {
   static_assert(kBoxBytes % 128 == 0, "boxes must keep 128-byte alignment");
 };
 
+// Run-scan segments for a tile of RUNS runs, NT threads and CT channels: the
+// most groups (4, 2 or 1) that split the runs into segments of at least four
+// and leave room beside them for the CT look-back threads, which poll while
+// the groups scan.
+template <int RUNS, int NT, int CT>
+constexpr int scan_segments() {
+  return (RUNS % 4 == 0 && RUNS / 4 >= 4 && 4 * (CT / 2) + CT <= NT) ? 4
+         : (RUNS % 2 == 0 && RUNS / 2 >= 4 && 2 * (CT / 2) + CT <= NT) ? 2
+                                                                          : 1;
+}
+
 // Shared-memory plan of the forward kernel: two stages of {a, v, q} boxes.
+// Misc area after the stage buffers: the carry per channel (CT floats), the
+// run-scan segment maps (SW x CT/2 float4), then barriers, tile infos, tag.
+template <typename Cfg>
+struct MiscPlan {
+  static constexpr size_t kSeg = Cfg::CT * sizeof(float);
+  static constexpr size_t kBars = kSeg + size_t(Cfg::SW) * Cfg::NP * sizeof(float4);
+  static constexpr size_t kBytes = kBars + 128;
+};
+
 template <typename Cfg>
 struct FwdSmem {
   static constexpr size_t kStage = 3 * size_t(Cfg::kBoxBytes);
-  static constexpr size_t kMisc = Cfg::CT * sizeof(float) + 128;
+  static constexpr size_t kMisc = MiscPlan<Cfg>::kBytes;
   static constexpr size_t kBytes = 2 * kStage + kMisc + 128;   // +128 for alignment
 };
 
@@ -145,7 +169,7 @@ template <typename Cfg>
 struct BwdSmem {
   static constexpr size_t kStage = 2 * size_t(Cfg::kBoxBytes);
   static constexpr size_t kQdy = 2 * size_t(Cfg::kBoxBytes);
-  static constexpr size_t kMisc = Cfg::CT * sizeof(float) + 128;
+  static constexpr size_t kMisc = MiscPlan<Cfg>::kBytes;
   static constexpr size_t kBytes = 2 * kStage + kQdy + kMisc + 128;
 };
 
@@ -210,67 +234,87 @@ __device__ __forceinline__ void scan_load8(const float *scan, int run, int ch, f
   }
 }
 
-// Scan over the runs of the channel pair (2 c2, 2 c2 + 1), packed, by SEG
-// consecutive lanes: lane `seg` serially scans the runs [seg RS, (seg+1) RS)
-// of the processing order (RS = RUNS / SEG; oldest run first, or latest first
-// for kReverse), the segment maps are combined across the lanes by shuffles,
-// and each lane folds its segment's prefix into its runs.  Every entry is
-// replaced by its exclusive prefix over the tile.  Returns in each lane the
-// prefix at the start of its own segment (sP, sS) and the tile map (tP, tS).
-template <int CT, int RUNS, int SEG, bool kReverse>
-__device__ __forceinline__ void scan_runs(float *scan, int c2, int seg, float2 &sP, float2 &sS, float2 &tP,
-                                          float2 &tS) {
-  constexpr int RS = RUNS / SEG;
-  float *col = scan + scan_pos<CT>(0, 2 * c2);   // P pair at col[0..1], S pair at col[2..3]
-  auto entry = [&](int j) -> float2 * {
+// Named barrier `id` over the first `n` threads of the CTA (n a multiple of 32).
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// The run scan of channel pair (2 c2, 2 c2 + 1), packed, part one: lane c2 of
+// group g serially scans the runs [g RS, (g+1) RS) of the processing order
+// (RS = RUNS / SW; oldest run first, or latest first for kReverse), replacing
+// each entry by its exclusive prefix within the segment.  The groups then
+// exchange their segment maps through `seg_s` ([SW][CT/2] float4: P pair, S
+// pair) under named barrier 2, and each lane returns the map of the segments
+// before its own (eP, eS), the tile map (tP, tS, valid in the last group) and
+// the map of the first SW/2 segments (mP, mS, valid in the last group).  The
+// tile map is known here, before part two, so it can be published at once.
+template <int CT, int RUNS, int SW, bool kReverse>
+__device__ __forceinline__ void scan_runs(float *scan, float4 *seg_s, int c2, int g, float2 &eP, float2 &eS,
+                                          float2 &tP, float2 &tS, float2 &mP, float2 &mS) {
+  constexpr int RS = RUNS / SW;
+  constexpr int NP = CT / 2;
+  float4 *col = reinterpret_cast<float4 *>(scan + scan_pos<CT>(0, 2 * c2));   // (P pair, S pair)
+  auto entry = [&](int j) -> float4 * {
     const int r = kReverse ? RUNS - 1 - j : j;
-    return reinterpret_cast<float2 *>(col + r * CT * 2);
+    return col + r * (CT / 2);
   };
   float2 cp = splat(1.0f), cs = splat(0.0f);
 #pragma unroll
   for (int k = 0; k < RS; ++k) {
-    float2 *pp = entry(seg * RS + k);
-    const float2 ep = pp[0], es = pp[1];
-    pp[0] = cp;
-    pp[1] = cs;
-    cs = fma2(ep, cs, es);
-    cp = mul2(cp, ep);
+    float4 *pp = entry(g * RS + k);
+    const float4 e = *pp;
+    *pp = make_float4(cp.x, cp.y, cs.x, cs.y);
+    cs = fma2(make_float2(e.x, e.y), cs, make_float2(e.z, e.w));
+    cp = mul2(cp, make_float2(e.x, e.y));
   }
-  if constexpr (SEG == 1) {
-    sP = splat(1.0f);
-    sS = splat(0.0f);
+  eP = splat(1.0f);
+  eS = splat(0.0f);
+  mP = splat(1.0f);
+  mS = splat(0.0f);
+  if constexpr (SW == 1) {
     tP = cp;
     tS = cs;
   } else {
-    // Inclusive composition of the segment maps over lanes 0..seg (a later
-    // map applied after the earlier ones), then shifted to exclusive.
-    float2 iP = cp, iS = cs;
+    seg_s[g * NP + c2] = make_float4(cp.x, cp.y, cs.x, cs.y);
+    named_sync(2, SW * NP);
 #pragma unroll
-    for (int o = 1; o < SEG; o <<= 1) {
-      const float2 oP = shfl_up2(iP, o, SEG), oS = shfl_up2(iS, o, SEG);
-      if (seg >= o) {
-        iS = fma2(iP, oS, iS);
-        iP = mul2(iP, oP);
+    for (int j = 0; j < SW - 1; ++j) {   // earlier segments, oldest applied first
+      if (j < g) {
+        if (j == SW / 2) {
+          mP = eP;
+          mS = eS;
+        }
+        const float4 m = seg_s[j * NP + c2];
+        eS = fma2(make_float2(m.x, m.y), eS, make_float2(m.z, m.w));
+        eP = mul2(eP, make_float2(m.x, m.y));
       }
     }
-    float2 eP = shfl_up2(iP, 1, SEG), eS = shfl_up2(iS, 1, SEG);
-    if (seg == 0) {
-      eP = splat(1.0f);
-      eS = splat(0.0f);
+    if (g == SW / 2) {
+      mP = eP;
+      mS = eS;
     }
-    tP = shfl_idx2(iP, SEG - 1, SEG);
-    tS = shfl_idx2(iS, SEG - 1, SEG);
-    if (seg > 0) {
+    tP = mul2(cp, eP);
+    tS = fma2(cp, eS, cs);
+  }
+}
+
+// Part two: fold the map of the earlier segments into the segment's entries,
+// which then hold their exclusive prefix over the whole tile.
+template <int CT, int RUNS, int SW, bool kReverse>
+__device__ __forceinline__ void scan_runs_fold(float *scan, int c2, int g, float2 eP, float2 eS) {
+  if constexpr (SW > 1) {
+    constexpr int RS = RUNS / SW;
+    if (g == 0) return;
+    float4 *col = reinterpret_cast<float4 *>(scan + scan_pos<CT>(0, 2 * c2));
 #pragma unroll
-      for (int k = 0; k < RS; ++k) {
-        float2 *pp = entry(seg * RS + k);
-        const float2 lp = pp[0], ls = pp[1];
-        pp[0] = mul2(lp, eP);
-        pp[1] = fma2(lp, eS, ls);
-      }
+    for (int k = 0; k < RS; ++k) {
+      const int j = g * RS + k;
+      float4 *pp = col + (kReverse ? RUNS - 1 - j : j) * (CT / 2);
+      const float4 e = *pp;
+      const float2 P = mul2(make_float2(e.x, e.y), eP);
+      const float2 S = fma2(make_float2(e.x, e.y), eS, make_float2(e.z, e.w));
+      *pp = make_float4(P.x, P.y, S.x, S.y);
     }
-    sP = eP;
-    sS = eS;
   }
 }
 
@@ -427,19 +471,22 @@ __device__ __forceinline__ float2 gate_A(float2 c) { return MODE == 0 ? c : sub2
 // and stores the chunk-end state of every slot it covers (the backward's
 // checkpoints), so taller forward tiles leave the workspace layout alone.
 // ===========================================================================
-template <typename T, int MODE, int LPH, int VPR, int L, int K, int SUB, int SEG>
+template <typename T, int MODE, int LPH, int VPR, int L, int K, int SUB, int SW>
 __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR * (L / K) <= 128) ? 4 : (VPR * (L / K) <= 256) ? 2 : 1)
     esa_scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_q, const FwdArgs args) {
   static_assert(SUB == 1 || SUB == 2, "a forward tile spans one or two slots");
-  using Cfg = TileCfg<T, LPH, VPR, L, K, SEG>;
+  using Cfg = TileCfg<T, LPH, VPR, L, K, SW>;
   using Sm = FwdSmem<Cfg>;
-  constexpr int CT = Cfg::CT, RUNS = Cfg::RUNS;
+  using Mp = MiscPlan<Cfg>;
+  constexpr int CT = Cfg::CT, RUNS = Cfg::RUNS, NP = Cfg::NP;
 
   extern __shared__ unsigned char smem_raw[];
   unsigned char *base = smem_aligned128(smem_raw);
-  float *es_s = reinterpret_cast<float *>(base + 2 * Sm::kStage);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(es_s + CT);     // [2]
+  unsigned char *misc_p = base + 2 * Sm::kStage;
+  float *es_s = reinterpret_cast<float *>(misc_p);
+  float4 *seg_s = reinterpret_cast<float4 *>(misc_p + Mp::kSeg);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(misc_p + Mp::kBars);     // [2]
   TileInfo *info_s = reinterpret_cast<TileInfo *>(bar + 2);    // [2], per stage
   unsigned *tag_s = reinterpret_cast<unsigned *>(info_s + 2);
 
@@ -504,6 +551,21 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     unsigned long long early = 0ull;
     if (lb_thread && chunk > 0) early = ld_relaxed_b64(&ws.incl_f[(slot_end - SUB) * CT + (tid - Cfg::LB0)]);
 
+    // The carry entering the chunk, one channel per look-back thread.
+    auto resolve_carry = [&]() {
+      const int c = tid - Cfg::LB0;
+      const int cg = c0 + c;
+      float E_start;
+      if (chunk == 0) {
+        E_start = (args.E_init != nullptr && cg < sh.C) ? args.E_init[static_cast<long>(b) * sh.C + cg] : 0.0f;
+      } else if (tag_of(early) == tag) {   // what the look-back returns at distance 1
+        E_start = val_of(early);
+      } else {
+        E_start = carry_in(ws.incl_f, ws.agg, slot_end * CT + c, -static_cast<long>(SUB) * CT, chunk, tag,
+                           &hdr->abort[0], &hdr->status);
+      }
+      es_s[c] = E_start;
+    };
     mbar_wait_bounded(&bar[s], (phase >> s) & 1u, &hdr->status);
     phase ^= 1u << s;
 
@@ -534,43 +596,27 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     __syncthreads();
 
     // ---- scan over runs, look-back, publish --------------------------------
-    // Scan lanes: SEG lanes per channel pair c2; the last one publishes.
-    const int c2 = tid / SEG, seg = tid % SEG;
-    const bool publisher = tid < Cfg::NSCAN && seg == SEG - 1;
-    float2 sP = splat(1.0f), sS = splat(0.0f), tP = splat(1.0f), tS = splat(0.0f);
+    // Scan lanes: lane c2 of segment group g; the last group publishes.
+    const int c2 = tid % NP, g = tid / NP;
+    const bool publisher = tid < Cfg::NSCAN && g == SW - 1;
+    float2 tP = splat(1.0f), tS = splat(0.0f);
     float2 mP = splat(1.0f), mS = splat(0.0f);   // prefix at the middle run (SUB == 2)
     if (tid < Cfg::NSCAN) {
-      scan_runs<CT, RUNS, SEG, false>(scan_s, c2, seg, sP, sS, tP, tS);
-      if constexpr (SUB == 2) {
-        if constexpr (SEG == 1) {   // this lane wrote the entry itself
-          const float2 *pm = reinterpret_cast<const float2 *>(scan_s + scan_pos<CT>(RUNS / 2, 2 * c2));
-          mP = pm[0];
-          mS = pm[1];
-        } else {                    // the middle run starts segment SEG / 2
-          mP = shfl_idx2(sP, SEG / 2, SEG);
-          mS = shfl_idx2(sS, SEG / 2, SEG);
-        }
-      }
+      float2 eP, eS;
+      scan_runs<CT, RUNS, SW, false>(scan_s, seg_s, c2, g, eP, eS, tP, tS, mP, mS);
       if (chunk > 0 && publisher) {   // the pair's chunk map, for successors' look-backs
         const long at = slot_end * CT + 2 * c2;
         st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tP.x, tag), pack_tag(tS.x, tag)));
         st_relaxed_v2b64(&ws.agg[at + 1], make_ulonglong2(pack_tag(tP.y, tag), pack_tag(tS.y, tag)));
       }
-    }
-    if (lb_thread) {   // carry entering the chunk, one channel each
-      const int c = tid - Cfg::LB0;
-      const int cg = c0 + c;
-      float E_start;
-      if (chunk == 0) {
-        E_start = (args.E_init != nullptr && cg < sh.C) ? args.E_init[static_cast<long>(b) * sh.C + cg] : 0.0f;
-      } else if (tag_of(early) == tag) {   // what the look-back returns at distance 1
-        E_start = val_of(early);
-      } else {
-        E_start = carry_in(ws.incl_f, ws.agg, slot_end * CT + c, -static_cast<long>(SUB) * CT, chunk, tag,
-                           &hdr->abort[0], &hdr->status);
+      scan_runs_fold<CT, RUNS, SW, false>(scan_s, c2, g, eP, eS);
+      if constexpr (SUB == 2 && SW == 1) {   // this lane wrote the middle run's entry itself
+        const float2 *pm = reinterpret_cast<const float2 *>(scan_s + scan_pos<CT>(RUNS / 2, 2 * c2));
+        mP = pm[0];
+        mS = pm[1];
       }
-      es_s[c] = E_start;
     }
+    if (lb_thread) resolve_carry();   // concurrently with the run scan
     __syncthreads();
     // The ticket of the tile after next is taken only now: tickets then follow
     // the order in which CTAs really reach their tiles more closely, so a
@@ -593,28 +639,30 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     }
 
     // ---- pass 2: exact states and the readout ------------------------------
-    float2 E[4];
-    run_carry<CT>(scan_s, es_s, pos.run, pos.ch, E);
-    const bool ch_ok = (c0 + pos.ch) < sh.C;
-    const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
+    {
+      float2 E[4];
+      run_carry<CT>(scan_s, es_s, pos.run, pos.ch, E);
+      const bool ch_ok = (c0 + pos.ch) < sh.C;
+      const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
 #pragma unroll
-    for (int i = 0; i < K; ++i) {
-      const int r = pos.row0 + i;
-      const bool valid = (t0 + r) < sh.T;
-      float2 vv[4], qq[4];
-      Io<T>::load8(v_s + r * CT + pos.ch, vv);
-      Io<T>::load8(q_s + r * CT + pos.ch, qq);
-      float2 ss = splat(0.0f);
+      for (int i = 0; i < K; ++i) {
+        const int r = pos.row0 + i;
+        const bool valid = (t0 + r) < sh.T;
+        float2 vv[4], qq[4];
+        Io<T>::load8(v_s + r * CT + pos.ch, vv);
+        Io<T>::load8(q_s + r * CT + pos.ch, qq);
+        float2 ss = splat(0.0f);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        E[q] = rec_step<MODE>(Ar[i][q], E[q], vv[q]);
-        ss = fma2(E[q], E[q], ss);
+        for (int q = 0; q < 4; ++q) {
+          E[q] = rec_step<MODE>(Ar[i][q], E[q], vv[q]);
+          ss = fma2(E[q], E[q], ss);
+        }
+        const float rr = rsqrt_approx(__fmaf_rn(head_sum2<LPH>(ss), sh.inv_D, kEps));
+        float2 yv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) yv[q] = mul2(qq[q], mul2(E[q], splat(rr)));
+        if (valid && ch_ok) Io<T>::store8(yg + gbase + static_cast<long>(r) * sh.C, yv);
       }
-      const float rr = rsqrt_approx(__fmaf_rn(head_sum2<LPH>(ss), sh.inv_D, kEps));
-      float2 yv[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) yv[q] = mul2(qq[q], mul2(E[q], splat(rr)));
-      if (valid && ch_ok) Io<T>::store8(yg + gbase + static_cast<long>(r) * sh.C, yv);
     }
 
     // ---- refill this stage --------------------------------------------------
@@ -649,21 +697,25 @@ __device__ __forceinline__ void get_ghat(const T *q_slot, const T *dy_slot, floa
 // ===========================================================================
 // Backward scan (persistent).
 // ===========================================================================
-template <typename T, int MODE, int LPH, int VPR, int L, int K>
+template <typename T, int MODE, int LPH, int VPR, int L, int K, int SW, int SUB>
 __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR * (L / K) <= 128) ? 4 : (VPR * (L / K) <= 256) ? 2 : 1)
     esa_scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dy,
                         const BwdArgs args) {
-  using Cfg = TileCfg<T, LPH, VPR, L, K>;
+  static_assert(SUB == 1 || SUB == 2, "a backward tile spans one or two slots");
+  using Cfg = TileCfg<T, LPH, VPR, L, K, SW>;
   using Sm = BwdSmem<Cfg>;
-  constexpr int CT = Cfg::CT, RUNS = Cfg::RUNS;
+  using Mp = MiscPlan<Cfg>;
+  constexpr int CT = Cfg::CT, RUNS = Cfg::RUNS, NP = Cfg::NP;
 
   extern __shared__ unsigned char smem_raw[];
   unsigned char *base = smem_aligned128(smem_raw);
   T *q_s = reinterpret_cast<T *>(base + 2 * Sm::kStage);
   T *dy_s = q_s + L * CT;
-  float *es_s = reinterpret_cast<float *>(base + 2 * Sm::kStage + Sm::kQdy);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(es_s + CT);     // [0..1] a/v stages, [2] q/dy
+  unsigned char *misc_p = base + 2 * Sm::kStage + Sm::kQdy;
+  float *es_s = reinterpret_cast<float *>(misc_p);
+  float4 *seg_s = reinterpret_cast<float4 *>(misc_p + Mp::kSeg);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(misc_p + Mp::kBars);     // [0..1] a/v stages, [2] q/dy
   TileInfo *info_s = reinterpret_cast<TileInfo *>(bar + 4);    // [2], per a/v stage
   unsigned *tag_s = reinterpret_cast<unsigned *>(info_s + 2);
 
@@ -677,7 +729,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
   };
   // Thread 0: decode a ticket into the stage's tile info and start its a/v loads.
   auto issue_av = [&](int stage, int tile) {
-    const TileInfo ti = decode_tile<true, 1>(tile, sh, CT, L);
+    const TileInfo ti = decode_tile<true, SUB>(tile, sh, CT, L);
     info_s[stage] = ti;
     if (tile >= sh.ntiles) return;
     mbar_expect_tx(&bar[stage], 2 * Cfg::kBoxBytes);
@@ -765,9 +817,13 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     scan_store8<CT>(scan_s, pos.run, pos.ch, P, S);
     if (tid < CT) es_s[tid] = E_ck;
     __syncthreads();
+    // Scan lanes: lane c2 of segment group g; the last group publishes.
+    const int c2 = tid % NP, g = tid / NP;
+    const bool publisher = tid < Cfg::NSCAN && g == SW - 1;
     if (tid < Cfg::NSCAN) {
-      float2 sP, sS, tP, tS;
-      scan_runs<CT, RUNS, 1, false>(scan_s, tid, 0, sP, sS, tP, tS);
+      float2 eP, eS, tP, tS, mP, mS;
+      scan_runs<CT, RUNS, SW, false>(scan_s, seg_s, c2, g, eP, eS, tP, tS, mP, mS);
+      scan_runs_fold<CT, RUNS, SW, false>(scan_s, c2, g, eP, eS);
     }
     __syncthreads();
 
@@ -816,11 +872,13 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
       }
     }
 
+
     // Look-back threads read the nearest later chunk's carry now, a pass ahead
     // of the look-back (see the forward).
     const bool lb_thread = tid >= Cfg::LB0 && tid < Cfg::LB0 + CT;
     unsigned long long early = 0ull;
-    if (lb_thread && chunk < sh.nchunks - 1) early = ld_relaxed_b64(&ws.incl_b[(slot + 1) * CT + (tid - Cfg::LB0)]);
+    if (lb_thread && chunk < sh.nchunks - 1)
+      early = ld_relaxed_b64(&ws.incl_b[(slot + SUB) * CT + (tid - Cfg::LB0)]);
 
     // ---- R1: the run's reverse map h -> P h + hl ----------------------------
     {
@@ -844,14 +902,16 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
 
     // ---- reverse scan over runs, look-back towards later chunks -------------
     {
-      float2 sP, sS, tP = splat(1.0f), tS = splat(0.0f);
+      float2 tP = splat(1.0f), tS = splat(0.0f);
       if (tid < Cfg::NSCAN) {
-        scan_runs<CT, RUNS, 1, true>(scan_s, tid, 0, sP, sS, tP, tS);
-        if (chunk < sh.nchunks - 1) {
-          const long at = slot * CT + 2 * tid;
+        float2 eP, eS, mP, mS;
+        scan_runs<CT, RUNS, SW, true>(scan_s, seg_s, c2, g, eP, eS, tP, tS, mP, mS);
+        if (chunk < sh.nchunks - 1 && publisher) {   // the pair's reverse chunk map
+          const long at = slot * CT + 2 * c2;
           st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tP.x, tag), pack_tag(tS.x, tag)));
           st_relaxed_v2b64(&ws.agg[at + 1], make_ulonglong2(pack_tag(tP.y, tag), pack_tag(tS.y, tag)));
         }
+        scan_runs_fold<CT, RUNS, SW, true>(scan_s, c2, g, eP, eS);
       }
       if (lb_thread) {
         const int c = tid - Cfg::LB0;
@@ -862,18 +922,18 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
         } else if (tag_of(early) == tag) {
           H_in = val_of(early);
         } else {
-          H_in = carry_in(ws.incl_b, ws.agg, slot * CT + c, CT, sh.nchunks - 1 - chunk, tag, &hdr->abort[1],
-                          &hdr->status);
+          H_in = carry_in(ws.incl_b, ws.agg, slot * CT + c, static_cast<long>(SUB) * CT, sh.nchunks - 1 - chunk,
+                          tag, &hdr->abort[1], &hdr->status);
         }
         es_s[c] = H_in;
       }
       __syncthreads();
-      if (tid < Cfg::NSCAN) {
-        const float2 H_out = fma2(tP, reinterpret_cast<const float2 *>(es_s)[tid], tS);
-        const long at = slot * CT + 2 * tid;
+      if (publisher) {
+        const float2 H_out = fma2(tP, reinterpret_cast<const float2 *>(es_s)[c2], tS);
+        const long at = slot * CT + 2 * c2;
         st_relaxed_v2b64(reinterpret_cast<ulonglong2 *>(&ws.incl_b[at]),
                          make_ulonglong2(pack_tag(H_out.x, tag), pack_tag(H_out.y, tag)));
-        const int cg = c0 + 2 * tid;
+        const int cg = c0 + 2 * c2;
         if (chunk == 0 && args.dE_init != nullptr && cg < sh.C)
           *reinterpret_cast<float2 *>(&args.dE_init[static_cast<long>(b) * sh.C + cg]) = H_out;
       }

@@ -23,6 +23,13 @@ template <typename T, int VPR>
 constexpr int fwd_sub() { return (sizeof(T) == 2 && VPR == 8) ? 2 : 1; }
 inline int fwd_slots_per_tile(int dtype, int D) { return (dtype != 0 && tile_cols(D) == 64) ? 2 : 1; }
 
+// Slots per backward tile: the same rule.  A backward tile keeps its
+// look-back words at its first slot (the end of the tile in processing order)
+// and replays from the checkpoint of the slot before it.
+template <typename T, int VPR>
+constexpr int bwd_sub() { return fwd_sub<T, VPR>(); }
+inline int bwd_slots_per_tile(int dtype, int D) { return fwd_slots_per_tile(dtype, D); }
+
 // Launch the forward / backward scan for (dtype, mode, D).  The tensor maps
 // describe a, v, q (and dy) as [B][T][C] boxes of [L][CT].  Return 0 or a
 // negative esa_status.
