@@ -53,6 +53,8 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the prefill + decode (esa_step) measurement reported under detail.decode")
     ap.add_argument("--batch", type=int, default=None,
                     help="run a smaller batch of the same workload (profiling cases only)")
     ap.add_argument("--seq", type=int, default=None,
@@ -259,6 +261,94 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+# Prefill + decode: esa_scan_fwd on a prompt, then one-token esa_step calls
+# (the decode workload: direct mode, fp16, B=64, H=4, D=32, 256 steps).
+# ---------------------------------------------------------------------------
+
+def measure_decode(dev, reps=5):
+    """Prefill tokens/s and per-step decode time, eager and as a CUDA graph.
+
+    Each decode step moves B*C*(4s + 8) bytes (read a_t, v_t, q_t and the
+    float32 state; write y_t and the state): 131 KB here, so a step is bound
+    by launch and latency, not by HBM; the graph removes the host launch cost.
+    """
+    import torch
+
+    from gated_linear_recurrence_b200 import esa, inputs
+    w = inputs.WORKLOADS["direct_f16_B64_H4_D32_prefill_decode"]
+    B, H, D, T, n = w.B, w.H, w.D, max(w.prompts), w.steps
+    x = inputs.make_scan_inputs(B, T, H, D, w.dtype, w.a_mean, w.seed, with_dy=False, device=dev)
+    g = x["generator"]
+    steps = [inputs.make_step_inputs(B, H, D, w.dtype, w.a_mean, generator=g, device=dev) for _ in range(n)]
+    y = torch.empty_like(x["a"])
+    Ef = torch.empty(B, H, D, dtype=torch.float32, device=dev)
+    ws = esa.new_workspace(B, T, H, D, x["a"].dtype, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def prefill():
+        esa.esa_scan_fwd(x["a"], x["v"], x["q"], y=y, E_final=Ef, mode=w.mode, workspace=ws)
+
+    for _ in range(3):
+        prefill()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        prefill()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    prefill_ms = e0.elapsed_time(e1) / reps
+    esa.esa_check(ws)
+
+    E = Ef.clone()
+    ys = [torch.empty_like(st["a"]) for st in steps]
+
+    def decode():
+        for st, yt in zip(steps, ys):
+            esa.esa_step(st["a"], st["v"], st["q"], E, y_t=yt, mode=w.mode)
+
+    decode()   # warm-up (also fills the library's per-device caches before capture)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        decode()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    eager_us = 1e3 * e0.elapsed_time(e1) / (reps * n)
+
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        decode()
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        decode()
+    graph.replay()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    graph_us = 1e3 * e0.elapsed_time(e1) / (reps * n)
+    del graph
+
+    s = x["a"].element_size()
+    step_bytes = B * H * D * (4 * s + 8)
+    return {"workload": w.name, "B": B, "H": H, "D": D, "mode": "direct", "io_dtype": w.dtype,
+            "prefill_T": T, "prefill_ms": prefill_ms, "prefill_tokens_per_s": B * T / (prefill_ms / 1e3),
+            "prefill_GBs": 4 * s * H * D * B * T / (prefill_ms / 1e3) / 1e9,
+            "decode_steps": n, "bytes_per_step": step_bytes,
+            "eager_us_per_step": eager_us, "graph_us_per_step": graph_us,
+            "graph_tokens_per_s": B / (graph_us / 1e6),
+            "graph_GBs": step_bytes / (graph_us / 1e6) / 1e9,
+            "note": "decode steps are launch/latency bound (131 KB per step); eager time includes the "
+                    "Python binding's launch cost"}
+
+
+# ---------------------------------------------------------------------------
 # Our arm.
 # ---------------------------------------------------------------------------
 
@@ -384,6 +474,10 @@ def run_ours(args):
                "path": "pinned host -> esa_scan_fwd -> esa_scan_bwd -> pinned host, one stream, device-timed"}
         del h_in, h_out, h_st, d_in
 
+    decode = None
+    if not args.no_decode:
+        decode = measure_decode(dev)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w)
@@ -399,7 +493,8 @@ def run_ours(args):
         "detail": {"fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "fwd_GBs": fwd_bytes / (fwd_ms / 1e3) / 1e9,
                    "bwd_GBs": bwd_bytes / (bwd_ms / 1e3) / 1e9, "step_GBs": step_gbs,
                    "step_frac_of_measured_peak": step_gbs / peak, "step_frac_of_nominal_8TBs":
-                   step_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes_per_step": fwd_bytes + bwd_bytes},
+                   step_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes_per_step": fwd_bytes + bwd_bytes,
+                   "decode": decode},
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": 2 * K,

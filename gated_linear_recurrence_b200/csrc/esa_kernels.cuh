@@ -245,12 +245,12 @@ __device__ __forceinline__ void named_sync(int id, int n) {
 // each entry by its exclusive prefix within the segment.  The groups then
 // exchange their segment maps through `seg_s` ([SW][CT/2] float4: P pair, S
 // pair) under named barrier 2, and each lane returns the map of the segments
-// before its own (eP, eS), the tile map (tP, tS, valid in the last group) and
-// the map of the first SW/2 segments (mP, mS, valid in the last group).  The
-// tile map is known here, before part two, so it can be published at once.
+// before its own (eP, eS: the prefix at the start of its segment) and the tile
+// map (tP, tS, valid in the last group).  The tile map is known here, before
+// part two, so it can be published at once.
 template <int CT, int RUNS, int SW, bool kReverse>
 __device__ __forceinline__ void scan_runs(float *scan, float4 *seg_s, int c2, int g, float2 &eP, float2 &eS,
-                                          float2 &tP, float2 &tS, float2 &mP, float2 &mS) {
+                                          float2 &tP, float2 &tS) {
   constexpr int RS = RUNS / SW;
   constexpr int NP = CT / 2;
   float4 *col = reinterpret_cast<float4 *>(scan + scan_pos<CT>(0, 2 * c2));   // (P pair, S pair)
@@ -269,8 +269,6 @@ __device__ __forceinline__ void scan_runs(float *scan, float4 *seg_s, int c2, in
   }
   eP = splat(1.0f);
   eS = splat(0.0f);
-  mP = splat(1.0f);
-  mS = splat(0.0f);
   if constexpr (SW == 1) {
     tP = cp;
     tS = cs;
@@ -280,18 +278,10 @@ __device__ __forceinline__ void scan_runs(float *scan, float4 *seg_s, int c2, in
 #pragma unroll
     for (int j = 0; j < SW - 1; ++j) {   // earlier segments, oldest applied first
       if (j < g) {
-        if (j == SW / 2) {
-          mP = eP;
-          mS = eS;
-        }
         const float4 m = seg_s[j * NP + c2];
         eS = fma2(make_float2(m.x, m.y), eS, make_float2(m.z, m.w));
         eP = mul2(eP, make_float2(m.x, m.y));
       }
-    }
-    if (g == SW / 2) {
-      mP = eP;
-      mS = eS;
     }
     tP = mul2(cp, eP);
     tS = fma2(cp, eS, cs);
@@ -475,7 +465,8 @@ template <typename T, int MODE, int LPH, int VPR, int L, int K, int SUB, int SW>
 __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR * (L / K) <= 128) ? 4 : (VPR * (L / K) <= 256) ? 2 : 1)
     esa_scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_q, const FwdArgs args) {
-  static_assert(SUB == 1 || SUB == 2, "a forward tile spans one or two slots");
+  static_assert(SUB == 1 || SUB == 2 || SUB == 4, "a forward tile spans one, two or four slots");
+  static_assert(SUB <= 2 || SW % SUB == 0, "taller tiles need a scan segment starting at every slot");
   using Cfg = TileCfg<T, LPH, VPR, L, K, SW>;
   using Sm = FwdSmem<Cfg>;
   using Mp = MiscPlan<Cfg>;
@@ -600,20 +591,19 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     const int c2 = tid % NP, g = tid / NP;
     const bool publisher = tid < Cfg::NSCAN && g == SW - 1;
     float2 tP = splat(1.0f), tS = splat(0.0f);
-    float2 mP = splat(1.0f), mS = splat(0.0f);   // prefix at the middle run (SUB == 2)
+    float2 eP = splat(1.0f), eS = splat(0.0f);   // prefix at the start of the lane's segment
     if (tid < Cfg::NSCAN) {
-      float2 eP, eS;
-      scan_runs<CT, RUNS, SW, false>(scan_s, seg_s, c2, g, eP, eS, tP, tS, mP, mS);
+      scan_runs<CT, RUNS, SW, false>(scan_s, seg_s, c2, g, eP, eS, tP, tS);
       if (chunk > 0 && publisher) {   // the pair's chunk map, for successors' look-backs
         const long at = slot_end * CT + 2 * c2;
         st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tP.x, tag), pack_tag(tS.x, tag)));
         st_relaxed_v2b64(&ws.agg[at + 1], make_ulonglong2(pack_tag(tP.y, tag), pack_tag(tS.y, tag)));
       }
       scan_runs_fold<CT, RUNS, SW, false>(scan_s, c2, g, eP, eS);
-      if constexpr (SUB == 2 && SW == 1) {   // this lane wrote the middle run's entry itself
+      if constexpr (SUB == 2 && SW == 1) {   // the middle run's prefix: this lane wrote the entry itself
         const float2 *pm = reinterpret_cast<const float2 *>(scan_s + scan_pos<CT>(RUNS / 2, 2 * c2));
-        mP = pm[0];
-        mS = pm[1];
+        eP = pm[0];
+        eS = pm[1];
       }
     }
     if (lb_thread) resolve_carry();   // concurrently with the run scan
@@ -622,14 +612,25 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     // the order in which CTAs really reach their tiles more closely, so a
     // tile's predecessors are rarely behind it.  Pass 2 hides the round trip.
     if (tid == 0) next = atomicAdd(&hdr->ticket[0], 1u);
-    if (publisher) {   // chunk-end states of the pair at every slot the tile covers
+    // States of the pair at the slot boundaries inside the tile (the
+    // backward's checkpoints): boundary j of the SUB - 1 is the start of
+    // segment j SW / SUB, whose lanes hold the prefix up to it.
+    if constexpr (SUB > 1) {
+      if (tid < Cfg::NSCAN) {
+        int j = 0;
+        if constexpr (SW == 1) j = 1;   // SUB == 2: the middle run's prefix
+        else if (g > 0 && g % (SW / SUB) == 0) j = g / (SW / SUB);
+        if (j > 0 && chunk * SUB + j - 1 < sh.nslots) {
+          const float2 E_in = reinterpret_cast<const float2 *>(es_s)[c2];
+          const float2 E_mid = fma2(eP, E_in, eS);
+          st_relaxed_v2b64(reinterpret_cast<ulonglong2 *>(&ws.incl_f[(slot + j - 1) * CT + 2 * c2]),
+                           make_ulonglong2(pack_tag(E_mid.x, tag), pack_tag(E_mid.y, tag)));
+        }
+      }
+    }
+    if (publisher) {   // chunk-end state of the pair
       const float2 E_in = reinterpret_cast<const float2 *>(es_s)[c2];
       const float2 E_end = fma2(tP, E_in, tS);
-      if constexpr (SUB == 2) {   // the slot ending halfway through the tile
-        const float2 E_mid = fma2(mP, E_in, mS);
-        st_relaxed_v2b64(reinterpret_cast<ulonglong2 *>(&ws.incl_f[slot * CT + 2 * c2]),
-                         make_ulonglong2(pack_tag(E_mid.x, tag), pack_tag(E_mid.y, tag)));
-      }
       if (chunk * SUB + SUB - 1 < sh.nslots)   // a ragged last tile may cover fewer slots
         st_relaxed_v2b64(reinterpret_cast<ulonglong2 *>(&ws.incl_f[slot_end * CT + 2 * c2]),
                          make_ulonglong2(pack_tag(E_end.x, tag), pack_tag(E_end.y, tag)));
@@ -821,8 +822,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     const int c2 = tid % NP, g = tid / NP;
     const bool publisher = tid < Cfg::NSCAN && g == SW - 1;
     if (tid < Cfg::NSCAN) {
-      float2 eP, eS, tP, tS, mP, mS;
-      scan_runs<CT, RUNS, SW, false>(scan_s, seg_s, c2, g, eP, eS, tP, tS, mP, mS);
+      float2 eP, eS, tP, tS;
+      scan_runs<CT, RUNS, SW, false>(scan_s, seg_s, c2, g, eP, eS, tP, tS);
       scan_runs_fold<CT, RUNS, SW, false>(scan_s, c2, g, eP, eS);
     }
     __syncthreads();
@@ -904,8 +905,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     {
       float2 tP = splat(1.0f), tS = splat(0.0f);
       if (tid < Cfg::NSCAN) {
-        float2 eP, eS, mP, mS;
-        scan_runs<CT, RUNS, SW, true>(scan_s, seg_s, c2, g, eP, eS, tP, tS, mP, mS);
+        float2 eP, eS;
+        scan_runs<CT, RUNS, SW, true>(scan_s, seg_s, c2, g, eP, eS, tP, tS);
         if (chunk < sh.nchunks - 1 && publisher) {   // the pair's reverse chunk map
           const long at = slot * CT + 2 * c2;
           st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tP.x, tag), pack_tag(tS.x, tag)));
