@@ -594,7 +594,10 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     float2 eP = splat(1.0f), eS = splat(0.0f);   // prefix at the start of the lane's segment
     if (tid < Cfg::NSCAN) {
       scan_runs<CT, RUNS, SW, false>(scan_s, seg_s, c2, g, eP, eS, tP, tS);
-      if (chunk > 0 && publisher) {   // the pair's chunk map, for successors' look-backs
+      // The pair's chunk map, for successors' look-backs.  The first tile of a
+      // chain needs none (its carry is E_init) and the last has no successor;
+      // a ragged last tile's slot_end may also lie past the chain's slots.
+      if (chunk > 0 && chunk < sh.nchunks - 1 && publisher) {
         const long at = slot_end * CT + 2 * c2;
         st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tP.x, tag), pack_tag(tS.x, tag)));
         st_relaxed_v2b64(&ws.agg[at + 1], make_ulonglong2(pack_tag(tP.y, tag), pack_tag(tS.y, tag)));
