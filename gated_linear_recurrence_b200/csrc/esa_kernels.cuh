@@ -123,6 +123,13 @@ struct TileCfg {
   // the scan when the block has room for both, else after it (LB0 = 0).
   static constexpr int NSCAN = SW * NP;
   static constexpr int LB0 = (NT >= ((NSCAN + 31) / 32) * 32 + CT) ? ((NSCAN + 31) / 32) * 32 : 0;
+  static constexpr int NW = NT / 32;               // warps per CTA
+  // The run-scan entries of run r (8 CT bytes at 8 CT r) cover exactly the
+  // gate-box rows of run r (K CT sizeof(T) bytes at the same offset) when
+  // K sizeof(T) == 8; a warp owns whole runs across all vectors when
+  // NVSEG == 1.  Then a warp may overwrite its own gate rows with its run maps
+  // as soon as its own lanes are done, without waiting for the CTA.
+  static constexpr bool kWarpScratch = (K * sizeof(T) == 8) && NVSEG == 1;
   static_assert(L % K == 0, "K must divide L");
   static_assert(SW == 1 || SW == 2 || SW == 4 || SW == 8, "1, 2, 4 or 8 scan segments");
   static_assert(RUNS % SW == 0, "segments must split the runs evenly");
@@ -480,6 +487,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
   uint64_t *bar = reinterpret_cast<uint64_t *>(misc_p + Mp::kBars);     // [2]
   TileInfo *info_s = reinterpret_cast<TileInfo *>(bar + 2);    // [2], per stage
   unsigned *tag_s = reinterpret_cast<unsigned *>(info_s + 2);
+  unsigned *done_s = tag_s + 1;   // [2] warps finished with the stage
+  unsigned *tk_s = tag_s + 3;     // [2] ticket that refills the stage
 
   const int tid = threadIdx.x;
   const ScanShape &sh = args.s;
@@ -510,6 +519,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     fence_proxy_async_smem();
     const unsigned tag = scan_prologue(hdr);
     *tag_s = tag;
+    done_s[0] = done_s[1] = 0u;
     const int t0 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[0], 1u)) : sh.ntiles;
     const int t1 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[0], 1u)) : sh.ntiles;
     issue(0, t0);
@@ -582,7 +592,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
         }
       }
     }
-    __syncthreads();   // the gate box is free from here on
+    // The gate rows are free from here on (only this warp read its own rows).
+    if constexpr (Cfg::kWarpScratch) __syncwarp(); else __syncthreads();
     scan_store8<CT>(scan_s, pos.run, pos.ch, P, S);
     __syncthreads();
 
@@ -670,10 +681,18 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     }
 
     // ---- refill this stage --------------------------------------------------
-    __syncthreads();   // everybody is done with stage s
-    if (tid == 0) {
-      fence_proxy_async_smem();   // generic writes (scan scratch) before the async refill
-      issue(s, static_cast<int>(next));
+    // No CTA barrier: every warp counts itself done with stage s, and the last
+    // one issues the refill (thread 0 leaves the ticket first).
+    if (tid == 0) tk_s[s] = next;
+    __syncwarp();
+    if ((tid & 31) == 0) {
+      __threadfence_block();
+      if (atomicAdd(&done_s[s], 1u) == Cfg::NW - 1) {
+        __threadfence_block();
+        done_s[s] = 0u;
+        fence_proxy_async_smem();   // generic writes (scan scratch) before the async refill
+        issue(s, static_cast<int>(*reinterpret_cast<volatile unsigned *>(&tk_s[s])));
+      }
     }
   }
   scan_epilogue(hdr, 0, tag != 0u);
@@ -722,6 +741,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
   uint64_t *bar = reinterpret_cast<uint64_t *>(misc_p + Mp::kBars);     // [0..1] a/v stages, [2] q/dy
   TileInfo *info_s = reinterpret_cast<TileInfo *>(bar + 4);    // [2], per a/v stage
   unsigned *tag_s = reinterpret_cast<unsigned *>(info_s + 2);
+  unsigned *done_s = tag_s + 1;   // [2] warps finished with the stage
+  unsigned *tk_s = tag_s + 3;     // [2] ticket that refills the stage
 
   const int tid = threadIdx.x;
   const ScanShape &sh = args.s;
@@ -758,6 +779,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     fence_proxy_async_smem();
     const unsigned tag = scan_prologue(hdr);
     *tag_s = tag;
+    done_s[0] = done_s[1] = 0u;
     const int t0 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[1], 1u)) : sh.ntiles;
     const int t1 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[1], 1u)) : sh.ntiles;
     issue_av(0, t0);
@@ -817,10 +839,13 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
         }
       }
     }
-    __syncthreads();
+    // The gate rows are free from here on (only this warp read its own rows).
+    if constexpr (Cfg::kWarpScratch) __syncwarp(); else __syncthreads();
     scan_store8<CT>(scan_s, pos.run, pos.ch, P, S);
-    if (tid < CT) es_s[tid] = E_ck;
     __syncthreads();
+    // The checkpoint carry goes in only now: every warp has left the previous
+    // tile (whose B1 read the array) by the barrier above.
+    if (tid < CT) es_s[tid] = E_ck;
     // Scan lanes: lane c2 of segment group g; the last group publishes.
     const int c2 = tid % NP, g = tid / NP;
     const bool publisher = tid < Cfg::NSCAN && g == SW - 1;
@@ -899,7 +924,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
           for (int q = 0; q < 4; ++q) hl[q] = mul2(gate_A<MODE>(Ar[i][q]), add2(gh[q], hl[q]));
         }
       }
-      __syncthreads();   // every thread has read its forward prefixes
+      // Each thread read (run_carry) and now overwrites only its own run's
+      // entries, so no barrier is needed between the two.
       scan_store8<CT>(scan_s, pos.run, pos.ch, P, hl);
     }
     __syncthreads();
@@ -997,11 +1023,18 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     }
 
     // ---- refill: next tile's q/dy, and this a/v stage -------------------------
-    __syncthreads();
-    if (tid == 0) {
-      fence_proxy_async_smem();   // generic smem writes before the async refills
-      if (info_s[s ^ 1].tile < sh.ntiles) issue_qdy(info_s[s ^ 1]);
-      issue_av(s, static_cast<int>(next));
+    // No CTA barrier: the last warp done with the tile refills (see the forward).
+    if (tid == 0) tk_s[s] = next;
+    __syncwarp();
+    if ((tid & 31) == 0) {
+      __threadfence_block();
+      if (atomicAdd(&done_s[s], 1u) == Cfg::NW - 1) {
+        __threadfence_block();
+        done_s[s] = 0u;
+        fence_proxy_async_smem();   // generic smem writes before the async refills
+        if (info_s[s ^ 1].tile < sh.ntiles) issue_qdy(info_s[s ^ 1]);
+        issue_av(s, static_cast<int>(*reinterpret_cast<volatile unsigned *>(&tk_s[s])));
+      }
     }
   }
   scan_epilogue(hdr, 1, tag != 0u);
