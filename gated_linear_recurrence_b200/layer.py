@@ -1,0 +1,130 @@
+"""PyTorch autograd wrapper and an ESA layer over the C ABI.
+
+* :func:`esa_scan` -- differentiable scan ``(a, v, q) -> (y, E_final)``: the
+  forward is ``esa_scan_fwd``, the backward ``esa_scan_bwd`` (the forward's
+  workspace, which holds the chunk checkpoints, is kept for it).
+* :class:`ESA` -- the sequence-mixing layer of "Entangled State Attention
+  v2.1", section 1 ("ESA layer": ``ESA(embd, head, ...)`` mapping
+  ``[B, T, embd]`` to ``[B, T, embd]``), computed as on the
+  "entangled-state-attention 0.1.0" page, section "Core idea":
+  gate logits ``a = x W_A``, values ``v = x W_V``, queries ``q = x W_Q``, the
+  recurrence (direct or controlled) over each head, and ``y = W_O(q * Norm(E))``
+  with Norm the per-head RMS.
+
+The projections are dense GEMMs outside the scan; they run as ordinary
+``torch.nn.Linear`` layers.  Every step of the recurrence and its readout runs
+in the CUDA library; there is no CPU path.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import esa as _esa
+
+__all__ = ["ESA", "esa_scan"]
+
+_MODES = {"direct": _esa.DIRECT, "controlled": _esa.CONTROLLED}
+
+
+class _EsaScanFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, a, v, q, E_init, mode):
+        a, v, q = a.contiguous(), v.contiguous(), q.contiguous()
+        E0 = None if E_init is None else E_init.detach().contiguous().float()
+        y, E_final, ws = _esa.esa_scan_fwd(a, v, q, mode=mode, E_init=E0)
+        ctx.mode = mode
+        ctx.ws = ws
+        ctx.has_E_init = E_init is not None
+        ctx.save_for_backward(a, v, q, E0 if E0 is not None else torch.empty(0, device=a.device))
+        return y, E_final
+
+    @staticmethod
+    def backward(ctx, dy, dE_final):
+        a, v, q, E0 = ctx.saved_tensors
+        E0 = E0 if ctx.has_E_init else None
+        if dy is None:
+            dy = torch.zeros_like(a)
+        dy = dy.to(a.dtype).contiguous()
+        dEf = None if dE_final is None else dE_final.float().contiguous()
+        da, dv, dq, dE0 = _esa.esa_scan_bwd(a, v, q, dy, ctx.ws, mode=ctx.mode, E_init=E0, dE_final=dEf,
+                                            want_dE_init=ctx.has_E_init)
+        ctx.ws = None
+        return da, dv, dq, (dE0 if ctx.has_E_init else None), None
+
+
+def esa_scan(a, v, q, mode="controlled", E_init=None):
+    """Differentiable scan of ``[B, T, H, D]`` CUDA tensors (float32, float16
+    or bfloat16).  Returns ``(y, E_final)``; ``E_final`` is float32
+    ``[B, H, D]``.  ``E_init`` (float32 ``[B, H, D]``) may require grad."""
+    m = _MODES[mode] if isinstance(mode, str) else int(mode)
+    return _EsaScanFn.apply(a, v, q, E_init, m)
+
+
+class ESA(torch.nn.Module):
+    """ESA sequence mixer: ``[B, T, embd] -> [B, T, embd]``.
+
+    Args:
+        embd: embedding width C.
+        head: number of heads H; the head dimension ``embd // head`` must be
+            one of 8, 16, 32, 64, 128, 256 (the library's head dimensions).
+        mode: ``"controlled"`` (default) or ``"direct"``.
+        bias: bias terms in the four projections.
+        scan_dtype: dtype the scan reads and writes (float16, bfloat16 or
+            float32); the state is float32 either way.  ``None`` keeps the
+            dtype of the projections' output.
+
+    ``forward(x, state=None, return_state=False)`` runs the whole sequence;
+    ``state`` (float32 ``[B, H, D]``) is the state before the first token and
+    ``return_state`` also returns the state after the last.  ``step(x_t,
+    state)`` is the one-token update for decoding: ``x_t`` is ``[B, embd]``,
+    ``state`` is updated in place and the output for the token returned.
+    """
+
+    def __init__(self, embd: int, head: int, mode: str = "controlled", bias: bool = False,
+                 scan_dtype: torch.dtype | None = None, device=None, dtype=None):
+        super().__init__()
+        if embd % head != 0:
+            raise ValueError("embd must be a multiple of head")
+        if embd // head not in (8, 16, 32, 64, 128, 256):
+            raise ValueError("head dimension embd // head must be one of 8, 16, 32, 64, 128, 256")
+        if mode not in _MODES:
+            raise ValueError("mode must be 'controlled' or 'direct'")
+        self.embd, self.head, self.mode = embd, head, mode
+        self.head_dim = embd // head
+        self.scan_dtype = scan_dtype
+        kw = {"device": device, "dtype": dtype}
+        self.W_A = torch.nn.Linear(embd, embd, bias=bias, **kw)
+        self.W_V = torch.nn.Linear(embd, embd, bias=bias, **kw)
+        self.W_Q = torch.nn.Linear(embd, embd, bias=bias, **kw)
+        self.W_O = torch.nn.Linear(embd, embd, bias=bias, **kw)
+
+    def _proj(self, x, shape):
+        dt = self.scan_dtype
+        out = []
+        for lin in (self.W_A, self.W_V, self.W_Q):
+            t = lin(x).reshape(shape)
+            out.append((t if dt is None else t.to(dt)).contiguous())
+        return out
+
+    def forward(self, x, state=None, return_state=False):
+        B, T, C = x.shape
+        if C != self.embd:
+            raise ValueError(f"expected last dimension {self.embd}, got {C}")
+        a, v, q = self._proj(x, (B, T, self.head, self.head_dim))
+        y, E = esa_scan(a, v, q, self.mode, E_init=state)
+        out = self.W_O(y.reshape(B, T, C).to(self.W_O.weight.dtype))
+        return (out, E) if return_state else out
+
+    @torch.no_grad()
+    def step(self, x_t, state):
+        B, C = x_t.shape
+        if C != self.embd:
+            raise ValueError(f"expected last dimension {self.embd}, got {C}")
+        a, v, q = self._proj(x_t, (B, self.head, self.head_dim))
+        y = _esa.esa_step(a, v, q, state, mode=_MODES[self.mode])
+        return self.W_O(y.reshape(B, C).to(self.W_O.weight.dtype))
+
+    def init_state(self, batch: int, device=None):
+        """A zero state ``[batch, head, head_dim]`` (float32)."""
+        return torch.zeros(batch, self.head, self.head_dim, dtype=torch.float32,
+                           device=device if device is not None else self.W_A.weight.device)

@@ -1,0 +1,99 @@
+"""The autograd scan and the ESA layer over the C ABI.
+
+* ``esa_scan`` forward values and every gradient (a, v, q, E_init) against the
+  fp64 oracle, for a loss that uses both y and E_final.
+* The ``ESA`` layer (projections + scan + readout + output projection) against
+  a float64 PyTorch reference written out as the plain per-token loop of the
+  "entangled-state-attention 0.1.0" page ("Core idea"), output and gradients
+  of the input and of all four weight matrices.
+* Decoding: a forward over a prompt returning its state, then one-token
+  ``step`` calls, equals one forward over prompt + tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_linear_recurrence_b200 import ESA, esa_scan, inputs
+from tests._parity import DT, TOL, assert_close, host64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("dt,mode", [("f32", "controlled"), ("f16", "direct"), ("bf16", "controlled")])
+def test_esa_scan_autograd_matches_oracle(cuda_device, dt, mode):
+    B, T, H, D = 2, 300, 4, 32
+    m = 1 if mode == "controlled" else 0
+    x = inputs.make_scan_inputs(B, T, H, D, dt, 1.0, 31)
+    a, v, q, w = (x[k].to(cuda_device).requires_grad_(k != "dy") for k in ("a", "v", "q", "dy"))
+    E0 = inputs.make_state(B, H, D, seed=32, scale=0.5).to(cuda_device).requires_grad_(True)
+    u = inputs.make_state(B, H, D, seed=33).to(cuda_device)
+    y, Ef = esa_scan(a, v, q, mode, E_init=E0)
+    loss = (y.float() * w.float()).sum() + (Ef * u).sum()
+    loss.backward()
+    f64 = lambda t: host64(t.detach())   # noqa: E731
+    y_r, Ef_r = oracle.scan_fwd(f64(a), f64(v), f64(q), m, E_init=f64(E0))
+    da_r, dv_r, dq_r, dE0_r = oracle.scan_bwd(f64(a), f64(v), f64(q), f64(w), m, E_init=f64(E0), dE_final=f64(u))
+    tol = TOL[DT[dt]]
+    assert_close(y, y_r, tol, "y")
+    assert_close(Ef, Ef_r, tol, "E_final")
+    assert_close(a.grad, da_r, tol, "da")
+    assert_close(v.grad, dv_r, tol, "dv")
+    assert_close(q.grad, dq_r, tol, "dq")
+    assert_close(E0.grad, dE0_r, tol, "dE_init")
+
+
+def _reference_layer(x, WA, WV, WQ, WO, H, mode, eps=1e-6):
+    """Float64 per-token loop: gates, values and queries by projection, the
+    recurrence per head, the per-head RMS readout and the output projection."""
+    B, T, C = x.shape
+    D = C // H
+    a = (x @ WA.T).reshape(B, T, H, D)
+    v = (x @ WV.T).reshape(B, T, H, D)
+    q = (x @ WQ.T).reshape(B, T, H, D)
+    E = torch.zeros(B, H, D, dtype=x.dtype)
+    ys = []
+    for t in range(T):
+        A = torch.sigmoid(a[:, t])
+        write = v[:, t] if mode == "direct" else (1.0 - A) * v[:, t]
+        E = A * E + write
+        r = torch.rsqrt(E.pow(2).mean(dim=-1, keepdim=True) + eps)
+        ys.append(q[:, t] * E * r)
+    y = torch.stack(ys, dim=1).reshape(B, T, C)
+    return y @ WO.T
+
+
+@pytest.mark.parametrize("mode", ["controlled", "direct"])
+def test_layer_matches_float64_reference(cuda_device, mode):
+    torch.manual_seed(5)
+    B, T, C, H = 2, 70, 64, 2
+    layer = ESA(C, H, mode=mode, device=cuda_device, dtype=torch.float32)
+    x = (torch.randn(B, T, C, device=cuda_device) * 0.5).requires_grad_(True)
+    g = torch.randn(B, T, C, device=cuda_device)
+    out = layer(x)
+    (out * g).sum().backward()
+
+    W = {n: getattr(layer, n).weight.detach().cpu().double().requires_grad_(True) for n in ("W_A", "W_V", "W_Q", "W_O")}
+    x64 = x.detach().cpu().double().requires_grad_(True)
+    ref = _reference_layer(x64, W["W_A"], W["W_V"], W["W_Q"], W["W_O"], H, mode)
+    (ref * g.cpu().double()).sum().backward()
+    tol = 1e-4   # float32 projections and scan against float64 (library GEMMs included)
+    assert_close(out, ref.detach().numpy(), tol, "out")
+    assert_close(x.grad, x64.grad.numpy(), tol, "dx")
+    for n in W:
+        assert_close(getattr(layer, n).weight.grad, W[n].grad.numpy(), tol, f"d{n}")
+
+
+def test_layer_decode_matches_full_sequence(cuda_device):
+    torch.manual_seed(6)
+    B, T, C, H, extra = 3, 100, 128, 4, 6
+    layer = ESA(C, H, mode="controlled", scan_dtype=torch.float16, device=cuda_device)
+    x = torch.randn(B, T + extra, C, device=cuda_device)
+    with torch.no_grad():
+        full = layer(x)
+        out, state = layer(x[:, :T], return_state=True)
+        steps = [layer.step(x[:, T + i], state) for i in range(extra)]
+    tol = TOL[torch.float16]
+    assert_close(out, host64(full[:, :T]), tol, "prefill")
+    assert_close(torch.stack(steps, dim=1), host64(full[:, T:]), tol, "decode")
+    assert np.isfinite(host64(state)).all()
