@@ -725,7 +725,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     esa_scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dy,
                         const BwdArgs args) {
-  static_assert(SUB == 1 || SUB == 2, "a backward tile spans one or two slots");
+  static_assert(SUB == 1 || SUB == 2 || SUB == 4, "a backward tile spans one, two or four slots");
   using Cfg = TileCfg<T, LPH, VPR, L, K, SW>;
   using Sm = BwdSmem<Cfg>;
   using Mp = MiscPlan<Cfg>;
