@@ -858,15 +858,14 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
 
     // ---- F2: replay states, readout backward, dq, ghat ---------------------
     // ghat of each row overwrites that row's q/dy slots (only this thread
-    // reads them again).
-    float2 Ec[4];   // the run's forward carry-in, kept for the da sweep
-    run_carry<CT>(scan_s, es_s, pos.run, pos.ch, Ec);
-    mbar_wait_bounded(&bar[2], (phase >> 2) & 1u, &hdr->status);
-    phase ^= 4u;
+    // reads them again).  The factor of da that depends on the forward state,
+    // E_{t-1} - v_t (direct mode: E_{t-1}), stays in registers for B.
+    float2 Em[K][4];
     {
       float2 E[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) E[q] = Ec[q];
+      run_carry<CT>(scan_s, es_s, pos.run, pos.ch, E);
+      mbar_wait_bounded(&bar[2], (phase >> 2) & 1u, &hdr->status);
+      phase ^= 4u;
 #pragma unroll
       for (int i = 0; i < K; ++i) {
         const int r = pos.row0 + i;
@@ -878,6 +877,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
         float2 ss = splat(0.0f);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
+          Em[i][q] = (MODE == 0) ? E[q] : sub2(E[q], vv[q]);
           E[q] = rec_step<MODE>(Ar[i][q], E[q], vv[q]);
           ss = fma2(E[q], E[q], ss);
         }
@@ -973,8 +973,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     // in the forward): B1 and B2 hide its round trip.
     if (tid == 0) next = atomicAdd(&hdr->ticket[1], 1u);
 
-    // ---- B1: total gradient G_t (latest step first): dv, and the da factor -
-    // G A (1 - A) replaces ghat in the row's slots.
+    // ---- B: total gradient G_t (latest step first): dv and
+    //      da = G A (1 - A) (E_{t-1} - v_t)  (direct mode: times E_{t-1}).
     const bool ch_ok = (c0 + pos.ch) < sh.C;
     const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
     {
@@ -984,7 +984,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
       for (int i = K - 1; i >= 0; --i) {
         const int r = pos.row0 + i;
         if ((t0 + r) < sh.T) {
-          float2 gh[4], dvv[4];
+          float2 gh[4], dvv[4], dav[4];
           get_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -992,33 +992,14 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
             const float2 A = gate_A<MODE>(Ar[i][q]);
             const float2 Ac = (MODE == 0) ? sub2(splat(1.0f), A) : Ar[i][q];
             dvv[q] = (MODE == 0) ? G : mul2(G, Ac);
-            gh[q] = mul2(G, mul2(A, Ac));
+            dav[q] = mul2(mul2(G, mul2(A, Ac)), Em[i][q]);
             h[q] = mul2(A, G);
           }
-          put_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
-          if (ch_ok) Io<T>::store8(dvg + gbase + static_cast<long>(r) * sh.C, dvv);
+          if (ch_ok) {
+            Io<T>::store8(dvg + gbase + static_cast<long>(r) * sh.C, dvv);
+            Io<T>::store8(dag + gbase + static_cast<long>(r) * sh.C, dav);
+          }
         }
-      }
-    }
-
-    // ---- B2: replay states forward: da = G A (1 - A) (E_{t-1} - v_t) --------
-    //      (direct mode: times E_{t-1})
-    {
-      float2 E[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) E[q] = Ec[q];
-#pragma unroll
-      for (int i = 0; i < K; ++i) {
-        const int r = pos.row0 + i;
-        float2 vv[4], ga[4], dav[4];
-        Io<T>::load8(v_s + r * CT + pos.ch, vv);
-        get_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, ga);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          dav[q] = mul2(ga[q], (MODE == 0) ? E[q] : sub2(E[q], vv[q]));
-          E[q] = rec_step<MODE>(Ar[i][q], E[q], vv[q]);
-        }
-        if ((t0 + r) < sh.T && ch_ok) Io<T>::store8(dag + gbase + static_cast<long>(r) * sh.C, dav);
       }
     }
 
