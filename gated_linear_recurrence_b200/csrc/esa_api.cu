@@ -265,6 +265,87 @@ int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy, co
   return esa::launch_bwd(dtype, mode, D, ta, tv, tq, tdy, args, args.s.ntiles, st);
 }
 
+int esa_scan_map(const void *a, const void *v, float *P, float *S, int B, int T, int H, int D, int mode,
+                 int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+  int rc = check_shape(B, T, H, D, mode, dtype);
+  if (rc) return rc;
+  if (B > 0 && (!P || !S)) return ESA_ERR_ARG;
+  if (B > 0 && T > 0 && (!a || !v)) return ESA_ERR_ARG;
+  for (const void *p : {a, v, static_cast<const void *>(P), static_cast<const void *>(S),
+                        static_cast<const void *>(workspace)})
+    if (p && !aligned16(p)) return ESA_ERR_ALIGN;
+  Layout lo;
+  if (!make_layout(B, T, H, D, dtype, &lo)) return ESA_ERR_ARG;
+  if (!workspace || workspace_bytes < lo.total) return ESA_ERR_WORKSPACE;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (B == 0) return ESA_OK;
+  const int C = H * D;
+  const int sub = fwd_slots_per_tile(dtype, D);
+  esa::FwdArgs args;
+  args.s = scan_shape(B, T, H, D, lo, sub);
+  args.y = nullptr;
+  args.E_final = nullptr;
+  args.E_init = nullptr;
+  args.ws = workspace_view(workspace, lo);
+  if (T > 0) {   // T = 0: no tiles, the fold writes the identity map
+    CUtensorMap ta, tv;
+    if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo, lo.L * sub))) return rc;
+    if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo, lo.L * sub))) return rc;
+    if ((rc = esa::launch_fwd_map(dtype, mode, D, ta, tv, ta, args, args.s.ntiles, st))) return rc;
+  }
+  return esa::launch_map_fold(lo.CT, args.ws, args.s, sub, 0, P, S, st);
+}
+
+int esa_scan_bwd_map(const void *a, const void *v, const void *q, const void *dy, float *P, float *S, int B,
+                     int T, int H, int D, int mode, const float *E_init, int dtype, void *workspace,
+                     size_t workspace_bytes, void *stream) {
+  int rc = check_shape(B, T, H, D, mode, dtype);
+  if (rc) return rc;
+  if (B > 0 && (!P || !S)) return ESA_ERR_ARG;
+  if (B > 0 && T > 0 && (!a || !v || !q || !dy)) return ESA_ERR_ARG;
+  for (const void *p : {a, v, q, dy, static_cast<const void *>(P), static_cast<const void *>(S),
+                        static_cast<const void *>(E_init), static_cast<const void *>(workspace)})
+    if (p && !aligned16(p)) return ESA_ERR_ALIGN;
+  Layout lo;
+  if (!make_layout(B, T, H, D, dtype, &lo)) return ESA_ERR_ARG;
+  if (!workspace || workspace_bytes < lo.total) return ESA_ERR_WORKSPACE;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (B == 0) return ESA_OK;
+  const int C = H * D;
+  const int sub = esa::bwd_slots_per_tile(dtype, D);
+  esa::BwdArgs args;
+  args.s = scan_shape(B, T, H, D, lo, sub);
+  args.da = args.dv = args.dq = nullptr;
+  args.dE_final = nullptr;
+  args.dE_init = nullptr;
+  args.E_init = E_init;
+  args.ws = workspace_view(workspace, lo);
+  if (T > 0) {
+    CUtensorMap ta, tv, tq, tdy;
+    if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo, lo.L * sub))) return rc;
+    if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo, lo.L * sub))) return rc;
+    if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo, lo.L * sub))) return rc;
+    if ((rc = make_tmap(&tdy, dy, dtype, B, T, C, lo, lo.L * sub))) return rc;
+    if ((rc = esa::launch_bwd_map(dtype, mode, D, ta, tv, tq, tdy, args, args.s.ntiles, st))) return rc;
+  }
+  return esa::launch_map_fold(lo.CT, args.ws, args.s, sub, 1, P, S, st);
+}
+
+int esa_compose(const float *P, const float *S, int n, long long count, int reverse, const float *x0, float *x,
+                void *stream) {
+  if (n < 0 || count < 0 || (reverse != 0 && reverse != 1)) return ESA_ERR_ARG;
+  if (count > 0 && (!x || (n > 0 && (!P || !S)))) return ESA_ERR_ARG;
+  if (static_cast<long long>(n) * count > LLONG_MAX / 8) return ESA_ERR_ARG;
+  for (const void *p : {static_cast<const void *>(P), static_cast<const void *>(S), static_cast<const void *>(x0),
+                        static_cast<const void *>(x)})
+    if (p && !aligned16(p)) return ESA_ERR_ALIGN;
+  int rc = check_device();
+  if (rc) return rc;
+  return esa::launch_compose(P, S, n, static_cast<long>(count), reverse, x0, x, static_cast<cudaStream_t>(stream));
+}
+
 int esa_step(const void *a_t, const void *v_t, const void *q_t, float *E, void *y_t, int B, int H, int D,
              int mode, int dtype, void *stream) {
   int rc = check_shape(B, 1, H, D, mode, dtype);

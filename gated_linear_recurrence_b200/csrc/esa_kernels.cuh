@@ -468,7 +468,7 @@ __device__ __forceinline__ float2 gate_A(float2 c) { return MODE == 0 ? c : sub2
 // and stores the chunk-end state of every slot it covers (the backward's
 // checkpoints), so taller forward tiles leave the workspace layout alone.
 // ===========================================================================
-template <typename T, int MODE, int LPH, int VPR, int L, int K, int SUB, int SW>
+template <typename T, int MODE, int LPH, int VPR, int L, int K, int SUB, int SW, bool MAP>
 __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR * (L / K) <= 128) ? 4 : (VPR * (L / K) <= 256) ? 2 : 1)
     esa_scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_q, const FwdArgs args) {
@@ -503,10 +503,10 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     const TileInfo ti = decode_tile<false, SUB>(tile, sh, CT, L);
     info_s[stage] = ti;
     if (tile >= sh.ntiles) return;
-    mbar_expect_tx(&bar[stage], 3 * Cfg::kBoxBytes);
+    mbar_expect_tx(&bar[stage], (MAP ? 2 : 3) * Cfg::kBoxBytes);
     tma_load_3d(box(stage, 0), &tm_a, ti.c0, ti.t0, ti.b, &bar[stage]);
     tma_load_3d(box(stage, 1), &tm_v, ti.c0, ti.t0, ti.b, &bar[stage]);
-    tma_load_3d(box(stage, 2), &tm_q, ti.c0, ti.t0, ti.b, &bar[stage]);
+    if constexpr (!MAP) tma_load_3d(box(stage, 2), &tm_q, ti.c0, ti.t0, ti.b, &bar[stage]);
   };
 
   if (tid == 0) {
@@ -550,7 +550,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     // look-back needs no further round trip.
     const bool lb_thread = tid >= Cfg::LB0 && tid < Cfg::LB0 + CT;
     unsigned long long early = 0ull;
-    if (lb_thread && chunk > 0) early = ld_relaxed_b64(&ws.incl_f[(slot_end - SUB) * CT + (tid - Cfg::LB0)]);
+    if (!MAP && lb_thread && chunk > 0) early = ld_relaxed_b64(&ws.incl_f[(slot_end - SUB) * CT + (tid - Cfg::LB0)]);
 
     // The carry entering the chunk, one channel per look-back thread.
     auto resolve_carry = [&]() {
@@ -608,19 +608,20 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
       // The pair's chunk map, for successors' look-backs.  The first tile of a
       // chain needs none (its carry is E_init) and the last has no successor;
       // a ragged last tile's slot_end may also lie past the chain's slots.
-      if (chunk > 0 && chunk < sh.nchunks - 1 && publisher) {
-        const long at = slot_end * CT + 2 * c2;
+      // (MAP: every tile's map, at its first slot, for the segment fold.)
+      if (MAP ? publisher : (chunk > 0 && chunk < sh.nchunks - 1 && publisher)) {
+        const long at = (MAP ? slot : slot_end) * CT + 2 * c2;
         st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tP.x, tag), pack_tag(tS.x, tag)));
         st_relaxed_v2b64(&ws.agg[at + 1], make_ulonglong2(pack_tag(tP.y, tag), pack_tag(tS.y, tag)));
       }
-      scan_runs_fold<CT, RUNS, SW, false>(scan_s, c2, g, eP, eS);
+      if constexpr (!MAP) scan_runs_fold<CT, RUNS, SW, false>(scan_s, c2, g, eP, eS);
       if constexpr (SUB == 2 && SW == 1) {   // the middle run's prefix: this lane wrote the entry itself
         const float2 *pm = reinterpret_cast<const float2 *>(scan_s + scan_pos<CT>(RUNS / 2, 2 * c2));
         eP = pm[0];
         eS = pm[1];
       }
     }
-    if (lb_thread) resolve_carry();   // concurrently with the run scan
+    if (!MAP && lb_thread) resolve_carry();   // concurrently with the run scan
     __syncthreads();
     // The ticket of the tile after next is taken only now: tickets then follow
     // the order in which CTAs really reach their tiles more closely, so a
@@ -629,7 +630,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     // States of the pair at the slot boundaries inside the tile (the
     // backward's checkpoints): boundary j of the SUB - 1 is the start of
     // segment j SW / SUB, whose lanes hold the prefix up to it.
-    if constexpr (SUB > 1) {
+    if constexpr (SUB > 1 && !MAP) {
       if (tid < Cfg::NSCAN) {
         int j = 0;
         if constexpr (SW == 1) j = 1;   // SUB == 2: the middle run's prefix
@@ -642,7 +643,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
         }
       }
     }
-    if (publisher) {   // chunk-end state of the pair
+    if (!MAP && publisher) {   // chunk-end state of the pair
       const float2 E_in = reinterpret_cast<const float2 *>(es_s)[c2];
       const float2 E_end = fma2(tP, E_in, tS);
       if (chunk * SUB + SUB - 1 < sh.nslots)   // a ragged last tile may cover fewer slots
@@ -654,7 +655,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     }
 
     // ---- pass 2: exact states and the readout ------------------------------
-    {
+    if constexpr (!MAP) {
       float2 E[4];
       run_carry<CT>(scan_s, es_s, pos.run, pos.ch, E);
       const bool ch_ok = (c0 + pos.ch) < sh.C;
@@ -720,7 +721,7 @@ __device__ __forceinline__ void get_ghat(const T *q_slot, const T *dy_slot, floa
 // ===========================================================================
 // Backward scan (persistent).
 // ===========================================================================
-template <typename T, int MODE, int LPH, int VPR, int L, int K, int SW, int SUB>
+template <typename T, int MODE, int LPH, int VPR, int L, int K, int SW, int SUB, bool MAP>
 __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR * (L / K) <= 128) ? 4 : (VPR * (L / K) <= 256) ? 2 : 1)
     esa_scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dy,
@@ -896,7 +897,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
 #pragma unroll
         for (int q = 0; q < 4; ++q) gh[q] = mul2(splat(rr), fma2(nn[q], splat(-dot), dn[q]));
         put_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
-        if (valid && (c0 + pos.ch) < sh.C)
+        if (!MAP && valid && (c0 + pos.ch) < sh.C)
           Io<T>::store8(dqg + (static_cast<long>(b) * sh.T + t0 + r) * sh.C + c0 + pos.ch, dqv);
       }
     }
@@ -906,7 +907,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     // of the look-back (see the forward).
     const bool lb_thread = tid >= Cfg::LB0 && tid < Cfg::LB0 + CT;
     unsigned long long early = 0ull;
-    if (lb_thread && chunk < sh.nchunks - 1)
+    if (!MAP && lb_thread && chunk < sh.nchunks - 1)
       early = ld_relaxed_b64(&ws.incl_b[(slot + SUB) * CT + (tid - Cfg::LB0)]);
 
     // ---- R1: the run's reverse map h -> P h + hl ----------------------------
@@ -936,14 +937,14 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
       if (tid < Cfg::NSCAN) {
         float2 eP, eS;
         scan_runs<CT, RUNS, SW, true>(scan_s, seg_s, c2, g, eP, eS, tP, tS);
-        if (chunk < sh.nchunks - 1 && publisher) {   // the pair's reverse chunk map
+        if ((MAP || chunk < sh.nchunks - 1) && publisher) {   // the pair's reverse chunk map
           const long at = slot * CT + 2 * c2;
           st_relaxed_v2b64(&ws.agg[at], make_ulonglong2(pack_tag(tP.x, tag), pack_tag(tS.x, tag)));
           st_relaxed_v2b64(&ws.agg[at + 1], make_ulonglong2(pack_tag(tP.y, tag), pack_tag(tS.y, tag)));
         }
-        scan_runs_fold<CT, RUNS, SW, true>(scan_s, c2, g, eP, eS);
+        if constexpr (!MAP) scan_runs_fold<CT, RUNS, SW, true>(scan_s, c2, g, eP, eS);
       }
-      if (lb_thread) {
+      if (!MAP && lb_thread) {
         const int c = tid - Cfg::LB0;
         const int cg = c0 + c;
         float H_in;
@@ -957,8 +958,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
         }
         es_s[c] = H_in;
       }
-      __syncthreads();
-      if (publisher) {
+      if constexpr (!MAP) __syncthreads();
+      if (!MAP && publisher) {
         const float2 H_out = fma2(tP, reinterpret_cast<const float2 *>(es_s)[c2], tS);
         const long at = slot * CT + 2 * c2;
         st_relaxed_v2b64(reinterpret_cast<ulonglong2 *>(&ws.incl_b[at]),
@@ -977,7 +978,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     //      da = G A (1 - A) (E_{t-1} - v_t)  (direct mode: times E_{t-1}).
     const bool ch_ok = (c0 + pos.ch) < sh.C;
     const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
-    {
+    if constexpr (!MAP) {
       float2 h[4];
       run_carry<CT>(scan_s, es_s, pos.run, pos.ch, h);
 #pragma unroll

@@ -38,6 +38,21 @@ int launch_fwd(int dtype, int mode, int D, const CUtensorMap &ta, const CUtensor
 int launch_bwd(int dtype, int mode, int D, const CUtensorMap &ta, const CUtensorMap &tv,
                const CUtensorMap &tq, const CUtensorMap &tdy, const BwdArgs &args, int ntiles,
                cudaStream_t stream);
+// Map-mode scans: the same tiles, leaving each tile's (reverse) map in the
+// workspace's agg words at the tile's first slot and writing no output.
+int launch_fwd_map(int dtype, int mode, int D, const CUtensorMap &ta, const CUtensorMap &tv,
+                   const CUtensorMap &tq, const FwdArgs &args, int ntiles, cudaStream_t stream);
+int launch_bwd_map(int dtype, int mode, int D, const CUtensorMap &ta, const CUtensorMap &tv,
+                   const CUtensorMap &tq, const CUtensorMap &tdy, const BwdArgs &args, int ntiles,
+                   cudaStream_t stream);
+// Fold the tile maps a map-mode scan just left (tiles of `sub` slots, CT
+// channels) into one map per channel: P, S [B][C] float32.  reverse = 1
+// composes the latest tile first (the backward's maps).
+int launch_map_fold(int CT, const Workspace &ws, const ScanShape &sh, int sub, int reverse, float *P, float *S,
+                    cudaStream_t stream);
+// x = map_{n-1}(... map_0(x0)), map_j(x) = P[j] x + S[j] over `count` floats.
+int launch_compose(const float *P, const float *S, int n, long count, int reverse, const float *x0, float *x,
+                   cudaStream_t stream);
 // Write the header of a freshly zeroed workspace (magic, epoch 1).
 int launch_ws_init(WsHeader *hdr, cudaStream_t stream);
 int launch_step(int dtype, int mode, int D, const void *a, const void *v, const void *q, float *E,

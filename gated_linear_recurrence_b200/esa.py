@@ -10,6 +10,9 @@ The functions carry the C names:
 * :func:`esa_scan_fwd`  -- forward scan (+ E_final, + checkpoints in the workspace)
 * :func:`esa_scan_bwd`  -- backward scan (da, dv, dq, dE_init)
 * :func:`esa_step`      -- one-token decode update (in place on E)
+* :func:`esa_scan_map`, :func:`esa_scan_bwd_map` -- forward / backward segment
+  maps ``(P, S)`` of a time slice (context parallelism)
+* :func:`esa_compose`   -- apply a sequence of segment maps to a state
 * :func:`esa_check`     -- synchronise and read the device status of a workspace
 * :func:`esa_workspace_init` -- zero a new workspace and write its header
 * :func:`esa_workspace_size`, :func:`esa_strerror`, :func:`esa_version`
@@ -68,6 +71,12 @@ def load_library():
         lib.esa_scan_fwd.restype = I
         lib.esa_scan_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, P, I, P, S, P]
         lib.esa_scan_bwd.restype = I
+        lib.esa_scan_map.argtypes = [P, P, P, P, I, I, I, I, I, I, P, S, P]
+        lib.esa_scan_map.restype = I
+        lib.esa_scan_bwd_map.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, I, P, S, P]
+        lib.esa_scan_bwd_map.restype = I
+        lib.esa_compose.argtypes = [P, P, I, ctypes.c_longlong, I, P, P, P]
+        lib.esa_compose.restype = I
         lib.esa_step.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
         lib.esa_step.restype = I
         lib.esa_check.argtypes = [P, P]
@@ -216,6 +225,87 @@ def esa_scan_bwd(a, v, q, dy, workspace, mode=CONTROLLED, E_init=None, dE_final=
     if rc != 0:
         raise EsaError("esa_scan_bwd", rc)
     return da, dv, dq, dE_init
+
+
+def esa_scan_map(a, v, mode=CONTROLLED, workspace=None, P=None, S=None, stream=None):
+    """Forward segment map of a time slice: ``E_T = P * E_0 + S`` per channel.
+
+    Returns ``(P, S, workspace)`` (float32 ``[B, H, D]``).  Only the
+    workspace's chunk-map words are written.
+    """
+    B, T, H, D = _dims(a)
+    _check_seq("v", v, a)
+    P = torch.empty((B, H, D), dtype=torch.float32, device=a.device) if P is None else P
+    S = torch.empty((B, H, D), dtype=torch.float32, device=a.device) if S is None else S
+    _check_state("P", P, B, H, D, a.device)
+    _check_state("S", S, B, H, D, a.device)
+    if workspace is None:
+        workspace = new_workspace(B, T, H, D, a.dtype, a.device)
+    lib = load_library()
+    with torch.cuda.device(a.device):
+        rc = lib.esa_scan_map(_ptr(a), _ptr(v), _ptr(P), _ptr(S), B, T, H, D, int(mode), _DTYPE_CODE[a.dtype],
+                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(a.device, stream))
+    if rc != 0:
+        raise EsaError("esa_scan_map", rc)
+    return P, S, workspace
+
+
+def esa_scan_bwd_map(a, v, q, dy, workspace, mode=CONTROLLED, E_init=None, P=None, S=None, stream=None):
+    """Backward segment map of a time slice: ``dE_init = P * dE_final + S``.
+
+    ``workspace`` must hold the chunk states of the matching forward (same
+    inputs and ``E_init``); they are kept.  Returns ``(P, S)``.
+    """
+    B, T, H, D = _dims(a)
+    for name, t in (("v", v), ("q", q), ("dy", dy)):
+        _check_seq(name, t, a)
+    P = torch.empty((B, H, D), dtype=torch.float32, device=a.device) if P is None else P
+    S = torch.empty((B, H, D), dtype=torch.float32, device=a.device) if S is None else S
+    _check_state("P", P, B, H, D, a.device)
+    _check_state("S", S, B, H, D, a.device)
+    _check_state("E_init", E_init, B, H, D, a.device)
+    if workspace is None or not workspace.is_cuda:
+        raise ValueError("esa_scan_bwd_map needs the CUDA workspace written by the matching esa_scan_fwd")
+    lib = load_library()
+    with torch.cuda.device(a.device):
+        rc = lib.esa_scan_bwd_map(_ptr(a), _ptr(v), _ptr(q), _ptr(dy), _ptr(P), _ptr(S), B, T, H, D, int(mode),
+                                  _ptr(E_init), _DTYPE_CODE[a.dtype], _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(a.device, stream))
+    if rc != 0:
+        raise EsaError("esa_scan_bwd_map", rc)
+    return P, S
+
+
+def esa_compose(P, S, x0=None, reverse=False, out=None, stream=None):
+    """Apply the maps ``x -> P[j] * x + S[j]`` for j in order (``reverse``:
+    from the last index down) to ``x0`` (zeros when None).
+
+    ``P``, ``S``: float32 CUDA tensors ``[n, *shape]``; ``x0`` and the result
+    have ``shape``.
+    """
+    if not isinstance(P, torch.Tensor) or not P.is_cuda or P.dtype != torch.float32 or P.dim() < 1:
+        raise TypeError("P must be a float32 CUDA tensor [n, ...]")
+    if S.shape != P.shape or S.dtype != P.dtype or S.device != P.device:
+        raise ValueError("S must match P")
+    if not (P.is_contiguous() and S.is_contiguous()):
+        raise ValueError("P and S must be contiguous")
+    n, shape = int(P.shape[0]), tuple(P.shape[1:])
+    count = 1
+    for d in shape:
+        count *= int(d)
+    for name, t in (("x0", x0), ("out", out)):
+        if t is not None and (tuple(t.shape) != shape or t.dtype != torch.float32 or t.device != P.device
+                              or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous float32 tensor of shape {shape} on {P.device}")
+    out = torch.empty(shape, dtype=torch.float32, device=P.device) if out is None else out
+    lib = load_library()
+    with torch.cuda.device(P.device):
+        rc = lib.esa_compose(_ptr(P), _ptr(S), n, count, int(bool(reverse)), _ptr(x0), _ptr(out),
+                             _stream(P.device, stream))
+    if rc != 0:
+        raise EsaError("esa_compose", rc)
+    return out
 
 
 def esa_step(a_t, v_t, q_t, E, y_t=None, mode=CONTROLLED, stream=None):

@@ -72,6 +72,10 @@ class ESA(torch.nn.Module):
         scan_dtype: dtype the scan reads and writes (float16, bfloat16 or
             float32); the state is float32 either way.  ``None`` keeps the
             dtype of the projections' output.
+        cp_group: a ``torch.distributed`` process group over which each
+            sequence is split along time (context parallelism: rank r of the
+            group passes the r-th time slice of the sequence); ``None`` runs
+            the whole sequence on this device.
 
     ``forward(x, state=None, return_state=False)`` runs the whole sequence;
     ``state`` (float32 ``[B, H, D]``) is the state before the first token and
@@ -81,7 +85,7 @@ class ESA(torch.nn.Module):
     """
 
     def __init__(self, embd: int, head: int, mode: str = "controlled", bias: bool = False,
-                 scan_dtype: torch.dtype | None = None, device=None, dtype=None):
+                 scan_dtype: torch.dtype | None = None, device=None, dtype=None, cp_group=None):
         super().__init__()
         if embd % head != 0:
             raise ValueError("embd must be a multiple of head")
@@ -92,6 +96,7 @@ class ESA(torch.nn.Module):
         self.embd, self.head, self.mode = embd, head, mode
         self.head_dim = embd // head
         self.scan_dtype = scan_dtype
+        self.cp_group = cp_group
         kw = {"device": device, "dtype": dtype}
         self.W_A = torch.nn.Linear(embd, embd, bias=bias, **kw)
         self.W_V = torch.nn.Linear(embd, embd, bias=bias, **kw)
@@ -111,7 +116,11 @@ class ESA(torch.nn.Module):
         if C != self.embd:
             raise ValueError(f"expected last dimension {self.embd}, got {C}")
         a, v, q = self._proj(x, (B, T, self.head, self.head_dim))
-        y, E = esa_scan(a, v, q, self.mode, E_init=state)
+        if self.cp_group is not None:
+            from .context_parallel import cp_esa_scan
+            y, E = cp_esa_scan(a, v, q, self.mode, E_init=state, group=self.cp_group)
+        else:
+            y, E = esa_scan(a, v, q, self.mode, E_init=state)
         out = self.W_O(y.reshape(B, T, C).to(self.W_O.weight.dtype))
         return (out, E) if return_state else out
 

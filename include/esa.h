@@ -167,6 +167,59 @@ int esa_scan_fwd_noalloc(const void *a, const void *v, const void *q, void *y, f
                          int dtype, void *stream);
 
 /*
+ * Segment maps, for splitting one sequence over several GPUs along time
+ * (context parallelism).  mlbricks-web.pages.dev/esa, opening panel
+ * "Long-context throughput": the state composition is associative, which is
+ * what gives a parallel path over the full sequence; here it is applied
+ * across devices.  Over the T steps of one call, every channel's state is an
+ * affine function of the state entering it, and the backward's carry is an
+ * affine function of the gradient leaving it:
+ *     E_T      = P (.) E_0      + S_fwd,     P = prod_{t=1..T} A_t,
+ *     dE_init  = P (.) dE_final + S_bwd.
+ * A time slice can therefore publish (P, S) -- 2 B C floats -- and find its
+ * own boundary state from the maps of the slices before it (esa_compose),
+ * instead of waiting for them to finish their scans.
+ *
+ * esa_scan_map: the forward map of one slice.
+ *   a, v      [B,T,H,D] gate logits and values (q is not needed).
+ *   P, S      [B,H,D] float32 outputs: P = prod A_t, S = E_T from E_0 = 0.
+ *             With T = 0: P = 1, S = 0.
+ *   workspace as for esa_scan_fwd.  Only its chunk-map words are written:
+ *             chunk states that an earlier esa_scan_fwd left there for its
+ *             backward are kept.  Two launches (tile maps, then their fold);
+ *             no output of size T.
+ */
+int esa_scan_map(const void *a, const void *v, float *P, float *S, int B, int T, int H, int D, int mode,
+                 int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * esa_scan_bwd_map: the backward (reverse) map of one slice.
+ *   a, v, q, dy, E_init  as for esa_scan_bwd (E_init: the slice's true
+ *             initial state, NULL = zeros).
+ *   P, S      [B,H,D] float32 outputs: dE_init = P (.) dE_final + S for any
+ *             dE_final; P = prod A_t, S = dE_init for dE_final = 0.
+ *   workspace the buffer of the matching esa_scan_fwd (same inputs, same
+ *             E_init), unchanged since: its chunk states are read and kept,
+ *             so esa_scan_bwd can follow on the same workspace.
+ */
+int esa_scan_bwd_map(const void *a, const void *v, const void *q, const void *dy, float *P, float *S, int B,
+                     int T, int H, int D, int mode, const float *E_init, int dtype, void *workspace,
+                     size_t workspace_bytes, void *stream);
+
+/*
+ * esa_compose: apply n segment maps in sequence to `count` values,
+ *     x = map_{n-1}( ... map_0(x0) ),   map_j(x) = P_j (.) x + S_j,
+ * with maps in index order (reverse = 0, forward: earliest slice first) or
+ * from index n - 1 down to 0 (reverse = 1, backward: latest slice first).
+ *   P, S      [n, count] float32 (may be NULL when n = 0).
+ *   x0        [count] float32 start value (NULL = zeros).
+ *   x         [count] float32 output; may alias x0.
+ * Each value is folded with float32 fused multiply-adds in map order.
+ */
+int esa_compose(const float *P, const float *S, int n, long long count, int reverse, const float *x0, float *x,
+                void *stream);
+
+/*
  * One-token recurrent update (decode): E <- A (.) E + B in place, then
  * y_t = q_t (.) E / rms(E).
  *   a_t, v_t, q_t [B,H,D] inputs of one token; y_t [B,H,D] output (I/O dtype).

@@ -11,7 +11,14 @@ three GPU entry points:
 
 * :func:`scan_fwd` -- the forward scan with the per-head RMS readout,
 * :func:`scan_bwd` -- the backward (reverse) scan,
-* :func:`step`     -- the one-token recurrent update.
+* :func:`step`     -- the one-token recurrent update,
+
+and, for splitting one sequence along time (context parallelism), the maps
+that summarise a time slice and their composition:
+
+* :func:`scan_map`     -- forward map (P, S) of a slice: E_T = P E_0 + S,
+* :func:`scan_bwd_map` -- backward map: dE_init = P dE_final + S,
+* :func:`compose`      -- a sequence of such maps applied to a state.
 
 Sources for each formula are given in the C file's header: the recurrence and
 its two modes ("entangled-state-attention 0.1.0", section "Core idea"), the
@@ -153,3 +160,53 @@ def step(a_t, v_t, q_t, E, mode):
     if rc != 0:
         raise ValueError(f"esa_oracle_step failed with {rc}")
     return y_t, E_new
+
+
+def _gates(a):
+    """A_t = sigmoid(a_t) in double precision."""
+    return 1.0 / (1.0 + np.exp(-_f64(a)))
+
+
+def scan_map(a, v, mode):
+    """Forward map of a time slice ([B, T, H, D] inputs): ``(P, S)``, float64
+    ``[B, H, D]``, such that the slice's final state is ``P * E_0 + S`` for
+    every initial state E_0.
+
+    The recurrence E_t = A_t E_{t-1} + B_t ("entangled-state-attention
+    0.1.0", section "Core idea"; B_t = v_t or (1 - A_t) v_t) is affine in
+    E_{t-1} with B_t independent of E, so by induction E_T = (prod_t A_t) E_0
+    + E_T|_{E_0 = 0}: P is the product of the gates, S the scan from a zero
+    state.  The readout does not enter, so q is zero here.
+    """
+    a = _f64(a)
+    P = np.prod(_gates(a), axis=1)
+    _, S = scan_fwd(a, v, np.zeros_like(a), mode)
+    return P, S
+
+
+def scan_bwd_map(a, v, q, dy, mode, E_init=None):
+    """Backward map of a time slice: ``(P, S)`` with ``dE_init = P * dE_final
+    + S`` for every dE_final.
+
+    The reverse recurrence G_t = ghat_t + A_{t+1} G_{t+1}, G_T = ghat_T +
+    dE_final, dE_init = A_1 G_1, is affine in dE_final, and ghat depends only
+    on the forward states (fixed by E_init), not on dE_final: dE_init =
+    (prod_t A_t) dE_final + dE_init|_{dE_final = 0}.
+    """
+    a = _f64(a)
+    P = np.prod(_gates(a), axis=1)
+    S = scan_bwd(a, v, q, dy, mode, E_init=E_init, dE_final=None)[3]
+    return P, S
+
+
+def compose(P, S, x0=None, reverse=False):
+    """Apply the maps x -> P[j] x + S[j] one after another to ``x0`` (zeros
+    when None): j = 0, 1, ..., n-1, or n-1, ..., 0 with ``reverse``.
+    ``P``, ``S``: ``[n, ...]``."""
+    P = _f64(P)
+    S = _f64(S, P.shape)
+    x = np.zeros(P.shape[1:]) if x0 is None else np.array(_f64(x0, P.shape[1:]), copy=True)
+    order = range(P.shape[0] - 1, -1, -1) if reverse else range(P.shape[0])
+    for j in order:
+        x = P[j] * x + S[j]
+    return x

@@ -145,3 +145,45 @@ def test_binding_rejects_cpu_tensors(lib):
         esa.esa_scan_fwd(x, x, x)
     with pytest.raises(TypeError):
         esa.esa_step(x[:, 0], x[:, 0], x[:, 0], torch.zeros(1, 2, 32))
+
+
+def test_segment_map_argument_errors(lib):
+    from gated_linear_recurrence_b200 import esa
+    P = _fake
+    # esa_scan_map(a, v, P, S, B, T, H, D, mode, dtype, ws, wsb, stream)
+    assert lib.esa_scan_map(P(0x1000), P(0x2000), None, P(0x4000), 2, 8, 2, 32, 1, 1, P(0x10000), 1 << 30,
+                            None) == esa.ESA_ERR_ARG                 # P missing
+    assert lib.esa_scan_map(None, P(0x2000), P(0x3000), P(0x4000), 2, 8, 2, 32, 1, 1, P(0x10000), 1 << 30,
+                            None) == esa.ESA_ERR_ARG                 # a missing
+    assert lib.esa_scan_map(P(0x1000), P(0x2000), P(0x3004), P(0x4000), 2, 8, 2, 32, 1, 1, P(0x10000),
+                            1 << 30, None) == esa.ESA_ERR_ALIGN
+    assert lib.esa_scan_map(P(0x1000), P(0x2000), P(0x3000), P(0x4000), 2, 8, 2, 24, 1, 1, P(0x10000),
+                            1 << 30, None) == esa.ESA_ERR_UNSUPPORTED
+    assert lib.esa_scan_map(P(0x1000), P(0x2000), P(0x3000), P(0x4000), 2, 8, 2, 32, 1, 1, P(0x10000), 64,
+                            None) == esa.ESA_ERR_WORKSPACE
+    # esa_scan_bwd_map(a, v, q, dy, P, S, B, T, H, D, mode, E_init, dtype, ws, wsb, stream)
+    assert lib.esa_scan_bwd_map(P(0x1000), P(0x2000), P(0x3000), None, P(0x5000), P(0x6000), 2, 8, 2, 32, 1,
+                                None, 1, P(0x10000), 1 << 30, None) == esa.ESA_ERR_ARG   # dy missing
+    assert lib.esa_scan_bwd_map(P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000), P(0x6000), 2, 8, 2, 32,
+                                3, None, 1, P(0x10000), 1 << 30, None) == esa.ESA_ERR_ARG   # mode
+    assert lib.esa_scan_bwd_map(P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000), P(0x6000), 2, 8, 2, 32,
+                                1, P(0x7008), 1, P(0x10000), 1 << 30, None) == esa.ESA_ERR_ALIGN
+    # esa_compose(P, S, n, count, reverse, x0, x, stream)
+    assert lib.esa_compose(P(0x1000), P(0x2000), -1, 16, 0, None, P(0x3000), None) == esa.ESA_ERR_ARG
+    assert lib.esa_compose(P(0x1000), P(0x2000), 2, 16, 2, None, P(0x3000), None) == esa.ESA_ERR_ARG
+    assert lib.esa_compose(None, P(0x2000), 2, 16, 0, None, P(0x3000), None) == esa.ESA_ERR_ARG
+    assert lib.esa_compose(P(0x1000), P(0x2000), 2, 16, 0, None, None, None) == esa.ESA_ERR_ARG
+    assert lib.esa_compose(P(0x1000), P(0x2004), 2, 16, 0, None, P(0x3000), None) == esa.ESA_ERR_ALIGN
+
+
+def test_segment_map_calls_need_a_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present; this checks the device-less path")
+    from gated_linear_recurrence_b200 import esa
+    P = _fake
+    assert lib.esa_scan_map(P(0x1000), P(0x2000), P(0x3000), P(0x4000), 2, 8, 2, 32, 1, 1, P(0x10000), 1 << 30,
+                            None) == esa.ESA_ERR_DEVICE
+    assert lib.esa_scan_bwd_map(P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000), P(0x6000), 2, 8, 2, 32,
+                                1, None, 1, P(0x10000), 1 << 30, None) == esa.ESA_ERR_DEVICE
+    assert lib.esa_compose(P(0x1000), P(0x2000), 2, 16, 0, None, P(0x3000), None) == esa.ESA_ERR_DEVICE

@@ -306,6 +306,86 @@ def test_backward_transpose_of_linear_state_map():
 
 
 # ---------------------------------------------------------------------------
+# Segment maps (a sequence split along time).
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", [D_, C_])
+def test_scan_map_is_the_affine_map_of_the_slice(mode):
+    # For every initial state the slice ends at P E_0 + S; two unrelated
+    # initial states (and zero) pin both P and S.
+    a, v, q, _, E0, dEf = rng_inputs(30, 2, 23, 2, 4, a_mean=1.0)
+    P, S = oracle.scan_map(a, v, mode)
+    for x in (E0, dEf, np.zeros_like(E0)):
+        _, Ef = oracle.scan_fwd(a, v, q, mode, E_init=x)
+        np.testing.assert_allclose(Ef, P * x + S, rtol=1e-12, atol=1e-13)
+
+
+def test_scan_map_brute_force_product():
+    # P is the product of the gates: 50-digit decimal evaluation, one channel.
+    a, v, _, _, _, _ = rng_inputs(31, 1, 9, 1, 2)
+    P, _ = oracle.scan_map(a, v, C_)
+    ctx = decimal.Context(prec=50)
+    for d in range(2):
+        prod = decimal.Decimal(1)
+        for t in range(9):
+            x = decimal.Decimal(float(a[0, t, 0, d]))
+            prod = ctx.multiply(prod, ctx.divide(1, ctx.add(1, ctx.exp(-x))))
+        assert abs(float(prod) - P[0, 0, d]) <= 1e-14 * abs(float(prod))
+
+
+@pytest.mark.parametrize("mode", [D_, C_])
+def test_scan_bwd_map_is_the_affine_map_of_the_slice(mode):
+    a, v, q, dy, E0, dEf = rng_inputs(32, 2, 19, 2, 4)
+    P, S = oracle.scan_bwd_map(a, v, q, dy, mode, E_init=E0)
+    for g in (dEf, 3.0 * E0, np.zeros_like(dEf)):
+        dE0 = oracle.scan_bwd(a, v, q, dy, mode, E_init=E0, dE_final=g)[3]
+        np.testing.assert_allclose(dE0, P * g + S, rtol=1e-11, atol=1e-12)
+
+
+def test_compose_order_small_example():
+    # maps x -> 2x + 1 then x -> 3x + 1 from x = 1: 3 then 10; reversed: 4 then 9.
+    P = np.array([[2.0], [3.0]])
+    S = np.array([[1.0], [1.0]])
+    assert oracle.compose(P, S, np.array([1.0]))[0] == 10.0
+    assert oracle.compose(P, S, np.array([1.0]), reverse=True)[0] == 9.0
+    assert oracle.compose(P, S)[0] == 4.0
+    assert oracle.compose(P[:0], S[:0], np.array([5.0]))[0] == 5.0
+
+
+@pytest.mark.parametrize("mode", [D_, C_])
+def test_slices_composed_equal_the_whole_sequence(mode):
+    # Three slices of unequal length: the forward maps of the earlier slices
+    # give each slice its initial state, the reverse maps of the later slices
+    # give each its final-state gradient, and the per-slice scans then equal
+    # the scan of the whole sequence.
+    a, v, q, dy, E0, dEf = rng_inputs(33, 2, 40, 2, 4, a_mean=0.5)
+    cuts = [0, 11, 12, 40]
+    sl = [slice(cuts[i], cuts[i + 1]) for i in range(3)]
+    y, Ef = oracle.scan_fwd(a, v, q, mode, E_init=E0)
+    da, dv, dq, dE0 = oracle.scan_bwd(a, v, q, dy, mode, E_init=E0, dE_final=dEf)
+    fmaps = [oracle.scan_map(a[:, s], v[:, s], mode) for s in sl]
+    Pf = np.stack([m[0] for m in fmaps])
+    Sf = np.stack([m[1] for m in fmaps])
+    E_in = [oracle.compose(Pf[:r], Sf[:r], E0) for r in range(3)]
+    np.testing.assert_allclose(oracle.compose(Pf, Sf, E0), Ef, rtol=1e-12, atol=1e-13)
+    bmaps = [oracle.scan_bwd_map(a[:, s], v[:, s], q[:, s], dy[:, s], mode, E_init=E_in[r])
+             for r, s in enumerate(sl)]
+    Pb = np.stack([m[0] for m in bmaps])
+    Sb = np.stack([m[1] for m in bmaps])
+    np.testing.assert_allclose(oracle.compose(Pb, Sb, dEf, reverse=True), dE0, rtol=1e-11, atol=1e-12)
+    parts = {k: [] for k in ("y", "da", "dv", "dq")}
+    for r, s in enumerate(sl):
+        yr, _ = oracle.scan_fwd(a[:, s], v[:, s], q[:, s], mode, E_init=E_in[r])
+        dE_out = oracle.compose(Pb[r + 1:], Sb[r + 1:], dEf, reverse=True)
+        dar, dvr, dqr, _ = oracle.scan_bwd(a[:, s], v[:, s], q[:, s], dy[:, s], mode, E_init=E_in[r],
+                                           dE_final=dE_out)
+        for k, val in zip(("y", "da", "dv", "dq"), (yr, dar, dvr, dqr)):
+            parts[k].append(val)
+    for k, ref in (("y", y), ("da", da), ("dv", dv), ("dq", dq)):
+        np.testing.assert_allclose(np.concatenate(parts[k], axis=1), ref, rtol=1e-10, atol=1e-12, err_msg=k)
+
+
+# ---------------------------------------------------------------------------
 # The only printed worked examples are shapes.
 # ---------------------------------------------------------------------------
 
