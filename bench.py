@@ -55,6 +55,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the prefill + decode (esa_step) measurement reported under detail.decode")
+    ap.add_argument("--no-cp", action="store_true",
+                    help="skip the per-rank context-parallel phase timing reported under detail.context_parallel")
+    ap.add_argument("--cp-only", action="store_true",
+                    help="run only the context-parallel phase timing (one JSON line; for profiling its kernels)")
     ap.add_argument("--batch", type=int, default=None,
                     help="run a smaller batch of the same workload (profiling cases only)")
     ap.add_argument("--seq", type=int, default=None,
@@ -92,13 +96,19 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
 
 
+# The files the two scan kernels are built from: bodies, helpers, tile
+# geometry and instantiation.  A profile summary's traffic applies while they
+# are unchanged.
+SCAN_KERNEL_SOURCES = ("esa_kernels.cuh", "esa_common.cuh", "esa_dispatch.cuh", "esa_launchers.cuh",
+                       "esa_launch.h", "esa_fwd.cu", "esa_bwd.cu")
+
+
 def source_hash():
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "gated_linear_recurrence_b200", "csrc", "*"))):
-        if p.endswith((".cu", ".cuh", ".h")):
-            with open(p, "rb") as f:
-                h.update(os.path.basename(p).encode())
-                h.update(f.read())
+    for name in sorted(SCAN_KERNEL_SOURCES):
+        with open(os.path.join(ROOT, "gated_linear_recurrence_b200", "csrc", name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -396,6 +406,92 @@ def measure_decode(dev, reps=5):
                     "Python binding's launch cost"}
 
 
+def measure_context_parallel(dev, n_slices=8, reps=5):
+    """Per-rank cost of the context-parallel scan, measured on one GPU.
+
+    The workload's sequence (T = 65536) split in ``n_slices`` time slices of
+    T / n_slices steps, as ``n_slices`` ranks would hold it.  Every rank runs
+    the same kernels on a slice of the same size, so one slice on one GPU
+    gives the per-rank device time of each phase: forward map (+ fold), two
+    compositions, forward scan, backward map (+ fold), one composition,
+    backward scan.  The two all-gathers between the phases (2 B C and 3 B C
+    float32 per rank) need several GPUs and are not part of this number.  The
+    plain forward + backward of the same slice is timed beside it.
+    """
+    import torch
+
+    from gated_linear_recurrence_b200 import esa, inputs
+    w = workload()
+    B, H, D, mode = w.B, w.H, w.D, w.mode
+    Tr = w.T // n_slices
+    x = inputs.make_scan_inputs(B, Tr, H, D, w.dtype, w.a_mean, w.seed + 7, device=dev)
+    a, v, q, dy = x["a"], x["v"], x["q"], x["dy"]
+    y, da, dv, dq = (torch.empty_like(a) for _ in range(4))
+    ws = esa.new_workspace(B, Tr, H, D, a.dtype, dev)
+    stream = torch.cuda.current_stream(dev)
+    st = {k: torch.empty(B, H, D, dtype=torch.float32, device=dev) for k in ("P", "S", "Pb", "Sb", "E", "Ef", "G")}
+    rank = n_slices - 1   # the longest compositions
+
+    def phases():
+        yield "fwd_map", lambda: esa.esa_scan_map(a, v, mode=mode, workspace=ws, P=st["P"], S=st["S"])
+        Pn = st["P"].expand(n_slices, B, H, D).contiguous()
+        Sn = st["S"].expand(n_slices, B, H, D).contiguous()
+        yield "fwd_compose", lambda: (esa.esa_compose(Pn[:rank], Sn[:rank], out=st["E"]),
+                                      esa.esa_compose(Pn, Sn, out=st["Ef"]))
+        yield "fwd_scan", lambda: esa.esa_scan_fwd(a, v, q, y=y, mode=mode, E_init=st["E"], workspace=ws,
+                                                   want_E_final=False)
+        yield "bwd_map", lambda: esa.esa_scan_bwd_map(a, v, q, dy, ws, mode=mode, E_init=st["E"], P=st["Pb"],
+                                                      S=st["Sb"])
+        yield "bwd_compose", lambda: esa.esa_compose(Pn[rank + 1:], Sn[rank + 1:], x0=st["Ef"], reverse=True,
+                                                     out=st["G"])
+        yield "bwd_scan", lambda: esa.esa_scan_bwd(a, v, q, dy, ws, mode=mode, E_init=st["E"], dE_final=st["G"],
+                                                   da=da, dv=dv, dq=dq, want_dE_init=False)
+
+    def run_all(times=None):
+        for name, fn in phases():
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            if times is not None:
+                times.setdefault(name, []).append((e0, e1))
+
+    def plain():
+        esa.esa_scan_fwd(a, v, q, y=y, mode=mode, workspace=ws, want_E_final=False)
+        esa.esa_scan_bwd(a, v, q, dy, ws, mode=mode, da=da, dv=dv, dq=dq, want_dE_init=False)
+
+    for _ in range(3):
+        run_all()
+        plain()
+    torch.cuda.synchronize()
+    times = {}
+    for _ in range(reps):
+        run_all(times)
+    torch.cuda.synchronize()
+    ph = {k: statistics.mean(e0.elapsed_time(e1) for e0, e1 in v_) for k, v_ in times.items()}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        plain()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    esa.esa_check(ws)
+    plain_ms = e0.elapsed_time(e1) / reps
+    rank_ms = sum(ph.values())
+    s = a.element_size()
+    C = H * D
+    return {"workload": f"{WORKLOAD_NAME} split in {n_slices} time slices of T={Tr}",
+            "phases_ms": ph, "rank_device_ms": rank_ms, "plain_fwd_bwd_ms": plain_ms,
+            "overhead_vs_plain": rank_ms / plain_ms - 1.0,
+            "allgather_bytes_per_rank": {"forward": 2 * B * C * 4, "backward": 3 * B * C * 4},
+            "map_GBs": {"fwd_map": 2 * s * C * B * Tr / (ph["fwd_map"] / 1e3) / 1e9,
+                        "bwd_map": 4 * s * C * B * Tr / (ph["bwd_map"] / 1e3) / 1e9},
+            "tokens_per_s_per_rank_excl_collectives": B * Tr / (rank_ms / 1e3),
+            "gpu_launches_per_rank_step": 11,
+            "note": "one GPU: per-rank device time of every phase; the all-gathers are not included"}
+
+
 # ---------------------------------------------------------------------------
 # Our arm.
 # ---------------------------------------------------------------------------
@@ -525,6 +621,9 @@ def run_ours(args):
     decode = None
     if not args.no_decode:
         decode = measure_decode(dev)
+    cpar = None
+    if not args.no_cp and args.batch is None and args.seq is None:
+        cpar = measure_context_parallel(dev)
 
     cpu = cpu_all = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -544,7 +643,7 @@ def run_ours(args):
                    "bwd_GBs": bwd_bytes / (bwd_ms / 1e3) / 1e9, "step_GBs": step_gbs,
                    "step_frac_of_measured_peak": step_gbs / peak, "step_frac_of_nominal_8TBs":
                    step_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes_per_step": fwd_bytes + bwd_bytes,
-                   "decode": decode, "cpu_baseline_all_cores": cpu_all},
+                   "decode": decode, "context_parallel": cpar, "cpu_baseline_all_cores": cpu_all},
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": 2 * K,
@@ -563,6 +662,12 @@ def main(argv=None):
         raise SystemExit("--warmup must be at least 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.cp_only:
+        import torch
+        dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+        torch.cuda.set_device(dev)
+        print(json.dumps({"context_parallel": measure_context_parallel(dev)}), flush=True)
+        return 0
     return run_ours(args)
 
 
