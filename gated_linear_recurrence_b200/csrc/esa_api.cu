@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "esa.h"
+#include "esa_fused_launch.h"
 #include "esa_launch.h"
 
 namespace {
@@ -141,6 +142,24 @@ int make_tmap(CUtensorMap *map, const void *ptr, int dtype, int B, int T, int C,
   std::memset(map, 0, sizeof(*map));
   const CUresult r = fn(map, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ESA_OK : ESA_ERR_LAUNCH;
+}
+
+// A 16-bit row-major matrix of `rank` 2 or 3 dimensions (innermost first),
+// read in boxes of 64 elements (128 bytes) x box_rows with the 128-byte
+// swizzle the tensor-core operands use.
+int make_tmap_sw128(CUtensorMap *map, const void *ptr, int dtype, int rank, const cuuint64_t *dims,
+                    cuuint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return ESA_ERR_LAUNCH;
+  const CUtensorMapDataType dt = dtype == ESA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cuuint64_t strides[2] = {dims[0] * 2, rank > 2 ? dims[0] * dims[1] * 2 : 0};
+  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  std::memset(map, 0, sizeof(*map));
+  const CUresult r = fn(map, dt, static_cast<cuuint32_t>(rank), const_cast<void *>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ESA_OK : ESA_ERR_LAUNCH;
 }
@@ -344,6 +363,45 @@ int esa_compose(const float *P, const float *S, int n, long long count, int reve
   int rc = check_device();
   if (rc) return rc;
   return esa::launch_compose(P, S, n, static_cast<long>(count), reverse, x0, x, static_cast<cudaStream_t>(stream));
+}
+
+int esa_fused_fwd(const void *x, const void *W, void *y, float *E_final, int B, int T, int H, int D, int C_in,
+                  int mode, const float *E_init, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+  int rc = check_shape(B, T, H, D, mode, dtype);
+  if (rc) return rc;
+  if (C_in < 1) return ESA_ERR_ARG;
+  Layout lo;
+  if (!make_layout(B, T, H, D, dtype, &lo)) return ESA_ERR_ARG;
+  if (!esa::fused_supported(dtype, D, C_in, lo.nct)) return ESA_ERR_UNSUPPORTED;
+  const bool has_tokens = B > 0 && T > 0;
+  if (has_tokens && (!x || !W || !y)) return ESA_ERR_ARG;
+  for (const void *p : {x, W, static_cast<const void *>(y), static_cast<const void *>(E_final),
+                        static_cast<const void *>(E_init), static_cast<const void *>(workspace)})
+    if (p && !aligned16(p)) return ESA_ERR_ALIGN;
+  if (!workspace || workspace_bytes < lo.total) return ESA_ERR_WORKSPACE;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int C = H * D;
+  if (B == 0) return ESA_OK;
+  if (T == 0) {
+    if (!E_final) return ESA_OK;
+    const size_t bytes = static_cast<size_t>(B) * C * sizeof(float);
+    return E_init ? rt(cudaMemcpyAsync(E_final, E_init, bytes, cudaMemcpyDeviceToDevice, st))
+                  : rt(cudaMemsetAsync(E_final, 0, bytes, st));
+  }
+  CUtensorMap tx, tw;
+  const cuuint64_t xdims[3] = {static_cast<cuuint64_t>(C_in), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
+  const cuuint64_t wdims[2] = {static_cast<cuuint64_t>(C_in), static_cast<cuuint64_t>(3) * C};
+  if ((rc = make_tmap_sw128(&tx, x, dtype, 3, xdims, 128))) return rc;
+  if ((rc = make_tmap_sw128(&tw, W, dtype, 2, wdims, 64))) return rc;
+  esa::FusedArgs args;
+  args.s = scan_shape(B, T, H, D, lo, 2);
+  args.ntiles_ct = B * args.s.nchunks;
+  args.y = y;
+  args.E_final = E_final;
+  args.E_init = E_init;
+  args.ws = workspace_view(workspace, lo);
+  return esa::launch_fused_fwd(dtype, mode, D, C_in, tx, tw, args, st);
 }
 
 int esa_step(const void *a_t, const void *v_t, const void *q_t, float *E, void *y_t, int B, int H, int D,

@@ -41,6 +41,8 @@ constexpr unsigned long long kWorkspaceMagic = 0x45534153434e3031ull;
 // per scan call (the kernel's last CTA does it) and is never 0; init zeroes
 // every word, so no stale word can carry a current tag.
 // ---------------------------------------------------------------------------
+constexpr int kMaxChannelTickets = 48;   // channel tiles of the fused projection + scan
+
 struct WsHeader {
   unsigned long long magic;   // kWorkspaceMagic once initialised
   unsigned epoch;             // tag used by the next scan call
@@ -48,7 +50,9 @@ struct WsHeader {
   unsigned ticket[2];         // tile ticket counters: [0] forward, [1] backward
   unsigned done[2];           // CTAs finished, per kernel
   unsigned abort[2];          // raised by a CTA whose wait gave up
+  unsigned ct_ticket[kMaxChannelTickets];   // fused forward: one ticket counter per channel tile
 };
+static_assert(sizeof(WsHeader) <= 256, "the workspace header is 256 bytes");
 
 struct Workspace {
   WsHeader *hdr;

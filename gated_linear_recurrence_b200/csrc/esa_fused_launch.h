@@ -1,0 +1,23 @@
+// esa_fused_launch.h -- host-side launch interface of the fused projection +
+// scan forward.  Internal to the library.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "esa_fused.cuh"
+
+namespace esa {
+
+// Shapes the fused kernel takes: 16-bit I/O, channel tiles of 64 (head
+// dimension <= 64), C_in of 64 or 128, at most kMaxChannelTickets channel tiles.
+inline bool fused_supported(int dtype, int D, int cin, int nct) {
+  return (dtype == 1 || dtype == 2) && D <= 64 && (cin == 64 || cin == 128) && nct <= kMaxChannelTickets;
+}
+
+// tx: x [B][T][C_in] in boxes of [128 rows][64 elements], 128-byte swizzle;
+// tw: W [3 C][C_in] in boxes of [64 rows][64 elements], 128-byte swizzle.
+int launch_fused_fwd(int dtype, int mode, int D, int cin, const CUtensorMap &tx, const CUtensorMap &tw,
+                     const FusedArgs &args, cudaStream_t stream);
+
+}  // namespace esa

@@ -251,13 +251,13 @@ __device__ __forceinline__ void named_sync(int id, int n) {
 // (RS = RUNS / SW; oldest run first, or latest first for kReverse), replacing
 // each entry by its exclusive prefix within the segment.  The groups then
 // exchange their segment maps through `seg_s` ([SW][CT/2] float4: P pair, S
-// pair) under named barrier 2, and each lane returns the map of the segments
+// pair) under named barrier `bar_id` (default 2), and each lane returns the map of the segments
 // before its own (eP, eS: the prefix at the start of its segment) and the tile
 // map (tP, tS, valid in the last group).  The tile map is known here, before
 // part two, so it can be published at once.
 template <int CT, int RUNS, int SW, bool kReverse>
 __device__ __forceinline__ void scan_runs(float *scan, float4 *seg_s, int c2, int g, float2 &eP, float2 &eS,
-                                          float2 &tP, float2 &tS) {
+                                          float2 &tP, float2 &tS, int bar_id = 2) {
   constexpr int RS = RUNS / SW;
   constexpr int NP = CT / 2;
   float4 *col = reinterpret_cast<float4 *>(scan + scan_pos<CT>(0, 2 * c2));   // (P pair, S pair)
@@ -281,7 +281,7 @@ __device__ __forceinline__ void scan_runs(float *scan, float4 *seg_s, int c2, in
     tS = cs;
   } else {
     seg_s[g * NP + c2] = make_float4(cp.x, cp.y, cs.x, cs.y);
-    named_sync(2, SW * NP);
+    named_sync(bar_id, SW * NP);
 #pragma unroll
     for (int j = 0; j < SW - 1; ++j) {   // earlier segments, oldest applied first
       if (j < g) {

@@ -13,6 +13,7 @@ The functions carry the C names:
 * :func:`esa_scan_map`, :func:`esa_scan_bwd_map` -- forward / backward segment
   maps ``(P, S)`` of a time slice (context parallelism)
 * :func:`esa_compose`   -- apply a sequence of segment maps to a state
+* :func:`esa_fused_fwd` -- forward scan with the a / v / q projections fused in
 * :func:`esa_check`     -- synchronise and read the device status of a workspace
 * :func:`esa_workspace_init` -- zero a new workspace and write its header
 * :func:`esa_workspace_size`, :func:`esa_strerror`, :func:`esa_version`
@@ -77,6 +78,8 @@ def load_library():
         lib.esa_scan_bwd_map.restype = I
         lib.esa_compose.argtypes = [P, P, I, ctypes.c_longlong, I, P, P, P]
         lib.esa_compose.restype = I
+        lib.esa_fused_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, P, I, P, S, P]
+        lib.esa_fused_fwd.restype = I
         lib.esa_step.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
         lib.esa_step.restype = I
         lib.esa_check.argtypes = [P, P]
@@ -306,6 +309,46 @@ def esa_compose(P, S, x0=None, reverse=False, out=None, stream=None):
     if rc != 0:
         raise EsaError("esa_compose", rc)
     return out
+
+
+def esa_fused_fwd(x, W, H, mode=CONTROLLED, E_init=None, y=None, E_final=None, workspace=None, stream=None,
+                  want_E_final=True):
+    """Forward scan of the projections of ``x``: a, v, q = x W[:C]^T,
+    x W[C:2C]^T, x W[2C:]^T (rounded to x's dtype), computed on the tensor
+    cores inside the scan.  ``x``: [B, T, C_in] float16 / bfloat16; ``W``:
+    [3C, C_in] of the same dtype; ``H`` heads of D = C / H channels.
+
+    Returns ``(y, E_final, workspace)`` with ``y`` [B, T, H, D].
+    """
+    if not isinstance(x, torch.Tensor) or not x.is_cuda or x.dim() != 3:
+        raise TypeError("x must be a CUDA tensor [B, T, C_in] (the ESA library has no CPU path)")
+    if not isinstance(W, torch.Tensor) or not W.is_cuda or W.dim() != 2 or W.dtype != x.dtype or W.device != x.device:
+        raise TypeError("W must be a CUDA tensor [3C, C_in] of x's dtype and device")
+    if x.dtype not in _DTYPE_CODE or not x.is_contiguous() or not W.is_contiguous():
+        raise ValueError("x and W must be contiguous float16 / bfloat16 tensors")
+    B, T, C_in = (int(s) for s in x.shape)
+    if W.shape[1] != C_in or W.shape[0] % 3 != 0 or (W.shape[0] // 3) % H != 0:
+        raise ValueError("W must be [3C, C_in] with C divisible by H")
+    C = W.shape[0] // 3
+    D = C // H
+    if y is None:
+        y = torch.empty((B, T, H, D), dtype=x.dtype, device=x.device)
+    if tuple(y.shape) != (B, T, H, D) or y.dtype != x.dtype or not y.is_contiguous():
+        raise ValueError(f"y must be a contiguous {x.dtype} tensor of shape {(B, T, H, D)}")
+    if E_final is None and want_E_final:
+        E_final = torch.empty((B, H, D), dtype=torch.float32, device=x.device)
+    _check_state("E_final", E_final, B, H, D, x.device)
+    _check_state("E_init", E_init, B, H, D, x.device)
+    if workspace is None:
+        workspace = new_workspace(B, T, H, D, x.dtype, x.device)
+    lib = load_library()
+    with torch.cuda.device(x.device):
+        rc = lib.esa_fused_fwd(_ptr(x), _ptr(W), _ptr(y), _ptr(E_final), B, T, H, D, C_in, int(mode), _ptr(E_init),
+                               _DTYPE_CODE[x.dtype], _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(x.device, stream))
+    if rc != 0:
+        raise EsaError("esa_fused_fwd", rc)
+    return y, E_final, workspace
 
 
 def esa_step(a_t, v_t, q_t, E, y_t=None, mode=CONTROLLED, stream=None):

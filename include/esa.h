@@ -220,6 +220,28 @@ int esa_compose(const float *P, const float *S, int n, long long count, int reve
                 void *stream);
 
 /*
+ * Forward scan with the input projections fused in (inference / prefill of
+ * the ESA layer).  "entangled-state-attention 0.1.0", section "Core idea":
+ * the layer's gate logits, values and queries are projections of its input,
+ * a = x W_A^T, v = x W_V^T, q = x W_Q^T; this call computes them on the
+ * tensor cores tile by tile, rounds them to the I/O dtype (the values an
+ * unfused projection writes) and runs the forward scan on them without
+ * writing them to memory.  Results equal esa_scan_fwd on those a, v, q.
+ *   x         [B,T,C_in] layer input, I/O dtype (required).
+ *   W         [3C, C_in] the three projection weights stacked (rows 0..C-1:
+ *             W_A, C..2C-1: W_V, 2C..3C-1: W_Q), each [out, in] as stored by
+ *             a linear layer, I/O dtype (required).
+ *   y, E_final, E_init, mode, workspace: as for esa_scan_fwd; the workspace
+ *             may be shared with esa_scan_fwd (same size), but no backward
+ *             can follow this call (a, v, q are not kept).
+ * Supported: dtype ESA_F16 or ESA_BF16, D <= 64, C_in of 64 or 128, C <= 3072;
+ * other shapes return ESA_ERR_UNSUPPORTED (compute the projections
+ * separately and call esa_scan_fwd).
+ */
+int esa_fused_fwd(const void *x, const void *W, void *y, float *E_final, int B, int T, int H, int D, int C_in,
+                  int mode, const float *E_init, int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * One-token recurrent update (decode): E <- A (.) E + B in place, then
  * y_t = q_t (.) E / rms(E).
  *   a_t, v_t, q_t [B,H,D] inputs of one token; y_t [B,H,D] output (I/O dtype).

@@ -18,7 +18,12 @@ that summarise a time slice and their composition:
 
 * :func:`scan_map`     -- forward map (P, S) of a slice: E_T = P E_0 + S,
 * :func:`scan_bwd_map` -- backward map: dE_init = P dE_final + S,
-* :func:`compose`      -- a sequence of such maps applied to a state.
+* :func:`compose`      -- a sequence of such maps applied to a state,
+
+and the forward of the layer from its input:
+
+* :func:`project`      -- a, v, q as projections of x, rounded to the I/O type,
+* :func:`fused_fwd`    -- those projections followed by :func:`scan_fwd`.
 
 Sources for each formula are given in the C file's header: the recurrence and
 its two modes ("entangled-state-attention 0.1.0", section "Core idea"), the
@@ -210,3 +215,44 @@ def compose(P, S, x0=None, reverse=False):
     for j in order:
         x = P[j] * x + S[j]
     return x
+
+
+def round_io(x, io_dtype):
+    """Round float64 values to the I/O type and widen them back: "f16" (IEEE
+    half, round to nearest even, by numpy), "bf16" (the upper 16 bits of the
+    float32 value, round to nearest even, after rounding to float32 first)
+    or "f32"."""
+    x = np.asarray(x, dtype=np.float64)
+    if io_dtype == "f16":
+        return x.astype(np.float16).astype(np.float64)
+    if io_dtype == "f32":
+        return x.astype(np.float32).astype(np.float64)
+    if io_dtype == "bf16":
+        u = np.ascontiguousarray(x.astype(np.float32)).view(np.uint32).astype(np.uint64)
+        u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16 << 16
+        return u.astype(np.uint32).view(np.float32).astype(np.float64)
+    raise ValueError(f"unknown I/O type {io_dtype}")
+
+
+def project(x, W, io_dtype):
+    """The layer's projections ("entangled-state-attention 0.1.0", section
+    "Core idea": a = x W_A, v = x W_V, q = x W_Q): ``x`` [B, T, C_in], ``W``
+    [3C, C_in] (W_A, W_V, W_Q stacked, each [out, in]); float64 products,
+    rounded to the I/O type.  Returns a, v, q as [B, T, C] float64."""
+    x = _f64(x)
+    W = _f64(W)
+    C = W.shape[0] // 3
+    out = []
+    for p in range(3):
+        out.append(round_io(x @ W[p * C:(p + 1) * C].T, io_dtype))
+    return tuple(out)
+
+
+def fused_fwd(x, W, H, mode, io_dtype, E_init=None):
+    """Forward of the layer from its input: :func:`project`, then
+    :func:`scan_fwd` over H heads.  Returns ``(y, E_final)``, y [B, T, H, D]."""
+    a, v, q = project(x, W, io_dtype)
+    B, T, C = a.shape
+    D = C // H
+    shape = (B, T, H, D)
+    return scan_fwd(a.reshape(shape), v.reshape(shape), q.reshape(shape), mode, E_init=E_init)

@@ -386,6 +386,45 @@ def test_slices_composed_equal_the_whole_sequence(mode):
 
 
 # ---------------------------------------------------------------------------
+# The layer's projections (input of the fused forward).
+# ---------------------------------------------------------------------------
+
+def test_project_hand_example():
+    # C = 1, C_in = 2: W_A = [1, 0], W_V = [0, 1], W_Q = [1, -1]; x = (3, 5)
+    x = np.array([[[3.0, 5.0]]])
+    W = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, -1.0]])
+    a, v, q = oracle.project(x, W, "f32")
+    assert (a.item(), v.item(), q.item()) == (3.0, 5.0, -2.0)
+    # not symmetric: x W^T differs from x W
+    W2 = np.array([[0.0, 2.0], [1.0, 0.0], [0.5, 0.5]])
+    a, v, q = oracle.project(x, W2, "f32")
+    assert (a.item(), v.item(), q.item()) == (10.0, 3.0, 4.0)
+
+
+def test_round_io_matches_torch_conversions():
+    import torch
+    r = np.random.default_rng(40)
+    x = np.concatenate([r.normal(0, 1, 2000) * 10.0 ** r.integers(-6, 5, 2000), [0.0, -0.0, 65504.0, 1e-8]])
+    f16 = torch.from_numpy(x).to(torch.float16).double().numpy()
+    np.testing.assert_array_equal(oracle.round_io(x, "f16"), f16)
+    bf = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(oracle.round_io(x, "bf16"), bf)
+
+
+def test_fused_forward_is_projection_then_scan():
+    r = np.random.default_rng(41)
+    x = r.normal(0, 1, (2, 9, 16))
+    W = r.normal(0, 0.25, (3 * 8, 16))
+    y, Ef = oracle.fused_fwd(x, W, 2, C_, "f16")
+    a = oracle.round_io(x @ W[:8].T, "f16").reshape(2, 9, 2, 4)
+    v = oracle.round_io(x @ W[8:16].T, "f16").reshape(2, 9, 2, 4)
+    q = oracle.round_io(x @ W[16:].T, "f16").reshape(2, 9, 2, 4)
+    y2, Ef2 = oracle.scan_fwd(a, v, q, C_)
+    np.testing.assert_array_equal(y, y2)
+    np.testing.assert_array_equal(Ef, Ef2)
+
+
+# ---------------------------------------------------------------------------
 # The only printed worked examples are shapes.
 # ---------------------------------------------------------------------------
 
