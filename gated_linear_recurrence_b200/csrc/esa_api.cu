@@ -365,8 +365,9 @@ int esa_compose(const float *P, const float *S, int n, long long count, int reve
   return esa::launch_compose(P, S, n, static_cast<long>(count), reverse, x0, x, static_cast<cudaStream_t>(stream));
 }
 
-int esa_fused_fwd(const void *x, const void *W, void *y, float *E_final, int B, int T, int H, int D, int C_in,
-                  int mode, const float *E_init, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+int esa_fused_fwd(const void *x, const void *W, void *y, float *E_final, void *a, void *v, void *q, int B, int T,
+                  int H, int D, int C_in, int mode, const float *E_init, int dtype, void *workspace,
+                  size_t workspace_bytes, void *stream) {
   int rc = check_shape(B, T, H, D, mode, dtype);
   if (rc) return rc;
   if (C_in < 1) return ESA_ERR_ARG;
@@ -375,7 +376,9 @@ int esa_fused_fwd(const void *x, const void *W, void *y, float *E_final, int B, 
   if (!esa::fused_supported(dtype, D, C_in, lo.nct)) return ESA_ERR_UNSUPPORTED;
   const bool has_tokens = B > 0 && T > 0;
   if (has_tokens && (!x || !W || !y)) return ESA_ERR_ARG;
+  if ((a == nullptr) != (v == nullptr) || (a == nullptr) != (q == nullptr)) return ESA_ERR_ARG;
   for (const void *p : {x, W, static_cast<const void *>(y), static_cast<const void *>(E_final),
+                        static_cast<const void *>(a), static_cast<const void *>(v), static_cast<const void *>(q),
                         static_cast<const void *>(E_init), static_cast<const void *>(workspace)})
     if (p && !aligned16(p)) return ESA_ERR_ALIGN;
   if (!workspace || workspace_bytes < lo.total) return ESA_ERR_WORKSPACE;
@@ -400,6 +403,9 @@ int esa_fused_fwd(const void *x, const void *W, void *y, float *E_final, int B, 
   args.y = y;
   args.E_final = E_final;
   args.E_init = E_init;
+  args.a_out = a;
+  args.v_out = v;
+  args.q_out = q;
   args.ws = workspace_view(workspace, lo);
   return esa::launch_fused_fwd(dtype, mode, D, C_in, tx, tw, args, st);
 }

@@ -44,6 +44,7 @@ struct FusedArgs {
   void *y;
   float *E_final;
   const float *E_init;
+  void *a_out, *v_out, *q_out;   // the rounded projections [B][T][C], or all null
   Workspace ws;
 };
 
@@ -245,6 +246,13 @@ __global__ void __launch_bounds__(512, 1)
         uint4 out[4];
         pack32<T>(acc, out);
         const int p = c >> 6;
+        if (args.a_out != nullptr && (t0 + r) < sh.T) {   // the projections themselves, when asked for
+          T *dst = static_cast<T *>(p == 0 ? args.a_out : p == 1 ? args.v_out : args.q_out) +
+                   (static_cast<long>(b) * sh.T + t0 + r) * sh.C + c0 + (c & 63);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (c0 + (c & 63) + 8 * i < sh.C) reinterpret_cast<uint4 *>(dst)[i] = out[i];
+        }
         T *row = (p == 0 ? a_s : p == 1 ? v_s : q_s) + r * CT + (c & 63);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {

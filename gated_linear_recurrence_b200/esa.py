@@ -78,7 +78,7 @@ def load_library():
         lib.esa_scan_bwd_map.restype = I
         lib.esa_compose.argtypes = [P, P, I, ctypes.c_longlong, I, P, P, P]
         lib.esa_compose.restype = I
-        lib.esa_fused_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, P, I, P, S, P]
+        lib.esa_fused_fwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P, I, P, S, P]
         lib.esa_fused_fwd.restype = I
         lib.esa_step.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
         lib.esa_step.restype = I
@@ -312,13 +312,15 @@ def esa_compose(P, S, x0=None, reverse=False, out=None, stream=None):
 
 
 def esa_fused_fwd(x, W, H, mode=CONTROLLED, E_init=None, y=None, E_final=None, workspace=None, stream=None,
-                  want_E_final=True):
+                  want_E_final=True, want_avq=False):
     """Forward scan of the projections of ``x``: a, v, q = x W[:C]^T,
     x W[C:2C]^T, x W[2C:]^T (rounded to x's dtype), computed on the tensor
     cores inside the scan.  ``x``: [B, T, C_in] float16 / bfloat16; ``W``:
     [3C, C_in] of the same dtype; ``H`` heads of D = C / H channels.
 
-    Returns ``(y, E_final, workspace)`` with ``y`` [B, T, H, D].
+    Returns ``(y, E_final, workspace)`` with ``y`` [B, T, H, D], or with
+    ``want_avq`` ``(y, E_final, workspace, (a, v, q))``: the projections the
+    scan consumed, for :func:`esa_scan_bwd`.
     """
     if not isinstance(x, torch.Tensor) or not x.is_cuda or x.dim() != 3:
         raise TypeError("x must be a CUDA tensor [B, T, C_in] (the ESA library has no CPU path)")
@@ -341,14 +343,17 @@ def esa_fused_fwd(x, W, H, mode=CONTROLLED, E_init=None, y=None, E_final=None, w
     _check_state("E_init", E_init, B, H, D, x.device)
     if workspace is None:
         workspace = new_workspace(B, T, H, D, x.dtype, x.device)
+    avq = tuple(torch.empty((B, T, H, D), dtype=x.dtype, device=x.device) for _ in range(3)) if want_avq \
+        else (None, None, None)
     lib = load_library()
     with torch.cuda.device(x.device):
-        rc = lib.esa_fused_fwd(_ptr(x), _ptr(W), _ptr(y), _ptr(E_final), B, T, H, D, C_in, int(mode), _ptr(E_init),
+        rc = lib.esa_fused_fwd(_ptr(x), _ptr(W), _ptr(y), _ptr(E_final), *(_ptr(t) for t in avq), B, T, H, D, C_in,
+                               int(mode), _ptr(E_init),
                                _DTYPE_CODE[x.dtype], _ptr(workspace), workspace.numel() * workspace.element_size(),
                                _stream(x.device, stream))
     if rc != 0:
         raise EsaError("esa_fused_fwd", rc)
-    return y, E_final, workspace
+    return (y, E_final, workspace, avq) if want_avq else (y, E_final, workspace)
 
 
 def esa_step(a_t, v_t, q_t, E, y_t=None, mode=CONTROLLED, stream=None):

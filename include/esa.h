@@ -231,15 +231,19 @@ int esa_compose(const float *P, const float *S, int n, long long count, int reve
  *   W         [3C, C_in] the three projection weights stacked (rows 0..C-1:
  *             W_A, C..2C-1: W_V, 2C..3C-1: W_Q), each [out, in] as stored by
  *             a linear layer, I/O dtype (required).
- *   y, E_final, E_init, mode, workspace: as for esa_scan_fwd; the workspace
- *             may be shared with esa_scan_fwd (same size), but no backward
- *             can follow this call (a, v, q are not kept).
+ *   a, v, q   [B,T,H,D] outputs (optional, all NULL or none): the rounded
+ *             projections the scan consumed.  With them written, the call
+ *             is a complete training forward: esa_scan_bwd(a, v, q, ...) on
+ *             the same workspace gives the scan's gradients.  Without them
+ *             the call only reads x and W and writes y (inference, prefill).
+ *   y, E_final, E_init, mode, workspace: as for esa_scan_fwd.
  * Supported: dtype ESA_F16 or ESA_BF16, D <= 64, C_in of 64 or 128, C <= 3072;
  * other shapes return ESA_ERR_UNSUPPORTED (compute the projections
  * separately and call esa_scan_fwd).
  */
-int esa_fused_fwd(const void *x, const void *W, void *y, float *E_final, int B, int T, int H, int D, int C_in,
-                  int mode, const float *E_init, int dtype, void *workspace, size_t workspace_bytes, void *stream);
+int esa_fused_fwd(const void *x, const void *W, void *y, float *E_final, void *a, void *v, void *q, int B, int T,
+                  int H, int D, int C_in, int mode, const float *E_init, int dtype, void *workspace,
+                  size_t workspace_bytes, void *stream);
 
 /*
  * One-token recurrent update (decode): E <- A (.) E + B in place, then

@@ -4,20 +4,26 @@ The kernel computes a, v, q = x W_A^T, x W_V^T, x W_Q^T on the tensor cores
 (tcgen05), rounds them to the I/O type and scans them without writing them
 out.  It is compared with
 
-* the oracle: float64 projections rounded to the I/O type, then the fp64
-  scan (``oracle.fused_fwd``), on ragged lengths, partial channel tiles,
-  both input widths, both modes and dtypes, and a given initial state;
-* the unfused library path: the projections by torch (cuBLAS) in the I/O
-  type, then ``esa_scan_fwd``.
+* the oracle, in two parts: every projection the kernel produced (it can
+  write them out) against the float64 product, within half a unit in the
+  last place plus the float32 accumulation bound -- the rounding of a value
+  that lies within the accumulation error of a rounding midpoint can go
+  either way, so the projections are not compared with a rounded oracle
+  value; then the kernel's scan against the oracle's scan of exactly those
+  projections; on ragged lengths, partial channel tiles, both input widths,
+  both modes and dtypes, and a given initial state;
+* the library's own forward scan on the same projections: bitwise equal;
+* the library's backward on the fused forward's outputs and workspace.
 
 Inputs: x ~ N(0, 1), weights ~ N(0, 1 / C_in), so a, v, q ~ N(0, 1).
 """
+import numpy as np
 import pytest
 import torch
 
 import oracle
 from gated_linear_recurrence_b200 import esa, inputs
-from tests._parity import DT, TOL, assert_close, host64
+from tests._parity import DT, TOL, assert_close, half_ulp, host64
 
 pytestmark = pytest.mark.gpu
 
@@ -39,32 +45,76 @@ def _inputs(B, T, C_in, C, dt, seed, device):
     return x, W
 
 
+def _check_projections(x, W, avq, C, dtype):
+    """Each projection the kernel produced is the float64 product rounded to
+    the I/O type, up to the float32 accumulation inside the tensor core: it
+    lies within half a unit in the last place (of the I/O type) plus the
+    accumulation error bound 2^-15 sum_k |x_k W_k| of the exact product."""
+    x64, W64 = host64(x), host64(W)
+    B, T, _ = x.shape
+    for p, t in enumerate(avq):
+        Wp = W64[p * C:(p + 1) * C]
+        exact = x64 @ Wp.T
+        g = host64(t).reshape(B, T, C)
+        allowed = np.maximum(half_ulp(exact, dtype), half_ulp(g, dtype)) + 2.0 ** -15 * (np.abs(x64) @ np.abs(Wp).T)
+        err = np.abs(g - exact)
+        worst = np.unravel_index(np.argmax(err / allowed), err.shape)
+        assert err[worst] <= allowed[worst], (f"projection {'avq'[p]}: |err| {err[worst]:.3e} at {worst} "
+                                              f"(allowed {allowed[worst]:.3e})")
+
+
 @pytest.mark.parametrize("case", CASES, ids=[f"B{c[0]}T{c[1]}H{c[2]}D{c[3]}Cin{c[4]}m{c[5]}{c[6]}" for c in CASES])
 def test_fused_forward_matches_oracle(cuda_device, case):
+    """Projections against their float64 values; the scan of the projections
+    the kernel consumed against the oracle's scan of the same values."""
     B, T, H, D, C_in, mode, dt = case
     C = H * D
     x, W = _inputs(B, T, C_in, C, dt, 90 + T, cuda_device)
     E0 = inputs.make_state(B, H, D, seed=91, scale=0.5).to(cuda_device)
-    y, Ef, ws = esa.esa_fused_fwd(x, W, H, mode=mode, E_init=E0)
+    y, Ef, ws, avq = esa.esa_fused_fwd(x, W, H, mode=mode, E_init=E0, want_avq=True)
     esa.esa_check(ws)
-    y_r, Ef_r = oracle.fused_fwd(host64(x), host64(W), H, mode, dt, E_init=host64(E0))
+    _check_projections(x, W, avq, C, DT[dt])
+    y_r, Ef_r = oracle.scan_fwd(*(host64(t) for t in avq), mode, E_init=host64(E0))
     tol = TOL[DT[dt]]
     assert_close(y, y_r, tol, "y")
     assert_close(Ef, Ef_r, tol, "E_final")
 
 
-@pytest.mark.parametrize("case", CASES[:3], ids=[f"B{c[0]}T{c[1]}H{c[2]}D{c[3]}" for c in CASES[:3]])
-def test_fused_forward_matches_unfused_library_path(cuda_device, case):
+@pytest.mark.parametrize("case", CASES, ids=[f"B{c[0]}T{c[1]}H{c[2]}D{c[3]}Cin{c[4]}m{c[5]}{c[6]}" for c in CASES])
+def test_fused_scan_is_bitwise_the_library_scan(cuda_device, case):
+    """Given the same a, v, q the fused kernel's scan is the forward scan
+    kernel's arithmetic, operation for operation: y and E_final are bitwise
+    equal; with the projections requested or not, y is the same."""
     B, T, H, D, C_in, mode, dt = case
     C = H * D
     x, W = _inputs(B, T, C_in, C, dt, 95 + T, cuda_device)
-    y, Ef, ws = esa.esa_fused_fwd(x, W, H, mode=mode)
-    proj = [(x @ W[p * C:(p + 1) * C].T).reshape(B, T, H, D).contiguous() for p in range(3)]
-    y2, Ef2, _ = esa.esa_scan_fwd(*proj, mode=mode, workspace=ws)
+    y, Ef, ws, avq = esa.esa_fused_fwd(x, W, H, mode=mode, want_avq=True)
+    y_only, Ef_only, _ = esa.esa_fused_fwd(x, W, H, mode=mode, workspace=ws)
+    y2, Ef2, _ = esa.esa_scan_fwd(*avq, mode=mode, workspace=ws)
     esa.esa_check(ws)
+    assert torch.equal(y, y2) and torch.equal(Ef, Ef2)
+    assert torch.equal(y, y_only) and torch.equal(Ef, Ef_only)
+    # and the projections agree with cuBLAS's up to the accumulation order
+    proj = [(x @ W[p * C:(p + 1) * C].T) for p in range(3)]
+    for p in range(3):
+        d = (avq[p].reshape(B, T, C).float() - proj[p].float()).abs()
+        assert bool((d <= 2.0 ** -7 * proj[p].float().abs() + 1e-6).all()), f"projection {p} vs cuBLAS"
+
+
+def test_fused_forward_then_library_backward(cuda_device):
+    """With the projections written, the fused call is a training forward:
+    esa_scan_bwd on its outputs and workspace gives the oracle's gradients."""
+    B, T, H, D, C_in, mode, dt = 2, 600, 4, 32, 128, 1, "f16"
+    C = H * D
+    x, W = _inputs(B, T, C_in, C, dt, 97, cuda_device)
+    dy = torch.randn(B, T, H, D, generator=torch.Generator().manual_seed(98)).to(DT[dt]).to(cuda_device)
+    y, Ef, ws, (a, v, q) = esa.esa_fused_fwd(x, W, H, mode=mode, want_avq=True)
+    da, dv, dq, dE0 = esa.esa_scan_bwd(a, v, q, dy, ws, mode=mode)
+    esa.esa_check(ws)
+    ref = oracle.scan_bwd(host64(a), host64(v), host64(q), host64(dy), mode)
     tol = TOL[DT[dt]]
-    assert_close(y, host64(y2), tol, "y")
-    assert_close(Ef, host64(Ef2), tol, "E_final")
+    for name, g, r in zip(("da", "dv", "dq", "dE_init"), (da, dv, dq, dE0), ref):
+        assert_close(g, r, tol, name)
 
 
 def test_fused_forward_empty_and_reuse(cuda_device):
@@ -78,9 +128,9 @@ def test_fused_forward_empty_and_reuse(cuda_device):
     ws = esa.new_workspace(2, 700, H, D, torch.float16, cuda_device)
     for k, T in enumerate((700, 129, 511)):
         x, W = _inputs(2, T, C_in, H * D, "f16", 7 + k, cuda_device)
-        y, Ef, _ = esa.esa_fused_fwd(x, W, H, mode=1, workspace=ws)
+        y, Ef, _, avq = esa.esa_fused_fwd(x, W, H, mode=1, workspace=ws, want_avq=True)
         esa.esa_check(ws)
-        y_r, Ef_r = oracle.fused_fwd(host64(x), host64(W), H, 1, "f16")
+        y_r, Ef_r = oracle.scan_fwd(*(host64(t) for t in avq), 1)
         assert_close(y, y_r, TOL[torch.float16], f"call{k}.y")
         assert_close(Ef, Ef_r, TOL[torch.float16], f"call{k}.E_final")
 
