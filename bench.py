@@ -57,6 +57,10 @@ def parse_args(argv=None):
                     help="skip the prefill + decode (esa_step) measurement reported under detail.decode")
     ap.add_argument("--no-cp", action="store_true",
                     help="skip the per-rank context-parallel phase timing reported under detail.context_parallel")
+    ap.add_argument("--no-fused", action="store_true",
+                    help="skip the fused projection + scan forward timing reported under detail.fused_layer_forward")
+    ap.add_argument("--fused-only", action="store_true",
+                    help="run only the fused projection + scan forward timing (one JSON line; for profiling)")
     ap.add_argument("--cp-only", action="store_true",
                     help="run only the context-parallel phase timing (one JSON line; for profiling its kernels)")
     ap.add_argument("--batch", type=int, default=None,
@@ -492,6 +496,85 @@ def measure_context_parallel(dev, n_slices=8, reps=5):
             "note": "one GPU: per-rank device time of every phase; the all-gathers are not included"}
 
 
+def measure_fused(dev, reps=10, seq=None):
+    """The layer's forward from its input: projections + scan.
+
+    Same shape as the benchmark workload (B = 64, T = 65536, H = 4, D = 32,
+    controlled, fp16) with C_in = C = 128: x ~ N(0, 1), W ~ N(0, 1/C_in).
+    Three ways, device-timed with CUDA events, inputs resident in HBM:
+      fused      esa_fused_fwd: x -> y (tcgen05 projections inside the scan);
+      fused_avq  the same, also writing a, v, q (what a backward needs);
+      unfused    three cuBLAS projections (torch matmul into contiguous
+                 a, v, q), then esa_scan_fwd.
+    Algorithmic bytes per token: fused (C_in + C) s, fused_avq (C_in + 4 C) s,
+    unfused (C_in + 3 C) s for the GEMMs + 4 C s for the scan.
+    """
+    import torch
+
+    from gated_linear_recurrence_b200 import esa
+    w = workload(seq=seq)
+    B, T, H, D, mode = w.B, w.T, w.H, w.D, w.mode
+    C = H * D
+    C_in = C
+    g = torch.Generator(device=dev).manual_seed(w.seed + 11)
+    x = torch.randn(B, T, C_in, generator=g, device=dev).half()
+    W = (torch.randn(3 * C, C_in, generator=g, device=dev) / C_in ** 0.5).half()
+    y = torch.empty(B, T, H, D, dtype=torch.float16, device=dev)
+    Ef = torch.empty(B, H, D, dtype=torch.float32, device=dev)
+    avq = [torch.empty(B, T, H, D, dtype=torch.float16, device=dev) for _ in range(3)]
+    ws = esa.new_workspace(B, T, H, D, torch.float16, dev)
+    stream = torch.cuda.current_stream(dev)
+    Wp = [W[p * C:(p + 1) * C] for p in range(3)]
+
+    def fused():
+        esa.esa_fused_fwd(x, W, H, mode=mode, y=y, E_final=Ef, workspace=ws)
+
+    def fused_avq():
+        lib = esa.load_library()
+        rc = lib.esa_fused_fwd(esa._ptr(x), esa._ptr(W), esa._ptr(y), esa._ptr(Ef), *(esa._ptr(t) for t in avq),
+                               B, T, H, D, C_in, mode, None, 1, esa._ptr(ws), ws.numel(), esa._stream(dev, None))
+        if rc != 0:
+            raise esa.EsaError("esa_fused_fwd", rc)
+
+    def unfused():
+        for p in range(3):
+            torch.matmul(x, Wp[p].T, out=avq[p].view(B, T, C))
+        esa.esa_scan_fwd(avq[0], avq[1], avq[2], y=y, E_final=Ef, mode=mode, workspace=ws)
+
+    out = {}
+    for name, fn in (("fused", fused), ("fused_avq", fused_avq), ("unfused", unfused)):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out[name + "_ms"] = e0.elapsed_time(e1) / reps
+    esa.esa_check(ws)
+    tok = B * T
+    s_ = 2
+    peak, _ = measured_peak()
+    fb = (C_in + C) * s_ * tok
+    fb_avq = (C_in + 4 * C) * s_ * tok
+    out.update({
+        "workload": f"controlled_f16_B{B}_T{T}_H{H}_D{D}_Cin{C_in}",
+        "fused_tokens_per_s": tok / (out["fused_ms"] / 1e3),
+        "fused_avq_tokens_per_s": tok / (out["fused_avq_ms"] / 1e3),
+        "unfused_tokens_per_s": tok / (out["unfused_ms"] / 1e3),
+        "speedup_vs_unfused": out["unfused_ms"] / out["fused_ms"],
+        "fused_algorithmic_bytes": fb, "fused_GBs": fb / (out["fused_ms"] / 1e3) / 1e9,
+        "fused_frac_of_measured_hbm": fb / (out["fused_ms"] / 1e3) / 1e9 / peak,
+        "fused_avq_GBs": fb_avq / (out["fused_avq_ms"] / 1e3) / 1e9,
+        "fused_tensor_TFLOPs": 2 * 3 * C * C_in * tok / (out["fused_ms"] / 1e3) / 1e12,
+        "note": "fused kernel: one CTA per SM, two tile groups of 256 threads, weights resident in shared memory"})
+    del x, W, y, avq, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------------------
 # Our arm.
 # ---------------------------------------------------------------------------
@@ -624,6 +707,9 @@ def run_ours(args):
     cpar = None
     if not args.no_cp and args.batch is None and args.seq is None:
         cpar = measure_context_parallel(dev)
+    fusedm = None
+    if not args.no_fused and args.batch is None and args.seq is None:
+        fusedm = measure_fused(dev)
 
     cpu = cpu_all = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -643,7 +729,7 @@ def run_ours(args):
                    "bwd_GBs": bwd_bytes / (bwd_ms / 1e3) / 1e9, "step_GBs": step_gbs,
                    "step_frac_of_measured_peak": step_gbs / peak, "step_frac_of_nominal_8TBs":
                    step_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes_per_step": fwd_bytes + bwd_bytes,
-                   "decode": decode, "context_parallel": cpar, "cpu_baseline_all_cores": cpu_all},
+                   "decode": decode, "context_parallel": cpar, "fused_layer_forward": fusedm, "cpu_baseline_all_cores": cpu_all},
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": 2 * K,
@@ -662,11 +748,14 @@ def main(argv=None):
         raise SystemExit("--warmup must be at least 3")
     if args.impl == "reference":
         return run_reference(args)
-    if args.cp_only:
+    if args.cp_only or args.fused_only:
         import torch
         dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
         torch.cuda.set_device(dev)
-        print(json.dumps({"context_parallel": measure_context_parallel(dev)}), flush=True)
+        if args.cp_only:
+            print(json.dumps({"context_parallel": measure_context_parallel(dev)}), flush=True)
+        else:
+            print(json.dumps({"fused_layer_forward": measure_fused(dev, seq=args.seq)}), flush=True)
         return 0
     return run_ours(args)
 

@@ -21,12 +21,14 @@
 //     tensor memory, and runs its own persistent loop over tiles taken from
 //     the channel tile's ticket counter (batch row fastest), so the two
 //     groups hide each other's latencies as two CTAs per SM would.
-//   * Per tile: wait for x (TMA); one thread issues C_in / 16 MMAs of
-//     128 x 192 x 16 and commits them to an mbarrier; once they are done the
+//   * Per tile: one thread issues C_in / 16 MMAs of 128 x 192 x 16 on the
+//     tile's x rows and commits them to an mbarrier; once they are done the
 //     x buffer is refilled with the next tile's rows; the group's 8 warps
 //     read the accumulator (warp w: lanes 32 (w mod 4).., 96 columns) and
 //     store a, v, q; then pass 1, the run scan, the look-back and pass 2 as
-//     in the forward scan.
+//     in the forward scan.  While the tile scans, the issuing thread checks
+//     (without blocking) whether the next tile's x has landed and, if so,
+//     starts its MMAs at once, so they run under this tile's scan.
 //   * Every wait is bounded; tensor memory is freed at the end whatever
 //     happened.
 #pragma once
@@ -64,6 +66,13 @@ struct FusedPlan {
   static_assert(kW % 1024 == 0 && kX % 1024 == 0 && kGroup % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static_assert(kBytes <= 227 * 1024, "shared memory");
 };
+
+// The a / v / q boxes are [128 rows][64 channels] with the eight 16-byte
+// vectors of a row permuted by the row: vector j of row r sits at position
+// j ^ (r mod 8).  The accumulator read-out writes 32 consecutive rows per
+// warp instruction and the scan reads 4 rows x 8 vectors; both touch every
+// bank once per 128 bytes.
+__device__ __forceinline__ int box_vec(int j, int r) { return j ^ (r & 7); }
 
 __device__ __forceinline__ unsigned char *smem_aligned1024(unsigned char *smem) {
   const uint32_t a = smem_u32(smem);
@@ -192,7 +201,30 @@ __global__ void __launch_bounds__(512, 1)
   const ThreadPos<Cfg> pos(tid);
   T *yg = static_cast<T *>(args.y);
   const unsigned tag = *tag_s;
-  unsigned ph_x = 0, ph_m = 0;
+  unsigned ph_x = 0, ph_m = 0;   // ph_x: the group's thread 0 only
+  bool pre = false;              // thread 0: the current tile's MMAs were issued during the previous tile
+  bool next_ok = false;          // thread 0: the next ticket is a tile
+  // MMAs of the tile whose x is in the buffer (thread 0; the accumulator is free).
+  auto issue_mma = [&]() {
+    tc_fence_after();
+    const uint32_t xa = smem_u32(x_s), wa = smem_u32(w_s);
+#pragma unroll
+    for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        umma_f16(tmem_d, umma_desc_sw128(xa + kb * Pl::kXkb) + 2 * kk, umma_desc_sw128(wa + kb * Pl::kWkb) + 2 * kk,
+                 kIdesc, (kb | kk) != 0);
+    umma_commit(&bar[1]);
+  };
+  // Start the next tile's MMAs as soon as its x has landed, while this tile
+  // is still scanning (thread 0, after this tile's accumulator was read).
+  auto try_issue_next = [&]() {
+    if (tid == 0 && next_ok && !pre && mbar_test_wait(&bar[0], ph_x)) {
+      ph_x ^= 1u;
+      issue_mma();
+      pre = true;
+    }
+  };
 
   for (int it = 0;; ++it) {
     const TileInfo ti = info_s[it & 1];
@@ -203,19 +235,14 @@ __global__ void __launch_bounds__(512, 1)
 
     // ---- projections on the tensor cores -----------------------------------
     if (tid == 0) {
-      if (it == 0) mbar_wait_bounded(w_bar, 0u, &hdr->status);
-      mbar_wait_bounded(&bar[0], ph_x, &hdr->status);
-      tc_fence_after();
-      const uint32_t xa = smem_u32(x_s), wa = smem_u32(w_s);
-#pragma unroll
-      for (int kb = 0; kb < KB; ++kb)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_f16(tmem_d, umma_desc_sw128(xa + kb * Pl::kXkb) + 2 * kk, umma_desc_sw128(wa + kb * Pl::kWkb) + 2 * kk,
-                   kIdesc, (kb | kk) != 0);
-      umma_commit(&bar[1]);
+      if (!pre) {
+        if (it == 0) mbar_wait_bounded(w_bar, 0u, &hdr->status);
+        mbar_wait_bounded(&bar[0], ph_x, &hdr->status);
+        ph_x ^= 1u;
+        issue_mma();
+      }
+      pre = false;
     }
-    ph_x ^= 1u;
 
     const bool lb_thread = tid >= Cfg::LB0 && tid < Cfg::LB0 + CT;
     unsigned long long early = 0ull;
@@ -228,7 +255,8 @@ __global__ void __launch_bounds__(512, 1)
       const int nt = static_cast<int>(atomicAdd(&hdr->ct_ticket[ct], 1u));
       const TileInfo tn = decode(nt);
       info_s[(it + 1) & 1] = tn;
-      if (nt < args.ntiles_ct) issue_x(tn);
+      next_ok = nt < args.ntiles_ct;
+      if (next_ok) issue_x(tn);
     }
 
     // ---- accumulator -> a, v, q boxes (rounded to the I/O type) ------------
@@ -253,13 +281,9 @@ __global__ void __launch_bounds__(512, 1)
           for (int i = 0; i < 4; ++i)
             if (c0 + (c & 63) + 8 * i < sh.C) reinterpret_cast<uint4 *>(dst)[i] = out[i];
         }
-        T *row = (p == 0 ? a_s : p == 1 ? v_s : q_s) + r * CT + (c & 63);
+        uint4 *row = reinterpret_cast<uint4 *>((p == 0 ? a_s : p == 1 ? v_s : q_s) + r * CT);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int piece = (i + lane) & 3;   // rotate the 16-byte pieces across lanes (bank spread)
-          const uint4 u = piece == 0 ? out[0] : piece == 1 ? out[1] : piece == 2 ? out[2] : out[3];
-          reinterpret_cast<uint4 *>(row)[piece] = u;
-        }
+        for (int i = 0; i < 4; ++i) row[box_vec(((c & 63) >> 3) + i, r)] = out[i];
       }
     }
     tc_fence_before();
@@ -292,8 +316,8 @@ __global__ void __launch_bounds__(512, 1)
       const int r = pos.row0 + i;
       const bool valid = (t0 + r) < sh.T;
       float2 x[4], vv[4];
-      Io<T>::load8_gate(a_s + r * CT + pos.ch, x);
-      Io<T>::load8(v_s + r * CT + pos.ch, vv);
+      Io<T>::load8_gate(a_s + r * CT + 8 * box_vec(pos.vec, r), x);
+      Io<T>::load8(v_s + r * CT + 8 * box_vec(pos.vec, r), vv);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const Gate2 gt = gate2(x[q]);
@@ -324,6 +348,7 @@ __global__ void __launch_bounds__(512, 1)
     }
     if (lb_thread) resolve_carry();
     named_sync(bar_all, Pl::NTG);
+    try_issue_next();
     if (publisher) {   // chunk-end state of the pair
       const float2 E_in = reinterpret_cast<const float2 *>(es_s)[c2];
       const float2 E_end = fma2(tP, E_in, tS);
@@ -346,8 +371,8 @@ __global__ void __launch_bounds__(512, 1)
         const int r = pos.row0 + i;
         const bool valid = (t0 + r) < sh.T;
         float2 vv[4], qq[4];
-        Io<T>::load8(v_s + r * CT + pos.ch, vv);
-        Io<T>::load8(q_s + r * CT + pos.ch, qq);
+        Io<T>::load8(v_s + r * CT + 8 * box_vec(pos.vec, r), vv);
+        Io<T>::load8(q_s + r * CT + 8 * box_vec(pos.vec, r), qq);
         float2 ss = splat(0.0f);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -361,6 +386,7 @@ __global__ void __launch_bounds__(512, 1)
         if (valid && ch_ok) Io<T>::store8(yg + gbase + static_cast<long>(r) * sh.C, yv);
       }
     }
+    try_issue_next();
     named_sync(bar_all, Pl::NTG);   // boxes, scratch and carries are free for the next tile
   }
 
