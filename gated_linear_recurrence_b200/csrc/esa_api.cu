@@ -397,6 +397,13 @@ int esa_fused_fwd(const void *x, const void *W, void *y, float *E_final, void *a
   const cuuint64_t wdims[2] = {static_cast<cuuint64_t>(C_in), static_cast<cuuint64_t>(3) * C};
   if ((rc = make_tmap_sw128(&tx, x, dtype, 3, xdims, 128))) return rc;
   if ((rc = make_tmap_sw128(&tw, W, dtype, 2, wdims, 64))) return rc;
+  CUtensorMap tavq[3] = {tx, tx, tx};   // placeholders when the projections are not stored
+  if (a != nullptr) {
+    const cuuint64_t pdims[3] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
+    const void *outs[3] = {a, v, q};
+    for (int i = 0; i < 3; ++i)
+      if ((rc = make_tmap_sw128(&tavq[i], outs[i], dtype, 3, pdims, 128))) return rc;
+  }
   esa::FusedArgs args;
   args.s = scan_shape(B, T, H, D, lo, 2);
   args.ntiles_ct = B * args.s.nchunks;
@@ -407,7 +414,7 @@ int esa_fused_fwd(const void *x, const void *W, void *y, float *E_final, void *a
   args.v_out = v;
   args.q_out = q;
   args.ws = workspace_view(workspace, lo);
-  return esa::launch_fused_fwd(dtype, mode, D, C_in, tx, tw, args, st);
+  return esa::launch_fused_fwd(dtype, mode, D, C_in, tx, tw, tavq, args, st);
 }
 
 int esa_step(const void *a_t, const void *v_t, const void *q_t, float *E, void *y_t, int B, int H, int D,

@@ -9,7 +9,8 @@ namespace esa {
 namespace {
 
 template <typename T, int MODE, int LPH, int CIN>
-int run_fused(const CUtensorMap &tx, const CUtensorMap &tw, const FusedArgs &args, cudaStream_t stream) {
+int run_fused(const CUtensorMap &tx, const CUtensorMap &tw, const CUtensorMap *tavq, const FusedArgs &args,
+              cudaStream_t stream) {
   using Pl = FusedPlan<T, CIN>;
   auto kern = esa_fused_fwd_kernel<T, MODE, LPH, CIN>;
   const size_t smem = Pl::kBytes;
@@ -27,26 +28,28 @@ int run_fused(const CUtensorMap &tx, const CUtensorMap &tw, const FusedArgs &arg
   const int need = (args.ntiles_ct + Pl::NG - 1) / Pl::NG;
   if (per_ct > need) per_ct = need;
   if (per_ct < 1) return -5;
-  kern<<<dim3(per_ct, nct), 512, smem, stream>>>(tx, tw, args);
+  kern<<<dim3(per_ct, nct), 512, smem, stream>>>(tx, tw, tavq[0], tavq[1], tavq[2], args);
   return launch_status(cudaGetLastError());
 }
 
 template <typename T, int MODE, int LPH>
-int by_cin(int cin, const CUtensorMap &tx, const CUtensorMap &tw, const FusedArgs &args, cudaStream_t st) {
+int by_cin(int cin, const CUtensorMap &tx, const CUtensorMap &tw, const CUtensorMap *tavq, const FusedArgs &args,
+           cudaStream_t st) {
   switch (cin) {
-    case 64: return run_fused<T, MODE, LPH, 64>(tx, tw, args, st);
-    case 128: return run_fused<T, MODE, LPH, 128>(tx, tw, args, st);
+    case 64: return run_fused<T, MODE, LPH, 64>(tx, tw, tavq, args, st);
+    case 128: return run_fused<T, MODE, LPH, 128>(tx, tw, tavq, args, st);
     default: return -3;
   }
 }
 
 template <typename T, int MODE>
-int by_d(int D, int cin, const CUtensorMap &tx, const CUtensorMap &tw, const FusedArgs &args, cudaStream_t st) {
+int by_d(int D, int cin, const CUtensorMap &tx, const CUtensorMap &tw, const CUtensorMap *tavq,
+         const FusedArgs &args, cudaStream_t st) {
   switch (D) {
-    case 8: return by_cin<T, MODE, 1>(cin, tx, tw, args, st);
-    case 16: return by_cin<T, MODE, 2>(cin, tx, tw, args, st);
-    case 32: return by_cin<T, MODE, 4>(cin, tx, tw, args, st);
-    case 64: return by_cin<T, MODE, 8>(cin, tx, tw, args, st);
+    case 8: return by_cin<T, MODE, 1>(cin, tx, tw, tavq, args, st);
+    case 16: return by_cin<T, MODE, 2>(cin, tx, tw, tavq, args, st);
+    case 32: return by_cin<T, MODE, 4>(cin, tx, tw, tavq, args, st);
+    case 64: return by_cin<T, MODE, 8>(cin, tx, tw, tavq, args, st);
     default: return -3;
   }
 }
@@ -54,13 +57,15 @@ int by_d(int D, int cin, const CUtensorMap &tx, const CUtensorMap &tw, const Fus
 }  // namespace
 
 int launch_fused_fwd(int dtype, int mode, int D, int cin, const CUtensorMap &tx, const CUtensorMap &tw,
-                     const FusedArgs &args, cudaStream_t stream) {
+                     const CUtensorMap *tavq, const FusedArgs &args, cudaStream_t stream) {
   if (mode != 0 && mode != 1) return -1;
   switch (dtype) {
-    case 1: return mode ? by_d<__half, 1>(D, cin, tx, tw, args, stream) : by_d<__half, 0>(D, cin, tx, tw, args, stream);
+    case 1:
+      return mode ? by_d<__half, 1>(D, cin, tx, tw, tavq, args, stream)
+                  : by_d<__half, 0>(D, cin, tx, tw, tavq, args, stream);
     case 2:
-      return mode ? by_d<__nv_bfloat16, 1>(D, cin, tx, tw, args, stream)
-                  : by_d<__nv_bfloat16, 0>(D, cin, tx, tw, args, stream);
+      return mode ? by_d<__nv_bfloat16, 1>(D, cin, tx, tw, tavq, args, stream)
+                  : by_d<__nv_bfloat16, 0>(D, cin, tx, tw, tavq, args, stream);
     default: return -3;
   }
 }

@@ -100,7 +100,8 @@ __device__ __forceinline__ void pack32(const uint32_t (&v)[32], uint4 (&out)[4])
 template <typename T, int MODE, int LPH, int CIN>
 __global__ void __launch_bounds__(512, 1)
     esa_fused_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                         const FusedArgs args) {
+                         const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
+                         const __grid_constant__ CUtensorMap tm_q, const FusedArgs args) {
   using Pl = FusedPlan<T, CIN>;
   constexpr int L = Pl::L, CT = Pl::CT, K = Pl::K, SUB = Pl::SUB, KB = Pl::KB;
   constexpr int SW = scan_segments<L / K, Pl::NTG, CT>();
@@ -274,20 +275,23 @@ __global__ void __launch_bounds__(512, 1)
         uint4 out[4];
         pack32<T>(acc, out);
         const int p = c >> 6;
-        if (args.a_out != nullptr && (t0 + r) < sh.T) {   // the projections themselves, when asked for
-          T *dst = static_cast<T *>(p == 0 ? args.a_out : p == 1 ? args.v_out : args.q_out) +
-                   (static_cast<long>(b) * sh.T + t0 + r) * sh.C + c0 + (c & 63);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            if (c0 + (c & 63) + 8 * i < sh.C) reinterpret_cast<uint4 *>(dst)[i] = out[i];
-        }
         uint4 *row = reinterpret_cast<uint4 *>((p == 0 ? a_s : p == 1 ? v_s : q_s) + r * CT);
 #pragma unroll
         for (int i = 0; i < 4; ++i) row[box_vec(((c & 63) >> 3) + i, r)] = out[i];
       }
     }
+    const bool store_avq = args.a_out != nullptr;
+    if (store_avq) fence_proxy_async_smem();   // box writes, before the TMA store reads them
     tc_fence_before();
     named_sync(bar_all, Pl::NTG);
+    // The projections themselves, when asked for: the boxes' layout is the
+    // 128-byte swizzle, so one TMA store per box writes them out.
+    if (store_avq && tid == 0) {
+      tma_store_3d(&tm_a, c0, t0, b, a_s);
+      tma_store_3d(&tm_v, c0, t0, b, v_s);
+      tma_store_3d(&tm_q, c0, t0, b, q_s);
+      bulk_commit();
+    }
 
     float *scan_s = reinterpret_cast<float *>(a_s);   // reused once pass 1 is done
 
@@ -328,7 +332,16 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
     }
-    if constexpr (Cfg::kWarpScratch) __syncwarp(); else named_sync(bar_all, Pl::NTG);
+    // The scan scratch overwrites the a box: with the projections being
+    // stored, the whole group waits until the TMA store has read it.
+    if (store_avq) {
+      if (tid == 0) bulk_wait_read0();
+      named_sync(bar_all, Pl::NTG);
+    } else if constexpr (Cfg::kWarpScratch) {
+      __syncwarp();
+    } else {
+      named_sync(bar_all, Pl::NTG);
+    }
     scan_store8<CT>(scan_s, pos.run, pos.ch, P, S);
     named_sync(bar_all, Pl::NTG);
 
@@ -392,8 +405,10 @@ __global__ void __launch_bounds__(512, 1)
 
   // ---- end: free tensor memory, count the CTA out ----------------------------
   // A CTA whose groups found no tile never waited for the weight slice; its
-  // copy must have landed before the CTA's shared memory goes away.
+  // copy must have landed before the CTA's shared memory goes away, and so
+  // must the groups' last projection stores.
   if (threadIdx.x == 0) mbar_wait_bounded(w_bar, 0u, &hdr->status);
+  if (tid == 0) bulk_wait0();
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x < 32) {

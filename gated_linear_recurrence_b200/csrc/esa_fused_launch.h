@@ -16,8 +16,10 @@ inline bool fused_supported(int dtype, int D, int cin, int nct) {
 }
 
 // tx: x [B][T][C_in] in boxes of [128 rows][64 elements], 128-byte swizzle;
-// tw: W [3 C][C_in] in boxes of [64 rows][64 elements], 128-byte swizzle.
+// tw: W [3 C][C_in] in boxes of [64 rows][64 elements], 128-byte swizzle;
+// tavq[3]: a, v, q [B][T][C] in boxes of [128 rows][64 channels], 128-byte
+// swizzle (used only when args.a_out is set).
 int launch_fused_fwd(int dtype, int mode, int D, int cin, const CUtensorMap &tx, const CUtensorMap &tw,
-                     const FusedArgs &args, cudaStream_t stream);
+                     const CUtensorMap *tavq, const FusedArgs &args, cudaStream_t stream);
 
 }  // namespace esa

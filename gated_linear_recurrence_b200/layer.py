@@ -11,9 +11,14 @@
   recurrence (direct or controlled) over each head, and ``y = W_O(q * Norm(E))``
   with Norm the per-head RMS.
 
-The projections are dense GEMMs outside the scan; they run as ordinary
-``torch.nn.Linear`` layers.  Every step of the recurrence and its readout runs
-in the CUDA library; there is no CPU path.
+When the shapes allow it (16-bit weights and input, no bias, head dimension
+<= 64, input width 64 or 128) the input projections run inside the scan
+kernel on the tensor cores (``esa_fused_fwd``); in training that call also
+writes a, v, q for the library backward, and the projections' own gradients
+(dx, dW) are ordinary GEMMs.  Otherwise the projections are
+``torch.nn.Linear`` layers feeding ``esa_scan``.  W_O is always a linear
+layer.  Every step of the recurrence and its readout runs in the CUDA
+library; there is no CPU path.
 """
 from __future__ import annotations
 
@@ -52,6 +57,42 @@ class _EsaScanFn(torch.autograd.Function):
         return da, dv, dq, (dE0 if ctx.has_E_init else None), None
 
 
+class _FusedProjScanFn(torch.autograd.Function):
+    """(x, W = [W_A; W_V; W_Q]) -> (y, E_final) through esa_fused_fwd; the
+    backward is esa_scan_bwd on the projections the forward wrote, then the
+    projections' gradients dx = [da dv dq] W and dW = [da dv dq]^T x."""
+
+    @staticmethod
+    def forward(ctx, x, W, E_init, mode, H):
+        x = x.contiguous()
+        W = W.contiguous()
+        E0 = None if E_init is None else E_init.detach().contiguous().float()
+        train = any(ctx.needs_input_grad[:3])
+        out = _esa.esa_fused_fwd(x, W, H, mode=mode, E_init=E0, want_avq=train)
+        y, E_final, ws = out[:3]
+        ctx.mode, ctx.has_E_init = mode, E_init is not None
+        if train:
+            a, v, q = out[3]
+            ctx.ws = ws
+            ctx.save_for_backward(x, W, a, v, q, E0 if E0 is not None else torch.empty(0, device=x.device))
+        return y, E_final
+
+    @staticmethod
+    def backward(ctx, dy, dE_final):
+        x, W, a, v, q, E0 = ctx.saved_tensors
+        E0 = E0 if ctx.has_E_init else None
+        dy = torch.zeros_like(a) if dy is None else dy.to(a.dtype).contiguous()
+        dEf = None if dE_final is None else dE_final.float().contiguous()
+        da, dv, dq, dE0 = _esa.esa_scan_bwd(a, v, q, dy, ctx.ws, mode=ctx.mode, E_init=E0, dE_final=dEf,
+                                            want_dE_init=ctx.has_E_init)
+        ctx.ws = None
+        B, T = x.shape[:2]
+        G = torch.cat([t.reshape(B * T, -1) for t in (da, dv, dq)], dim=1)   # [B T, 3 C]
+        dx = (G @ W).reshape(x.shape)
+        dW = G.t() @ x.reshape(B * T, -1)
+        return dx, dW, (dE0 if ctx.has_E_init else None), None, None
+
+
 def esa_scan(a, v, q, mode="controlled", E_init=None):
     """Differentiable scan of ``[B, T, H, D]`` CUDA tensors (float32, float16
     or bfloat16).  Returns ``(y, E_final)``; ``E_final`` is float32
@@ -72,6 +113,9 @@ class ESA(torch.nn.Module):
         scan_dtype: dtype the scan reads and writes (float16, bfloat16 or
             float32); the state is float32 either way.  ``None`` keeps the
             dtype of the projections' output.
+        fused: run the input projections inside the scan kernel
+            (``esa_fused_fwd``): ``None`` (default) whenever the shapes and
+            dtypes allow it, ``True`` to require it, ``False`` never.
         cp_group: a ``torch.distributed`` process group over which each
             sequence is split along time (context parallelism: rank r of the
             group passes the r-th time slice of the sequence); ``None`` runs
@@ -85,7 +129,8 @@ class ESA(torch.nn.Module):
     """
 
     def __init__(self, embd: int, head: int, mode: str = "controlled", bias: bool = False,
-                 scan_dtype: torch.dtype | None = None, device=None, dtype=None, cp_group=None):
+                 scan_dtype: torch.dtype | None = None, device=None, dtype=None, cp_group=None,
+                 fused: bool | None = None):
         super().__init__()
         if embd % head != 0:
             raise ValueError("embd must be a multiple of head")
@@ -97,6 +142,7 @@ class ESA(torch.nn.Module):
         self.head_dim = embd // head
         self.scan_dtype = scan_dtype
         self.cp_group = cp_group
+        self.fused = fused
         kw = {"device": device, "dtype": dtype}
         self.W_A = torch.nn.Linear(embd, embd, bias=bias, **kw)
         self.W_V = torch.nn.Linear(embd, embd, bias=bias, **kw)
@@ -111,10 +157,26 @@ class ESA(torch.nn.Module):
             out.append((t if dt is None else t.to(dt)).contiguous())
         return out
 
+    def _fused_ok(self, x):
+        dt = self.W_A.weight.dtype
+        return (x.is_cuda and self.cp_group is None and self.W_A.bias is None and dt in (torch.float16, torch.bfloat16)
+                and x.dtype == dt and self.scan_dtype in (None, dt) and self.head_dim <= 64
+                and self.embd in (64, 128) and -(-self.embd // 64) <= 48)
+
     def forward(self, x, state=None, return_state=False):
         B, T, C = x.shape
         if C != self.embd:
             raise ValueError(f"expected last dimension {self.embd}, got {C}")
+        use_fused = self._fused_ok(x) if self.fused is None else bool(self.fused)
+        if use_fused:
+            if not self._fused_ok(x):
+                raise ValueError("fused=True needs 16-bit CUDA input and weights of the same dtype, no bias, "
+                                 "head_dim <= 64, embd of 64 or 128 and no context-parallel group")
+            W = torch.cat([self.W_A.weight, self.W_V.weight, self.W_Q.weight], dim=0)
+            m = _MODES[self.mode]
+            y, E = _FusedProjScanFn.apply(x, W, state, m, self.head)
+            out = self.W_O(y.reshape(B, T, C).to(self.W_O.weight.dtype))
+            return (out, E) if return_state else out
         a, v, q = self._proj(x, (B, T, self.head, self.head_dim))
         if self.cp_group is not None:
             from .context_parallel import cp_esa_scan

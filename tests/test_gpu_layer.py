@@ -97,3 +97,50 @@ def test_layer_decode_matches_full_sequence(cuda_device):
     assert_close(out, host64(full[:, :T]), tol, "prefill")
     assert_close(torch.stack(steps, dim=1), host64(full[:, T:]), tol, "decode")
     assert np.isfinite(host64(state)).all()
+
+
+@pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("mode", ["controlled", "direct"])
+def test_fused_layer_matches_unfused_layer(cuda_device, dt, mode):
+    """16-bit layer: the projections inside the scan kernel (tcgen05) against
+    the same layer with linear projections, output and every gradient.  Both
+    round a, v, q to the 16-bit type; their GEMMs accumulate in different
+    orders, so a few roundings differ by one unit: tolerance 1e-2 (bf16) /
+    5e-3 (fp16) relative to (1 + |ref|)."""
+    torch.manual_seed(7)
+    B, T, C, H = 2, 333, 128, 4
+    fused = ESA(C, H, mode=mode, device=cuda_device, dtype=dt)
+    plain = ESA(C, H, mode=mode, device=cuda_device, dtype=dt, fused=False)
+    plain.load_state_dict(fused.state_dict())
+    assert fused._fused_ok(torch.empty(1, 1, C, device=cuda_device, dtype=dt))
+    x = torch.randn(B, T, C, device=cuda_device, dtype=dt)
+    E0 = torch.randn(B, H, C // H, device=cuda_device) * 0.3
+    g = torch.randn(B, T, C, device=cuda_device, dtype=dt)
+    res = []
+    for layer in (fused, plain):
+        xi = x.clone().requires_grad_(True)
+        Ei = E0.clone().requires_grad_(True)
+        out, E = layer(xi, state=Ei, return_state=True)
+        ((out.float() * g.float()).sum() + E.sum()).backward()
+        res.append([out.detach(), E.detach(), xi.grad, Ei.grad] +
+                   [getattr(layer, n).weight.grad for n in ("W_A", "W_V", "W_Q", "W_O")])
+    tol = 1e-2 if dt == torch.bfloat16 else 5e-3
+    names = ("out", "E_final", "dx", "dE0", "dW_A", "dW_V", "dW_Q", "dW_O")
+    for name, f_, p_ in zip(names, res[0], res[1]):
+        scale = float(p_.float().abs().max()) or 1.0
+        assert_close(f_.float() / scale, host64(p_.float()) / scale, tol, name)
+
+
+def test_fused_layer_inference_matches_reference(cuda_device):
+    """Inference through the fused path (no projections written) against
+    the float64 per-token loop, on the layer's own 16-bit weights."""
+    torch.manual_seed(8)
+    B, T, C, H = 2, 200, 64, 2
+    layer = ESA(C, H, mode="controlled", device=cuda_device, dtype=torch.float16)
+    x = torch.randn(B, T, C, device=cuda_device, dtype=torch.float16)
+    with torch.no_grad():
+        out = layer(x)
+    W = {n: getattr(layer, n).weight.detach().cpu().double() for n in ("W_A", "W_V", "W_Q", "W_O")}
+    ref = _reference_layer(x.cpu().double(), W["W_A"], W["W_V"], W["W_Q"], W["W_O"], H, "controlled")
+    scale = float(ref.abs().max())
+    assert_close(out.float() / scale, ref.numpy() / scale, 1e-2, "out")
