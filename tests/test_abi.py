@@ -187,3 +187,23 @@ def test_segment_map_calls_need_a_device(lib):
     assert lib.esa_scan_bwd_map(P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000), P(0x6000), 2, 8, 2, 32,
                                 1, None, 1, P(0x10000), 1 << 30, None) == esa.ESA_ERR_DEVICE
     assert lib.esa_compose(P(0x1000), P(0x2000), 2, 16, 0, None, P(0x3000), None) == esa.ESA_ERR_DEVICE
+
+
+def test_fused_forward_argument_errors(lib):
+    from gated_linear_recurrence_b200 import esa
+    P = _fake
+
+    def call(x=0x1000, W=0x2000, y=0x3000, a=None, v=None, q=None, B=2, T=8, H=2, D=32, cin=128, dtype=1, wsb=1 << 30):
+        return lib.esa_fused_fwd(P(x) if x else None, P(W) if W else None, P(y) if y else None, None,
+                                 P(a) if a else None, P(v) if v else None, P(q) if q else None, B, T, H, D, cin, 1,
+                                 None, dtype, P(0x10000), wsb, None)
+    assert call(cin=96) == esa.ESA_ERR_UNSUPPORTED           # input width
+    assert call(D=128) == esa.ESA_ERR_UNSUPPORTED            # head dimension above 64
+    assert call(dtype=0) == esa.ESA_ERR_UNSUPPORTED          # float32 I/O
+    assert call(W=0) == esa.ESA_ERR_ARG
+    assert call(a=0x4000) == esa.ESA_ERR_ARG                 # a without v and q
+    assert call(x=0x1008) == esa.ESA_ERR_ALIGN
+    assert call(wsb=64) == esa.ESA_ERR_WORKSPACE
+    if not __import__("torch").cuda.is_available():
+        assert call() == esa.ESA_ERR_DEVICE
+        assert call(a=0x4000, v=0x5000, q=0x6000) == esa.ESA_ERR_DEVICE
