@@ -665,6 +665,50 @@ def measure_e2e(args, world, dev, a, v, q, dy, mode, B, T, H, D):
             "h2d_GBs": h2d * K2 / (e2e_ms / 1e3) / 1e9, "d2h_GBs": d2h * K2 / (e2e_ms / 1e3) / 1e9}
 
 
+def measure_layer(dev, reps=5, seq=None):
+    """A training step of one ESA layer (forward + backward, fp16 weights and
+    activations, no bias) on the benchmark workload's shape: B = 64,
+    T = 65536, embd = 128, 4 heads, controlled.  Fused: the input
+    projections inside the scan kernel (esa_fused_fwd writing a, v, q for
+    esa_scan_bwd); unfused: linear projections + esa_scan.  W_O and the
+    projections' gradients are cuBLAS GEMMs in both."""
+    import torch
+
+    from gated_linear_recurrence_b200 import ESA
+    w = workload(seq=seq)
+    B, T, H, D = w.B, w.T, w.H, w.D
+    C = H * D
+    torch.manual_seed(w.seed + 12)
+    fused = ESA(C, H, mode="controlled", device=dev, dtype=torch.float16)
+    plain = ESA(C, H, mode="controlled", device=dev, dtype=torch.float16, fused=False)
+    plain.load_state_dict(fused.state_dict())
+    x = torch.randn(B, T, C, device=dev, dtype=torch.float16).requires_grad_(True)
+    g = torch.randn(B, T, C, device=dev, dtype=torch.float16)
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    for name, layer in (("fused", fused), ("unfused", plain)):
+        def step():
+            x.grad = None
+            layer.zero_grad(set_to_none=True)
+            layer(x).backward(g)
+        for _ in range(3):
+            step()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out[name + "_ms"] = e0.elapsed_time(e1) / reps
+        out[name + "_tokens_per_s"] = B * T / (out[name + "_ms"] / 1e3)
+    out["speedup"] = out["unfused_ms"] / out["fused_ms"]
+    out["workload"] = f"ESA layer fwd+bwd, fp16, B{B} T{T} embd{C} H{H}, controlled"
+    del fused, plain, x, g
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------------------
 # Our arm.
 # ---------------------------------------------------------------------------
@@ -758,9 +802,10 @@ def run_ours(args):
     cpar = None
     if not args.no_cp and args.batch is None and args.seq is None:
         cpar = measure_context_parallel(dev)
-    fusedm = None
+    fusedm = layerm = None
     if not args.no_fused and args.batch is None and args.seq is None:
         fusedm = measure_fused(dev)
+        layerm = measure_layer(dev)
 
     cpu = cpu_all = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -780,7 +825,7 @@ def run_ours(args):
                    "bwd_GBs": bwd_bytes / (bwd_ms / 1e3) / 1e9, "step_GBs": step_gbs,
                    "step_frac_of_measured_peak": step_gbs / peak, "step_frac_of_nominal_8TBs":
                    step_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes_per_step": fwd_bytes + bwd_bytes,
-                   "decode": decode, "context_parallel": cpar, "fused_layer_forward": fusedm, "cpu_baseline_all_cores": cpu_all},
+                   "decode": decode, "context_parallel": cpar, "fused_layer_forward": fusedm, "layer_train_step": layerm, "cpu_baseline_all_cores": cpu_all},
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": 2 * K,
@@ -806,7 +851,8 @@ def main(argv=None):
         if args.cp_only:
             print(json.dumps({"context_parallel": measure_context_parallel(dev)}), flush=True)
         else:
-            print(json.dumps({"fused_layer_forward": measure_fused(dev, seq=args.seq)}), flush=True)
+            print(json.dumps({"fused_layer_forward": measure_fused(dev, seq=args.seq),
+                              "layer_train_step": measure_layer(dev, seq=args.seq)}), flush=True)
         return 0
     return run_ours(args)
 

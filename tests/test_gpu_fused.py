@@ -146,3 +146,37 @@ def test_fused_forward_rejects_unsupported_shapes(cuda_device):
     W32 = torch.zeros(384, 128, device=cuda_device)
     with pytest.raises(esa.EsaError):
         esa.esa_fused_fwd(x32, W32, 4)                  # float32 I/O
+
+
+def _random_fused_cases(n, seed=20261203):
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    cases = []
+    while len(cases) < n:
+        D = int(rng.choice([8, 16, 32, 64]))
+        H = int(rng.integers(1, 9))
+        C_in = int(rng.choice([64, 128]))
+        B = int(rng.integers(1, 4))
+        T = int(rng.choice([1, 127, 128, 129, 255, 256, 700])) if rng.random() < 0.5 else int(rng.integers(1, 2000))
+        if B * T * H * D > 800_000:
+            continue
+        cases.append((B, T, H, D, C_in, int(rng.integers(0, 2)), str(rng.choice(["f16", "bf16"])), len(cases)))
+    return cases
+
+
+RANDOM = _random_fused_cases(12)
+
+
+@pytest.mark.parametrize("case", RANDOM, ids=[f"{c[7]}-B{c[0]}T{c[1]}H{c[2]}D{c[3]}Cin{c[4]}m{c[5]}{c[6]}" for c in RANDOM])
+def test_fused_random_shapes(cuda_device, case):
+    B, T, H, D, C_in, mode, dt, k = case
+    C = H * D
+    x, W = _inputs(B, T, C_in, C, dt, 300 + k, cuda_device)
+    E0 = inputs.make_state(B, H, D, seed=301 + k, scale=0.5).to(cuda_device) if k % 2 else None
+    y, Ef, ws, avq = esa.esa_fused_fwd(x, W, H, mode=mode, E_init=E0, want_avq=True)
+    esa.esa_check(ws)
+    _check_projections(x, W, avq, C, DT[dt])
+    y_r, Ef_r = oracle.scan_fwd(*(host64(t) for t in avq), mode, E_init=None if E0 is None else host64(E0))
+    tol = TOL[DT[dt]]
+    assert_close(y, y_r, tol, "y")
+    assert_close(Ef, Ef_r, tol, "E_final")
