@@ -60,7 +60,9 @@ class _EsaScanFn(torch.autograd.Function):
 class _FusedProjScanFn(torch.autograd.Function):
     """(x, W = [W_A; W_V; W_Q]) -> (y, E_final) through esa_fused_fwd; the
     backward is esa_scan_bwd on the projections the forward wrote, then the
-    projections' gradients dx = [da dv dq] W and dW = [da dv dq]^T x."""
+    projections' gradients dx = da W_A + dv W_V + dq W_Q and
+    dW = [da^T x; dv^T x; dq^T x] (GEMMs, no concatenated copy of the
+    gradients)."""
 
     @staticmethod
     def forward(ctx, x, W, E_init, mode, H):
@@ -87,10 +89,13 @@ class _FusedProjScanFn(torch.autograd.Function):
                                             want_dE_init=ctx.has_E_init)
         ctx.ws = None
         B, T = x.shape[:2]
-        G = torch.cat([t.reshape(B * T, -1) for t in (da, dv, dq)], dim=1)   # [B T, 3 C]
-        dx = (G @ W).reshape(x.shape)
-        dW = G.t() @ x.reshape(B * T, -1)
-        return dx, dW, (dE0 if ctx.has_E_init else None), None, None
+        C = W.shape[0] // 3
+        x2 = x.reshape(B * T, -1)
+        gs = [t.reshape(B * T, C) for t in (da, dv, dq)]
+        dx = gs[0] @ W[:C]
+        dx.addmm_(gs[1], W[C:2 * C]).addmm_(gs[2], W[2 * C:])
+        dW = torch.cat([g.t() @ x2 for g in gs], dim=0)
+        return dx.reshape(x.shape), dW, (dE0 if ctx.has_E_init else None), None, None
 
 
 def esa_scan(a, v, q, mode="controlled", E_init=None):
