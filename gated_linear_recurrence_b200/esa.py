@@ -117,6 +117,25 @@ def _stream(device, stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+class _NoDeviceSwitch:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+_SAME_DEVICE = _NoDeviceSwitch()
+
+
+def _on(device):
+    """Make `device` current for a library call; a no-op when it already is
+    (the common case, and the one on decode's latency-bound path)."""
+    if device.index is None or device.index == torch.cuda.current_device():
+        return _SAME_DEVICE
+    return torch.cuda.device(device)
+
+
 def _check_seq(name, t, ref):
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor (the ESA library has no CPU path)")
@@ -150,7 +169,7 @@ def _dims(a):
 def esa_workspace_init(workspace, stream=None):
     """Zero a workspace and write its header (once, after allocation)."""
     lib = load_library()
-    with torch.cuda.device(workspace.device):
+    with _on(workspace.device):
         rc = lib.esa_workspace_init(_ptr(workspace), workspace.numel() * workspace.element_size(),
                                     _stream(workspace.device, stream))
     if rc != 0:
@@ -189,7 +208,7 @@ def esa_scan_fwd(a, v, q, y=None, E_final=None, mode=CONTROLLED, E_init=None, wo
     if workspace is None:
         workspace = new_workspace(B, T, H, D, a.dtype, a.device)
     lib = load_library()
-    with torch.cuda.device(a.device):
+    with _on(a.device):
         rc = lib.esa_scan_fwd(_ptr(a), _ptr(v), _ptr(q), _ptr(y), _ptr(E_final), B, T, H, D, int(mode),
                               _ptr(E_init), _DTYPE_CODE[a.dtype], _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(a.device, stream))
@@ -220,7 +239,7 @@ def esa_scan_bwd(a, v, q, dy, workspace, mode=CONTROLLED, E_init=None, dE_final=
     if workspace is None or not workspace.is_cuda:
         raise ValueError("esa_scan_bwd needs the CUDA workspace written by the matching esa_scan_fwd")
     lib = load_library()
-    with torch.cuda.device(a.device):
+    with _on(a.device):
         rc = lib.esa_scan_bwd(_ptr(a), _ptr(v), _ptr(q), _ptr(dy), _ptr(dE_final), _ptr(da), _ptr(dv),
                               _ptr(dq), _ptr(dE_init), B, T, H, D, int(mode), _ptr(E_init),
                               _DTYPE_CODE[a.dtype], _ptr(workspace),
@@ -245,7 +264,7 @@ def esa_scan_map(a, v, mode=CONTROLLED, workspace=None, P=None, S=None, stream=N
     if workspace is None:
         workspace = new_workspace(B, T, H, D, a.dtype, a.device)
     lib = load_library()
-    with torch.cuda.device(a.device):
+    with _on(a.device):
         rc = lib.esa_scan_map(_ptr(a), _ptr(v), _ptr(P), _ptr(S), B, T, H, D, int(mode), _DTYPE_CODE[a.dtype],
                               _ptr(workspace), workspace.numel() * workspace.element_size(),
                               _stream(a.device, stream))
@@ -271,7 +290,7 @@ def esa_scan_bwd_map(a, v, q, dy, workspace, mode=CONTROLLED, E_init=None, P=Non
     if workspace is None or not workspace.is_cuda:
         raise ValueError("esa_scan_bwd_map needs the CUDA workspace written by the matching esa_scan_fwd")
     lib = load_library()
-    with torch.cuda.device(a.device):
+    with _on(a.device):
         rc = lib.esa_scan_bwd_map(_ptr(a), _ptr(v), _ptr(q), _ptr(dy), _ptr(P), _ptr(S), B, T, H, D, int(mode),
                                   _ptr(E_init), _DTYPE_CODE[a.dtype], _ptr(workspace),
                                   workspace.numel() * workspace.element_size(), _stream(a.device, stream))
@@ -303,7 +322,7 @@ def esa_compose(P, S, x0=None, reverse=False, out=None, stream=None):
             raise ValueError(f"{name} must be a contiguous float32 tensor of shape {shape} on {P.device}")
     out = torch.empty(shape, dtype=torch.float32, device=P.device) if out is None else out
     lib = load_library()
-    with torch.cuda.device(P.device):
+    with _on(P.device):
         rc = lib.esa_compose(_ptr(P), _ptr(S), n, count, int(bool(reverse)), _ptr(x0), _ptr(out),
                              _stream(P.device, stream))
     if rc != 0:
@@ -346,7 +365,7 @@ def esa_fused_fwd(x, W, H, mode=CONTROLLED, E_init=None, y=None, E_final=None, w
     avq = tuple(torch.empty((B, T, H, D), dtype=x.dtype, device=x.device) for _ in range(3)) if want_avq \
         else (None, None, None)
     lib = load_library()
-    with torch.cuda.device(x.device):
+    with _on(x.device):
         rc = lib.esa_fused_fwd(_ptr(x), _ptr(W), _ptr(y), _ptr(E_final), *(_ptr(t) for t in avq), B, T, H, D, C_in,
                                int(mode), _ptr(E_init),
                                _DTYPE_CODE[x.dtype], _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -372,7 +391,7 @@ def esa_step(a_t, v_t, q_t, E, y_t=None, mode=CONTROLLED, stream=None):
     if y_t is None:
         y_t = torch.empty_like(a_t)
     lib = load_library()
-    with torch.cuda.device(a_t.device):
+    with _on(a_t.device):
         rc = lib.esa_step(_ptr(a_t), _ptr(v_t), _ptr(q_t), _ptr(E), _ptr(y_t), B, H, D, int(mode),
                           _DTYPE_CODE[a_t.dtype], _stream(a_t.device, stream))
     if rc != 0:
@@ -383,7 +402,7 @@ def esa_step(a_t, v_t, q_t, E, y_t=None, mode=CONTROLLED, stream=None):
 def esa_check(workspace, stream=None):
     """Synchronise the stream and raise :class:`EsaError` if a device-side wait gave up."""
     lib = load_library()
-    with torch.cuda.device(workspace.device):
+    with _on(workspace.device):
         rc = lib.esa_check(_ptr(workspace), _stream(workspace.device, stream))
     if rc != 0:
         raise EsaError("esa_check", rc)
