@@ -21,9 +21,11 @@
 //     tensor memory, and runs its own persistent loop over tiles taken from
 //     the channel tile's ticket counter (batch row fastest), so the two
 //     groups hide each other's latencies as two CTAs per SM would.
-//   * Per tile: one thread issues C_in / 16 MMAs of 128 x 192 x 16 on the
-//     tile's x rows and commits them to an mbarrier; once they are done the
-//     x buffer is refilled with the next tile's rows; the group's 8 warps
+//   * Per tile: one thread takes the next tile's ticket (the atomic's result
+//     is used only after the read-out, so its round trip is hidden), issues
+//     C_in / 16 MMAs of 128 x 192 x 16 on the tile's x rows and commits them
+//     to an mbarrier; after the read-out the x buffer is refilled with the
+//     next tile's rows; the group's 8 warps
 //     read the accumulator (warp w: lanes 32 (w mod 4).., 96 columns) and
 //     store a, v, q; then pass 1, the run scan, the look-back and pass 2 as
 //     in the forward scan.  While the tile scans, the issuing thread checks
@@ -235,7 +237,9 @@ __global__ void __launch_bounds__(512, 1)
     const long slot_end = slot + SUB - 1;
 
     // ---- projections on the tensor cores -----------------------------------
+    unsigned nt_raw = 0;
     if (tid == 0) {
+      nt_raw = atomicAdd(&hdr->ct_ticket[ct], 1u);   // the next tile; its value is needed only after the read-out
       if (!pre) {
         if (it == 0) mbar_wait_bounded(w_bar, 0u, &hdr->status);
         mbar_wait_bounded(&bar[0], ph_x, &hdr->status);
@@ -252,13 +256,6 @@ __global__ void __launch_bounds__(512, 1)
     mbar_wait_bounded(&bar[1], ph_m, &hdr->status);
     ph_m ^= 1u;
     tc_fence_after();
-    if (tid == 0) {   // x has been consumed: the next tile's rows go in now
-      const int nt = static_cast<int>(atomicAdd(&hdr->ct_ticket[ct], 1u));
-      const TileInfo tn = decode(nt);
-      info_s[(it + 1) & 1] = tn;
-      next_ok = nt < args.ntiles_ct;
-      if (next_ok) issue_x(tn);
-    }
 
     // ---- accumulator -> a, v, q boxes (rounded to the I/O type) ------------
     __syncwarp();   // the tensor-memory loads below are warp-collective
@@ -284,6 +281,13 @@ __global__ void __launch_bounds__(512, 1)
     if (store_avq) fence_proxy_async_smem();   // box writes, before the TMA store reads them
     tc_fence_before();
     named_sync(bar_all, Pl::NTG);
+    if (tid == 0) {   // x has been consumed: the next tile's rows go in now
+      const int nt = static_cast<int>(nt_raw);
+      const TileInfo tn = decode(nt);
+      info_s[(it + 1) & 1] = tn;
+      next_ok = nt < args.ntiles_ct;
+      if (next_ok) issue_x(tn);
+    }
     // The projections themselves, when asked for: the boxes' layout is the
     // 128-byte swizzle, so one TMA store per box writes them out.
     if (store_avq && tid == 0) {
