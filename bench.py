@@ -531,11 +531,7 @@ def measure_fused(dev, reps=10, seq=None):
         esa.esa_fused_fwd(x, W, H, mode=mode, y=y, E_final=Ef, workspace=ws)
 
     def fused_avq():
-        lib = esa.load_library()
-        rc = lib.esa_fused_fwd(esa._ptr(x), esa._ptr(W), esa._ptr(y), esa._ptr(Ef), *(esa._ptr(t) for t in avq),
-                               B, T, H, D, C_in, mode, None, 1, esa._ptr(ws), ws.numel(), esa._stream(dev, None))
-        if rc != 0:
-            raise esa.EsaError("esa_fused_fwd", rc)
+        esa.esa_fused_fwd(x, W, H, mode=mode, y=y, E_final=Ef, workspace=ws, avq=avq)
 
     def unfused():
         for p in range(3):

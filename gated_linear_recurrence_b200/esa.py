@@ -331,15 +331,16 @@ def esa_compose(P, S, x0=None, reverse=False, out=None, stream=None):
 
 
 def esa_fused_fwd(x, W, H, mode=CONTROLLED, E_init=None, y=None, E_final=None, workspace=None, stream=None,
-                  want_E_final=True, want_avq=False):
+                  want_E_final=True, want_avq=False, avq=None):
     """Forward scan of the projections of ``x``: a, v, q = x W[:C]^T,
     x W[C:2C]^T, x W[2C:]^T (rounded to x's dtype), computed on the tensor
     cores inside the scan.  ``x``: [B, T, C_in] float16 / bfloat16; ``W``:
     [3C, C_in] of the same dtype; ``H`` heads of D = C / H channels.
 
     Returns ``(y, E_final, workspace)`` with ``y`` [B, T, H, D], or with
-    ``want_avq`` ``(y, E_final, workspace, (a, v, q))``: the projections the
-    scan consumed, for :func:`esa_scan_bwd`.
+    ``want_avq`` (or ``avq``, three preallocated [B, T, H, D] tensors of x's
+    dtype) ``(y, E_final, workspace, (a, v, q))``: the projections the scan
+    consumed, for :func:`esa_scan_bwd`.
     """
     if not isinstance(x, torch.Tensor) or not x.is_cuda or x.dim() != 3:
         raise TypeError("x must be a CUDA tensor [B, T, C_in] (the ESA library has no CPU path)")
@@ -362,8 +363,19 @@ def esa_fused_fwd(x, W, H, mode=CONTROLLED, E_init=None, y=None, E_final=None, w
     _check_state("E_init", E_init, B, H, D, x.device)
     if workspace is None:
         workspace = new_workspace(B, T, H, D, x.dtype, x.device)
-    avq = tuple(torch.empty((B, T, H, D), dtype=x.dtype, device=x.device) for _ in range(3)) if want_avq \
-        else (None, None, None)
+    if avq is not None:
+        want_avq = True
+        avq = tuple(avq)
+        if len(avq) != 3:
+            raise ValueError("avq must be three tensors (a, v, q)")
+        for name, t in zip(("a", "v", "q"), avq):
+            if (not isinstance(t, torch.Tensor) or tuple(t.shape) != (B, T, H, D) or t.dtype != x.dtype
+                    or t.device != x.device or not t.is_contiguous()):
+                raise ValueError(f"{name} must be a contiguous {x.dtype} tensor of shape {(B, T, H, D)} on {x.device}")
+    elif want_avq:
+        avq = tuple(torch.empty((B, T, H, D), dtype=x.dtype, device=x.device) for _ in range(3))
+    else:
+        avq = (None, None, None)
     lib = load_library()
     with _on(x.device):
         rc = lib.esa_fused_fwd(_ptr(x), _ptr(W), _ptr(y), _ptr(E_final), *(_ptr(t) for t in avq), B, T, H, D, C_in,
