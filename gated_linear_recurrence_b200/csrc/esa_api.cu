@@ -30,7 +30,7 @@ bool supported_d(int D) {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-size_t elem_bytes(int dtype) { return dtype == ESA_F32 ? 4 : 2; }
+size_t elem_bytes(int dtype) { return dtype == ESA_F32 ? 4 : dtype == ESA_E4M3 ? 1 : 2; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -52,7 +52,7 @@ constexpr size_t kHeaderBytes = 256;
 
 bool make_layout(int B, int T, int H, int D, int dtype, Layout *lo) {
   if (B < 0 || T < 0 || H < 1 || D < 1) return false;
-  if (dtype < ESA_F32 || dtype > ESA_BF16) return false;
+  if (dtype < ESA_F32 || dtype > ESA_E4M3) return false;
   if (!supported_d(D)) return false;
   const long long C = static_cast<long long>(H) * D;
   if (C > INT_MAX / 2) return false;
@@ -129,9 +129,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 int make_tmap(CUtensorMap *map, const void *ptr, int dtype, int B, int T, int C, const Layout &lo, int rows) {
   auto fn = encode_fn();
   if (fn == nullptr) return ESA_ERR_LAUNCH;
-  const CUtensorMapDataType dt = dtype == ESA_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                                 : dtype == ESA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
-                                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapDataType dt = dtype == ESA_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : dtype == ESA_F16  ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                 : dtype == ESA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                     : CU_TENSOR_MAP_DATA_TYPE_UINT8;   // e4m3 bytes
   const cuuint64_t s = elem_bytes(dtype);
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(T),
                               static_cast<cuuint64_t>(B)};
@@ -167,7 +168,7 @@ int make_tmap_sw128(CUtensorMap *map, const void *ptr, int dtype, int rank, cons
 int check_shape(int B, int T, int H, int D, int mode, int dtype) {
   if (B < 0 || T < 0 || H < 1 || D < 1) return ESA_ERR_ARG;
   if (mode != ESA_DIRECT && mode != ESA_CONTROLLED) return ESA_ERR_ARG;
-  if (dtype < ESA_F32 || dtype > ESA_BF16) return ESA_ERR_ARG;
+  if (dtype < ESA_F32 || dtype > ESA_E4M3) return ESA_ERR_ARG;
   if (!supported_d(D)) return ESA_ERR_UNSUPPORTED;
   if (static_cast<long long>(H) * D > INT_MAX / 2) return ESA_ERR_ARG;
   return ESA_OK;
@@ -246,6 +247,7 @@ int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy, co
                  const float *E_init, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
   int rc = check_shape(B, T, H, D, mode, dtype);
   if (rc) return rc;
+  if (dtype == ESA_E4M3) return ESA_ERR_UNSUPPORTED;   // fp8 inputs: forward scans only
   const bool has_tokens = B > 0 && T > 0;   // empty tensors may carry NULL pointers
   if (has_tokens && (!a || !v || !q || !dy || !da || !dv || !dq)) return ESA_ERR_ARG;
   for (const void *p : {a, v, q, dy, static_cast<const void *>(dE_final), static_cast<const void *>(da),
@@ -321,6 +323,7 @@ int esa_scan_bwd_map(const void *a, const void *v, const void *q, const void *dy
                      size_t workspace_bytes, void *stream) {
   int rc = check_shape(B, T, H, D, mode, dtype);
   if (rc) return rc;
+  if (dtype == ESA_E4M3) return ESA_ERR_UNSUPPORTED;   // fp8 inputs: forward scans only
   if (B > 0 && (!P || !S)) return ESA_ERR_ARG;
   if (B > 0 && T > 0 && (!a || !v || !q || !dy)) return ESA_ERR_ARG;
   for (const void *p : {a, v, q, dy, static_cast<const void *>(P), static_cast<const void *>(S),
@@ -421,6 +424,7 @@ int esa_step(const void *a_t, const void *v_t, const void *q_t, float *E, void *
              int mode, int dtype, void *stream) {
   int rc = check_shape(B, 1, H, D, mode, dtype);
   if (rc) return rc;
+  if (dtype == ESA_E4M3) return ESA_ERR_UNSUPPORTED;   // fp8 inputs: forward scans only
   if (B > 0 && (!a_t || !v_t || !q_t || !E || !y_t)) return ESA_ERR_ARG;
   for (const void *p : {a_t, v_t, q_t, static_cast<const void *>(E), static_cast<const void *>(y_t)})
     if (p && !aligned16(p)) return ESA_ERR_ALIGN;

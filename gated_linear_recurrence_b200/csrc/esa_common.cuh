@@ -8,6 +8,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 namespace esa {
@@ -97,6 +98,11 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __
 // ---------------------------------------------------------------------------
 template <typename T> struct Io;
 
+// The output type of a scan whose inputs are T: the input type itself, except
+// that fp8 (e4m3) inputs produce fp16 outputs.
+template <typename T> struct OutOf { using type = T; };
+template <> struct OutOf<__nv_fp8_e4m3> { using type = __half; };
+
 template <> struct Io<float> {
   static __device__ __forceinline__ void load8(const float *p, float2 (&x)[4]) {
     const float4 u = reinterpret_cast<const float4 *>(p)[0];
@@ -158,6 +164,28 @@ template <> struct Io<__nv_bfloat16> {
 #pragma unroll
     for (int i = 0; i < 4; ++i) h[i] = __float22bfloat162_rn(x[i]);
     *reinterpret_cast<uint4 *>(p) = u;
+  }
+};
+
+// fp8 e4m3 inputs (forward scans only): 8 channels = 8 bytes; each byte pair
+// is widened exactly to half precision, then to float.
+template <> struct Io<__nv_fp8_e4m3> {
+  static __device__ __forceinline__ __half2 h2(unsigned short pair) {
+    const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(pair), __NV_E4M3);
+    return __half2(r);
+  }
+  static __device__ __forceinline__ void load8(const __nv_fp8_e4m3 *p, float2 (&x)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    const unsigned short *w = reinterpret_cast<const unsigned short *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = __half22float2(h2(w[i]));
+  }
+  static __device__ __forceinline__ void load8_gate(const __nv_fp8_e4m3 *p, float2 (&x)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    const unsigned short *w = reinterpret_cast<const unsigned short *>(&u);
+    const __half2 lo = __float2half2_rn(-80.0f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = __half22float2(__hmax2(h2(w[i]), lo));
   }
 };
 

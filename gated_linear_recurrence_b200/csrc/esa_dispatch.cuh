@@ -23,13 +23,18 @@ int dispatch_d(int D, F &&f) {
   }
 }
 
-template <typename F>
+// kFp8: also dispatch fp8 (e4m3) inputs, dtype 3 (forward scans only; the
+// other kernels return ESA_ERR_UNSUPPORTED for it).
+template <bool kFp8 = false, typename F>
 int dispatch(int dtype, int mode, int D, F &&f) {
   if (mode != 0 && mode != 1) return -1;
   switch (dtype) {
     case 0: return mode ? dispatch_d<float, 1>(D, f) : dispatch_d<float, 0>(D, f);
     case 1: return mode ? dispatch_d<__half, 1>(D, f) : dispatch_d<__half, 0>(D, f);
     case 2: return mode ? dispatch_d<__nv_bfloat16, 1>(D, f) : dispatch_d<__nv_bfloat16, 0>(D, f);
+    case 3:
+      if constexpr (kFp8) return mode ? dispatch_d<__nv_fp8_e4m3, 1>(D, f) : dispatch_d<__nv_fp8_e4m3, 0>(D, f);
+      else return -3;
     default: return -1;
   }
 }

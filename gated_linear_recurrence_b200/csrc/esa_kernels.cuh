@@ -130,6 +130,10 @@ struct TileCfg {
   // NVSEG == 1.  Then a warp may overwrite its own gate rows with its run maps
   // as soon as its own lanes are done, without waiting for the CTA.
   static constexpr bool kWarpScratch = (K * sizeof(T) == 8) && NVSEG == 1;
+  // 1-byte inputs: the gate box is too small for the run-scan scratch, which
+  // gets its own region per stage (forward scans only).
+  static constexpr bool kSeparateScratch = sizeof(T) == 1;
+  static constexpr unsigned kScratchBytes = RUNS * CT * sizeof(float2);
   static_assert(L % K == 0, "K must divide L");
   static_assert(SW == 1 || SW == 2 || SW == 4 || SW == 8, "1, 2, 4 or 8 scan segments");
   static_assert(RUNS % SW == 0, "segments must split the runs evenly");
@@ -138,7 +142,7 @@ struct TileCfg {
   static_assert(NT % 32 == 0 && NT <= 1024, "bad block size");
   static_assert(RUNS % RW == 0, "runs must fill warps");
   static_assert(CT % 32 == 0 && NT >= CT, "look-back needs CT threads");
-  static_assert(RUNS * CT * sizeof(float2) <= kBoxBytes, "scan scratch must fit in the gate box");
+  static_assert(kSeparateScratch || RUNS * CT * sizeof(float2) <= kBoxBytes, "scan scratch must fit in the gate box");
   static_assert(VW % LPH == 0, "a head must stay inside a warp");
   static_assert(kBoxBytes % 128 == 0, "boxes must keep 128-byte alignment");
 };
@@ -166,7 +170,7 @@ struct MiscPlan {
 
 template <typename Cfg>
 struct FwdSmem {
-  static constexpr size_t kStage = 3 * size_t(Cfg::kBoxBytes);
+  static constexpr size_t kStage = 3 * size_t(Cfg::kBoxBytes) + (Cfg::kSeparateScratch ? Cfg::kScratchBytes : 0);
   static constexpr size_t kMisc = MiscPlan<Cfg>::kBytes;
   static constexpr size_t kBytes = 2 * kStage + kMisc + 128;   // +128 for alignment
 };
@@ -528,7 +532,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
   __syncthreads();
 
   const ThreadPos<Cfg> pos(tid);
-  T *yg = static_cast<T *>(args.y);
+  using TO = typename OutOf<T>::type;
+  TO *yg = static_cast<TO *>(args.y);
   const unsigned tag = *tag_s;
   unsigned phase = 0;   // bit s = parity of stage s
 
@@ -543,7 +548,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     const T *a_s = box(s, 0);
     const T *v_s = box(s, 1);
     const T *q_s = box(s, 2);
-    float *scan_s = reinterpret_cast<float *>(box(s, 0));   // reused once pass 1 is done
+    // Run-scan scratch: the gate box once pass 1 is done (its own region for 1-byte inputs).
+    float *scan_s = reinterpret_cast<float *>(box(s, Cfg::kSeparateScratch ? 3 : 0));
 
     // Look-back threads read the nearest predecessor's chunk-end carry now, a
     // pass ahead of the look-back: when that tile has already finished, the
@@ -677,7 +683,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
         float2 yv[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) yv[q] = mul2(qq[q], mul2(E[q], splat(rr)));
-        if (valid && ch_ok) Io<T>::store8(yg + gbase + static_cast<long>(r) * sh.C, yv);
+        if (valid && ch_ok) Io<TO>::store8(yg + gbase + static_cast<long>(r) * sh.C, yv);
       }
     }
 

@@ -20,7 +20,7 @@ constexpr int kStepsPerThread = 4;
 // two slots (128 rows) tall -- twice the time between consecutive chunks of a
 // chain, so a tile's predecessors are further ahead when it looks back.
 template <typename T, int VPR>
-constexpr int fwd_sub() { return (sizeof(T) == 2 && VPR == 8) ? 2 : 1; }
+constexpr int fwd_sub() { return (sizeof(T) <= 2 && VPR == 8) ? 2 : 1; }
 inline int fwd_slots_per_tile(int dtype, int D) { return (dtype != 0 && tile_cols(D) == 64) ? 2 : 1; }
 
 // Slots per backward tile: the same rule.  A backward tile keeps its

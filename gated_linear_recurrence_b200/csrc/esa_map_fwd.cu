@@ -6,7 +6,7 @@ namespace esa {
 
 int launch_fwd_map(int dtype, int mode, int D, const CUtensorMap &ta, const CUtensorMap &tv,
                    const CUtensorMap &tq, const FwdArgs &args, int ntiles, cudaStream_t stream) {
-  return dispatch(dtype, mode, D, FwdLauncher<true>{ta, tv, tq, args, ntiles, stream});
+  return dispatch<true>(dtype, mode, D, FwdLauncher<true>{ta, tv, tq, args, ntiles, stream});
 }
 
 }  // namespace esa

@@ -14,6 +14,9 @@ The functions carry the C names:
   maps ``(P, S)`` of a time slice (context parallelism)
 * :func:`esa_compose`   -- apply a sequence of segment maps to a state
 * :func:`esa_fused_fwd` -- forward scan with the a / v / q projections fused in
+
+Input dtypes: float32, float16, bfloat16, and float8_e4m3fn for the forward
+scans (esa_scan_fwd, esa_scan_map), whose outputs are then float16.
 * :func:`esa_check`     -- synchronise and read the device status of a workspace
 * :func:`esa_workspace_init` -- zero a new workspace and write its header
 * :func:`esa_workspace_size`, :func:`esa_strerror`, :func:`esa_version`
@@ -31,7 +34,13 @@ LIB_PATH = os.path.join(_PKG, "lib", "libesa_b200.so")
 
 DIRECT = 0
 CONTROLLED = 1
-_DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+_DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2, torch.float8_e4m3fn: 3}
+
+
+def out_dtype(dtype):
+    """The dtype of a scan's outputs for inputs of `dtype`: the same, except
+    that fp8 (e4m3) inputs give fp16 outputs (forward scans only)."""
+    return torch.float16 if dtype == torch.float8_e4m3fn else dtype
 
 ESA_OK = 0
 ESA_ERR_ARG = -1
@@ -198,9 +207,12 @@ def esa_scan_fwd(a, v, q, y=None, E_final=None, mode=CONTROLLED, E_init=None, wo
     B, T, H, D = _dims(a)
     _check_seq("v", v, a)
     _check_seq("q", q, a)
+    ydt = out_dtype(a.dtype)
     if y is None:
-        y = torch.empty_like(a)
-    _check_seq("y", y, a)
+        y = torch.empty(a.shape, dtype=ydt, device=a.device)
+    if not isinstance(y, torch.Tensor) or tuple(y.shape) != tuple(a.shape) or y.dtype != ydt \
+            or y.device != a.device or not y.is_contiguous():
+        raise ValueError(f"y must be a contiguous {ydt} tensor of shape {tuple(a.shape)} on {a.device}")
     if E_final is None and want_E_final:
         E_final = torch.empty((B, H, D), dtype=torch.float32, device=a.device)
     _check_state("E_final", E_final, B, H, D, a.device)

@@ -29,7 +29,9 @@
  *     [B, T, H, D] in the I/O dtype; state tensors (E_init, E_final, E,
  *     dE_final, dE_init) are contiguous [B, H, D] in float32.  C = H * D.
  *   - dtype is one of esa_dtype; all arithmetic and the state are float32,
- *     outputs are rounded to the I/O dtype with round-to-nearest-even.
+ *     outputs are rounded to the I/O dtype with round-to-nearest-even (fp16
+ *     for ESA_E4M3 inputs).  Calls that do not take ESA_E4M3 return
+ *     ESA_ERR_UNSUPPORTED for it.
  *   - D must be one of 8, 16, 32, 64, 128, 256; H >= 1; B >= 0; T >= 0.
  *   - stream is a cudaStream_t passed as void* (NULL = the legacy default
  *     stream).  Every call only enqueues work and returns; it does not
@@ -52,8 +54,13 @@ extern "C" {
 /* Recurrence mode ("entangled-state-attention 0.1.0", "Direct vs controlled mode"). */
 typedef enum { ESA_DIRECT = 0, ESA_CONTROLLED = 1 } esa_mode;
 
-/* I/O element type of the sequence tensors. */
-typedef enum { ESA_F32 = 0, ESA_F16 = 1, ESA_BF16 = 2 } esa_dtype;
+/* I/O element type of the sequence tensors.  ESA_E4M3: inputs a, v, q in
+ * fp8 e4m3 (1 sign, 4 exponent, 3 mantissa bits, finite, largest 448) and
+ * the output y in fp16; accepted by the forward scans only (esa_scan_fwd,
+ * esa_scan_fwd_noalloc, esa_scan_map), which are the calls of prefill and
+ * inference.  "Entangled State Attention v2.1" lists fp8 as an experimental
+ * precision mode. */
+typedef enum { ESA_F32 = 0, ESA_F16 = 1, ESA_BF16 = 2, ESA_E4M3 = 3 } esa_dtype;
 
 typedef enum {
     ESA_OK = 0,

@@ -1,0 +1,72 @@
+"""GPU parity of the fp8 (e4m3) input mode of the forward scans.
+
+a, v, q are e4m3 (torch.float8_e4m3fn); the state and the arithmetic are
+fp32 and y is fp16.  The oracle scans the same e4m3 values widened to fp64,
+so the comparison is the fp16 one (2e-3 (1 + |ref|) plus half an fp16 unit
+in the last place).  The backward, the decode step and the fused forward do
+not take fp8 inputs and must say so.
+"""
+import pytest
+import torch
+
+import oracle
+from gated_linear_recurrence_b200 import esa, inputs
+from tests._parity import TOL, assert_close, host64
+
+pytestmark = pytest.mark.gpu
+
+F8 = torch.float8_e4m3fn
+CASES = [
+    (2, 300, 4, 32, 1),
+    (3, 1000, 2, 64, 0),
+    (1, 97, 8, 8, 1),
+    (2, 257, 5, 16, 0),    # C = 80: a partial channel tile
+    (1, 129, 1, 128, 1),   # 128-channel tiles
+    (1, 200, 1, 256, 0),   # 256-channel tiles
+    (2, 4100, 4, 32, 1),
+]
+
+
+def _fp8_inputs(B, T, H, D, seed, device):
+    x = inputs.make_scan_inputs(B, T, H, D, "f32", 1.5, seed, with_dy=False)
+    return {k: x[k].to(F8).to(device) for k in ("a", "v", "q")}
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"B{c[0]}T{c[1]}H{c[2]}D{c[3]}m{c[4]}" for c in CASES])
+def test_fp8_forward_matches_oracle(cuda_device, case):
+    B, T, H, D, mode = case
+    x = _fp8_inputs(B, T, H, D, 400 + T, cuda_device)
+    E0 = inputs.make_state(B, H, D, seed=401, scale=0.5).to(cuda_device)
+    y, Ef, ws = esa.esa_scan_fwd(x["a"], x["v"], x["q"], mode=mode, E_init=E0)
+    esa.esa_check(ws)
+    assert y.dtype == torch.float16
+    f64 = lambda t: t.to(torch.float32).to("cpu", torch.float64).numpy()  # noqa: E731
+    y_r, Ef_r = oracle.scan_fwd(f64(x["a"]), f64(x["v"]), f64(x["q"]), mode, E_init=host64(E0))
+    assert_close(y, y_r, TOL[torch.float16], "y")
+    assert_close(Ef, Ef_r, TOL[torch.float16], "E_final")
+
+
+def test_fp8_segment_map_matches_oracle(cuda_device):
+    B, T, H, D = 2, 700, 4, 32
+    x = _fp8_inputs(B, T, H, D, 410, cuda_device)
+    P, S, ws = esa.esa_scan_map(x["a"], x["v"], mode=1)
+    esa.esa_check(ws)
+    f64 = lambda t: t.to(torch.float32).to("cpu", torch.float64).numpy()  # noqa: E731
+    P_r, S_r = oracle.scan_map(f64(x["a"]), f64(x["v"]), 1)
+    assert_close(P, P_r, TOL[torch.float16], "P")
+    assert_close(S, S_r, TOL[torch.float16], "S")
+
+
+def test_fp8_is_refused_outside_the_forward(cuda_device):
+    B, T, H, D = 1, 64, 2, 32
+    x = _fp8_inputs(B, T, H, D, 420, cuda_device)
+    _, _, ws = esa.esa_scan_fwd(x["a"], x["v"], x["q"], mode=1)
+    dy = torch.zeros_like(x["a"])
+    with pytest.raises(esa.EsaError) as err:
+        esa.esa_scan_bwd(x["a"], x["v"], x["q"], dy, ws, mode=1, da=torch.empty_like(x["a"]),
+                         dv=torch.empty_like(x["a"]), dq=torch.empty_like(x["a"]))
+    assert err.value.code == esa.ESA_ERR_UNSUPPORTED
+    E = torch.zeros(B, H, D, device=cuda_device)
+    with pytest.raises(esa.EsaError) as err:
+        esa.esa_step(x["a"][:, 0].contiguous(), x["v"][:, 0].contiguous(), x["q"][:, 0].contiguous(), E, mode=1)
+    assert err.value.code == esa.ESA_ERR_UNSUPPORTED
