@@ -705,6 +705,44 @@ def measure_layer(dev, reps=5, seq=None):
     return out
 
 
+def measure_fp8_forward(dev, a, v, q, mode, reps=10):
+    """The forward scan with fp8 (e4m3) inputs and fp16 output against the
+    fp16 forward, on the benchmark workload's inputs (rounded to e4m3).
+    Algorithmic bytes per element: 3 (e4m3 a, v, q) + 2 (fp16 y) = 5,
+    against 8 for fp16."""
+    import torch
+
+    from gated_linear_recurrence_b200 import esa
+    B, T, H, D = (int(x) for x in a.shape)
+    a8, v8, q8 = (t.to(torch.float8_e4m3fn) for t in (a, v, q))
+    y = torch.empty(a.shape, dtype=torch.float16, device=dev)
+    ws = esa.new_workspace(B, T, H, D, torch.float8_e4m3fn, dev)
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    for name, args in (("fp8", (a8, v8, q8)), ("fp16", (a, v, q))):
+        for _ in range(3):
+            esa.esa_scan_fwd(*args, y=y, mode=mode, workspace=ws, want_E_final=False)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            esa.esa_scan_fwd(*args, y=y, mode=mode, workspace=ws, want_E_final=False)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out[name + "_fwd_ms"] = e0.elapsed_time(e1) / reps
+    esa.esa_check(ws)
+    el = B * T * H * D
+    peak, _ = measured_peak()
+    out.update({"workload": f"{WORKLOAD_NAME} forward, a/v/q rounded to e4m3, y fp16",
+                "fp8_tokens_per_s": B * T / (out["fp8_fwd_ms"] / 1e3),
+                "fp16_tokens_per_s": B * T / (out["fp16_fwd_ms"] / 1e3),
+                "fp8_algorithmic_bytes": 5 * el, "fp8_GBs": 5 * el / (out["fp8_fwd_ms"] / 1e3) / 1e9,
+                "fp8_frac_of_measured_hbm": 5 * el / (out["fp8_fwd_ms"] / 1e3) / 1e9 / peak})
+    del a8, v8, q8, y, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------------------
 # Our arm.
 # ---------------------------------------------------------------------------
@@ -798,10 +836,11 @@ def run_ours(args):
     cpar = None
     if not args.no_cp and args.batch is None and args.seq is None:
         cpar = measure_context_parallel(dev)
-    fusedm = layerm = None
+    fusedm = layerm = fp8m = None
     if not args.no_fused and args.batch is None and args.seq is None:
         fusedm = measure_fused(dev)
         layerm = measure_layer(dev)
+        fp8m = measure_fp8_forward(dev, a, v, q, mode)
 
     cpu = cpu_all = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -821,7 +860,8 @@ def run_ours(args):
                    "bwd_GBs": bwd_bytes / (bwd_ms / 1e3) / 1e9, "step_GBs": step_gbs,
                    "step_frac_of_measured_peak": step_gbs / peak, "step_frac_of_nominal_8TBs":
                    step_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes_per_step": fwd_bytes + bwd_bytes,
-                   "decode": decode, "context_parallel": cpar, "fused_layer_forward": fusedm, "layer_train_step": layerm, "cpu_baseline_all_cores": cpu_all},
+                   "decode": decode, "context_parallel": cpar, "fused_layer_forward": fusedm, "layer_train_step": layerm,
+                   "fp8_forward": fp8m, "cpu_baseline_all_cores": cpu_all},
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": 2 * K,

@@ -599,7 +599,14 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
       }
     }
     // The gate rows are free from here on (only this warp read its own rows).
-    if constexpr (Cfg::kWarpScratch) __syncwarp(); else __syncthreads();
+    // A separate scratch region needs no wait: its last readers (pass 2 of
+    // this stage's previous tile) finished before the stage was refilled.
+    if constexpr (Cfg::kSeparateScratch) {
+    } else if constexpr (Cfg::kWarpScratch) {
+      __syncwarp();
+    } else {
+      __syncthreads();
+    }
     scan_store8<CT>(scan_s, pos.run, pos.ch, P, S);
     __syncthreads();
 
