@@ -62,6 +62,9 @@ def parse_args(argv=None):
                     help="skip the fused projection + scan forward timing reported under detail.fused_layer_forward")
     ap.add_argument("--fused-only", action="store_true",
                     help="run only the fused projection + scan forward timing (one JSON line; for profiling)")
+    ap.add_argument("--context-parallel", action="store_true",
+                    help="split each sequence of the workload along time over the ranks (NCCL all-gather of the "
+                         "segment maps) instead of giving every rank its own batch: strong scaling")
     ap.add_argument("--cp-only", action="store_true",
                     help="run only the context-parallel phase timing (one JSON line; for profiling its kernels)")
     ap.add_argument("--batch", type=int, default=None,
@@ -747,6 +750,72 @@ def measure_fp8_forward(dev, a, v, q, mode, reps=10):
 # Our arm.
 # ---------------------------------------------------------------------------
 
+def run_context_parallel(args):
+    """The workload's sequences split along time over the ranks: rank r holds
+    steps [r T / N, (r + 1) T / N) of every sequence and runs
+    cp_scan_fwd + cp_scan_bwd (segment maps, one NCCL all-gather each way,
+    compositions, scans).  Total work is fixed as N grows (strong scaling);
+    value = B T / the slowest rank's device time per step."""
+    import torch
+    import torch.distributed as dist
+
+    from gated_linear_recurrence_b200 import context_parallel as cp
+    from gated_linear_recurrence_b200 import esa, inputs
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if not dist.is_initialized():
+        if "MASTER_ADDR" in os.environ:
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+        else:   # one process without a launcher
+            dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1, device_id=dev)
+    w = workload(args.batch, args.seq)
+    B, T, H, D, mode = w.B, w.T, w.H, w.D, w.mode
+    if T % world:
+        raise SystemExit(f"T={T} is not divisible by {world} ranks")
+    Tr = T // world
+    x = inputs.make_scan_inputs(B, Tr, H, D, w.dtype, w.a_mean, rank_seed(w, rank), device=dev)
+    a, v, q, dy = x["a"], x["v"], x["q"], x["dy"]
+    stream = torch.cuda.current_stream(dev)
+    ws0 = esa.new_workspace(B, Tr, H, D, a.dtype, dev)
+
+    def step():
+        y, Ef, E_in, ws = cp.cp_scan_fwd(a, v, q, mode, workspace=ws0)
+        cp.cp_scan_bwd(a, v, q, dy, ws, E_in, mode, dE_final=None)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local).start()
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    elapsed_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    line = {
+        "metric": METRIC, "value": B * T * args.steps / (elapsed_ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(config_dict(w), parallelism=f"context-parallel over {world} ranks, T/rank={Tr}"),
+        "clocks": clk, "gpu_launches": 11 * args.steps,
+        "note": "per step and rank: esa_scan_map (2 launches), 2 esa_compose, esa_scan_fwd, esa_scan_bwd_map "
+                "(2), 1 esa_compose, esa_scan_bwd, plus two NCCL all-gathers"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.destroy_process_group()
+    return 0
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -880,6 +949,8 @@ def main(argv=None):
         raise SystemExit("--warmup must be at least 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.context_parallel:
+        return run_context_parallel(args)
     if args.cp_only or args.fused_only:
         import torch
         dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))

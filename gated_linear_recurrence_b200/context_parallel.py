@@ -105,16 +105,17 @@ def boundary_grad(P_all, S_all, rank, dE_final=None, ops=LibraryOps):
     return ops.compose(P_all[rank + 1:], S_all[rank + 1:], dE_final, True)
 
 
-def cp_scan_fwd(a, v, q, mode=_esa.CONTROLLED, E_init=None, group=None, ops=LibraryOps):
+def cp_scan_fwd(a, v, q, mode=_esa.CONTROLLED, E_init=None, group=None, ops=LibraryOps, workspace=None):
     """Forward scan of this rank's slice.  ``E_init`` is the state before the
-    first slice (the same on every rank, or None).
+    first slice (the same on every rank, or None); ``workspace`` is reused
+    when given (allocated otherwise).
 
     Returns ``(y, E_final, E_in, workspace)``: this slice's readout, the state
     after the last slice, the state entering this slice and the workspace
     (keep both for :func:`cp_scan_bwd`).
     """
     rank = dist.get_rank(group)
-    P, S, ws = forward_map(a, v, mode, None, ops)
+    P, S, ws = forward_map(a, v, mode, workspace, ops)
     maps = gather_stacked(torch.stack([P, S]), group)
     E_in, E_final = boundary_state(maps[:, 0], maps[:, 1], rank, E_init, ops)
     y, ws = ops.scan_fwd(a, v, q, mode, E_in, ws)
