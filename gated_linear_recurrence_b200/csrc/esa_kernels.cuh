@@ -32,6 +32,13 @@
 //   * The forward stores the state at every chunk end (incl_f); the backward
 //     replays each chunk from that checkpoint, so nothing of size T x C is
 //     stored besides the outputs.
+//   * Map mode (template flag MAP, for splitting a sequence along time over
+//     several GPUs): the same tiles, gates and run scans, but each tile only
+//     publishes its own (reverse) map at its first slot and skips the
+//     look-back, checkpoints, readout and outputs; a fold kernel then
+//     composes a chain's tile maps into the map of the whole slice.
+//   * fp8 (e4m3) inputs (forward only): 1-byte boxes are too small for the
+//     run-scan scratch, which gets its own region per stage.
 #pragma once
 
 #include "esa_common.cuh"
@@ -858,7 +865,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     scan_store8<CT>(scan_s, pos.run, pos.ch, P, S);
     __syncthreads();
     // The checkpoint carry goes in only now: every warp has left the previous
-    // tile (whose B1 read the array) by the barrier above.
+    // tile (whose B phase read the array) by the barrier above.
     if (tid < CT) es_s[tid] = E_ck;
     // Scan lanes: lane c2 of segment group g; the last group publishes.
     const int c2 = tid % NP, g = tid / NP;
@@ -984,7 +991,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     }
 
     // Ticket of the tile after next, taken once the look-back is resolved (as
-    // in the forward): B1 and B2 hide its round trip.
+    // in the forward): the B phase hides its round trip.
     if (tid == 0) next = atomicAdd(&hdr->ticket[1], 1u);
 
     // ---- B: total gradient G_t (latest step first): dv and
