@@ -16,9 +16,10 @@ inline int tile_rows(int dtype) { return dtype == 0 ? 32 : 64; }   // f32 : 16-b
 inline int tile_cols(int D) { return D <= 64 ? 64 : D; }
 constexpr int kStepsPerThread = 4;
 
-// Slots per forward tile: 64-channel tiles of 16-bit data run the forward
-// two slots (128 rows) tall -- twice the time between consecutive chunks of a
-// chain, so a tile's predecessors are further ahead when it looks back.
+// Slots per forward tile: 64-channel tiles of 16-bit (and 8-bit) data run the
+// forward two slots (128 rows) tall -- twice the time between consecutive
+// chunks of a chain, so a tile's predecessors are further ahead when it looks
+// back.
 template <typename T, int VPR>
 constexpr int fwd_sub() { return (sizeof(T) <= 2 && VPR == 8) ? 2 : 1; }
 inline int fwd_slots_per_tile(int dtype, int D) { return (dtype != 0 && tile_cols(D) == 64) ? 2 : 1; }
