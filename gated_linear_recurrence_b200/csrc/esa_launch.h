@@ -12,7 +12,7 @@ namespace esa {
 // Rows per workspace slot (the backward's tile height) and channels per tile,
 // as chosen for each I/O dtype and head dimension.  The workspace layout and
 // the kernels both follow these.
-inline int tile_rows(int dtype) { return dtype == 0 ? 32 : 64; }   // f32 : 16-bit
+inline int tile_rows(int dtype) { return dtype == 0 ? 32 : 64; }   // f32 : 16- and 8-bit
 inline int tile_cols(int D) { return D <= 64 ? 64 : D; }
 constexpr int kStepsPerThread = 4;
 
