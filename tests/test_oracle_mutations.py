@@ -64,3 +64,80 @@ def test_pins_catch_mutant(tmp_path, name, old, new, which):
                           os.path.join(ROOT, "tests", "test_oracle_pins.py")],
                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert res.returncode != 0, f"mutant {name} survived the pins:\n{res.stdout[-2000:]}"
+
+
+# ---------------------------------------------------------------------------
+# The Python-level oracle functions (segment maps, composition, projections,
+# I/O rounding): each mutant replaces one function with a plausible mistake
+# and one of the pins in tests/test_oracle_pins.py must fail.
+# ---------------------------------------------------------------------------
+
+def _mut_compose_reversed(orig):
+    return lambda P, S, x0=None, reverse=False: orig(P, S, x0, not reverse)
+
+
+def _mut_compose_swapped(orig):
+    import numpy as np
+
+    def f(P, S, x0=None, reverse=False):
+        P = np.asarray(P, dtype=np.float64)
+        S = np.asarray(S, dtype=np.float64)
+        x = np.zeros(P.shape[1:]) if x0 is None else np.array(x0, dtype=np.float64)
+        for j in (range(P.shape[0] - 1, -1, -1) if reverse else range(P.shape[0])):
+            x = S[j] * x + P[j]
+        return x
+    return f
+
+
+def _mut_project_order(orig):
+    def f(x, W, io_dtype):
+        a, v, q = orig(x, W, io_dtype)
+        return v, a, q
+    return f
+
+
+def _mut_round_bf16_truncates(orig):
+    import numpy as np
+
+    def f(x, io_dtype):
+        if io_dtype != "bf16":
+            return orig(x, io_dtype)
+        u = np.ascontiguousarray(np.asarray(x, dtype=np.float64).astype(np.float32)).view(np.uint32)
+        return (u >> 16 << 16).astype(np.uint32).view(np.float32).astype(np.float64)
+    return f
+
+
+def _mut_scan_map_short_product(orig):
+    import numpy as np
+
+    def f(a, v, mode):
+        P, S = orig(a, v, mode)
+        a = np.asarray(a, dtype=np.float64)
+        return np.prod(1.0 / (1.0 + np.exp(-a[:, :-1])), axis=1), S
+    return f
+
+
+def _mut_bwd_map_ignores_E_init(orig):
+    return lambda a, v, q, dy, mode, E_init=None: orig(a, v, q, dy, mode, E_init=None)
+
+
+PY_MUTANTS = [
+    ("compose_order_reversed", "compose", _mut_compose_reversed, "test_compose_order_small_example", ()),
+    ("compose_P_S_swapped", "compose", _mut_compose_swapped, "test_compose_order_small_example", ()),
+    ("project_order_swapped", "project", _mut_project_order, "test_project_hand_example", ()),
+    ("round_bf16_truncates", "round_io", _mut_round_bf16_truncates, "test_round_io_matches_torch_conversions", ()),
+    ("scan_map_drops_last_gate", "scan_map", _mut_scan_map_short_product,
+     "test_scan_map_is_the_affine_map_of_the_slice", (1,)),
+    ("bwd_map_ignores_E_init", "scan_bwd_map", _mut_bwd_map_ignores_E_init,
+     "test_scan_bwd_map_is_the_affine_map_of_the_slice", (1,)),
+]
+
+
+@pytest.mark.parametrize("name,fn,make,pin,args", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_pins_catch_python_mutant(monkeypatch, name, fn, make, pin, args):
+    import oracle
+    from tests import test_oracle_pins as pins
+    getattr(pins, pin)(*args)                       # the pin passes on the real oracle
+    monkeypatch.setattr(oracle, fn, make(getattr(oracle, fn)))
+    with pytest.raises(AssertionError):
+        getattr(pins, pin)(*args)
