@@ -247,7 +247,6 @@ int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy, co
                  const float *E_init, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
   int rc = check_shape(B, T, H, D, mode, dtype);
   if (rc) return rc;
-  if (dtype == ESA_E4M3) return ESA_ERR_UNSUPPORTED;   // fp8 inputs: forward scans only
   const bool has_tokens = B > 0 && T > 0;   // empty tensors may carry NULL pointers
   if (has_tokens && (!a || !v || !q || !dy || !da || !dv || !dq)) return ESA_ERR_ARG;
   for (const void *p : {a, v, q, dy, static_cast<const void *>(dE_final), static_cast<const void *>(da),
@@ -323,7 +322,6 @@ int esa_scan_bwd_map(const void *a, const void *v, const void *q, const void *dy
                      size_t workspace_bytes, void *stream) {
   int rc = check_shape(B, T, H, D, mode, dtype);
   if (rc) return rc;
-  if (dtype == ESA_E4M3) return ESA_ERR_UNSUPPORTED;   // fp8 inputs: forward scans only
   if (B > 0 && (!P || !S)) return ESA_ERR_ARG;
   if (B > 0 && T > 0 && (!a || !v || !q || !dy)) return ESA_ERR_ARG;
   for (const void *p : {a, v, q, dy, static_cast<const void *>(P), static_cast<const void *>(S),

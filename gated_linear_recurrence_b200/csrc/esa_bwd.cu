@@ -6,7 +6,7 @@ namespace esa {
 int launch_bwd(int dtype, int mode, int D, const CUtensorMap &ta, const CUtensorMap &tv,
                const CUtensorMap &tq, const CUtensorMap &tdy, const BwdArgs &args, int ntiles,
                cudaStream_t stream) {
-  return dispatch(dtype, mode, D, BwdLauncher<false>{ta, tv, tq, tdy, args, ntiles, stream});
+  return dispatch<true>(dtype, mode, D, BwdLauncher<false>{ta, tv, tq, tdy, args, ntiles, stream});
 }
 
 }  // namespace esa

@@ -187,8 +187,12 @@ template <typename Cfg>
 struct BwdSmem {
   static constexpr size_t kStage = 2 * size_t(Cfg::kBoxBytes);
   static constexpr size_t kQdy = 2 * size_t(Cfg::kBoxBytes);
+  // 1-byte inputs: the run-scan scratch and ghat (8 float32 per thread and
+  // row) do not fit in the boxes; each gets one region of its own.
+  static constexpr size_t kScratch = Cfg::kSeparateScratch ? size_t(Cfg::kScratchBytes) : 0;
+  static constexpr size_t kGhat = Cfg::kSeparateScratch ? size_t(Cfg::L) * Cfg::CT * sizeof(float) : 0;
   static constexpr size_t kMisc = MiscPlan<Cfg>::kBytes;
-  static constexpr size_t kBytes = 2 * kStage + kQdy + kMisc + 128;
+  static constexpr size_t kBytes = 2 * kStage + kQdy + kScratch + kGhat + kMisc + 128;
 };
 
 // The first 128-byte-aligned byte of the dynamic shared memory.  The offset
@@ -756,7 +760,9 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
   unsigned char *base = smem_aligned128(smem_raw);
   T *q_s = reinterpret_cast<T *>(base + 2 * Sm::kStage);
   T *dy_s = q_s + L * CT;
-  unsigned char *misc_p = base + 2 * Sm::kStage + Sm::kQdy;
+  float *xscratch = reinterpret_cast<float *>(base + 2 * Sm::kStage + Sm::kQdy);             // 1-byte inputs only
+  float *gh_s = reinterpret_cast<float *>(base + 2 * Sm::kStage + Sm::kQdy + Sm::kScratch);  // 1-byte inputs only
+  unsigned char *misc_p = base + 2 * Sm::kStage + Sm::kQdy + Sm::kScratch + Sm::kGhat;
   float *es_s = reinterpret_cast<float *>(misc_p);
   float4 *seg_s = reinterpret_cast<float4 *>(misc_p + Mp::kSeg);
   uint64_t *bar = reinterpret_cast<uint64_t *>(misc_p + Mp::kBars);     // [0..1] a/v stages, [2] q/dy
@@ -810,9 +816,15 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
   __syncthreads();
 
   const ThreadPos<Cfg> pos(tid);
-  T *dag = static_cast<T *>(args.da);
-  T *dvg = static_cast<T *>(args.dv);
-  T *dqg = static_cast<T *>(args.dq);
+  // ghat of row r of this thread: in its q / dy slots, or (1-byte inputs) its own region.
+  auto get_ghat_any = [&](int r, float2 (&g)[4]) {
+    if constexpr (Cfg::kSeparateScratch) get_ghat<float>(gh_s + r * CT + pos.ch, nullptr, g);
+    else get_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, g);
+  };
+  using TO = typename OutOf<T>::type;
+  TO *dag = static_cast<TO *>(args.da);
+  TO *dvg = static_cast<TO *>(args.dv);
+  TO *dqg = static_cast<TO *>(args.dq);
   const unsigned tag = *tag_s;
   unsigned phase = 0;   // bits 0..1: a/v stages, bit 2: q/dy
 
@@ -825,7 +837,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     const long slot = ti.slot;
     const T *a_s = box(s, 0);
     const T *v_s = box(s, 1);
-    float *scan_s = reinterpret_cast<float *>(box(s, 0));
+    float *scan_s = Cfg::kSeparateScratch ? xscratch : reinterpret_cast<float *>(box(s, 0));
 
     float E_ck = 0.0f;   // forward state entering the chunk, channel tid (checkpoint)
     if (tid < CT) {
@@ -916,9 +928,10 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
         float2 gh[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) gh[q] = mul2(splat(rr), fma2(nn[q], splat(-dot), dn[q]));
-        put_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
+        if constexpr (Cfg::kSeparateScratch) put_ghat<float>(gh_s + r * CT + pos.ch, nullptr, gh);
+        else put_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
         if (!MAP && valid && (c0 + pos.ch) < sh.C)
-          Io<T>::store8(dqg + (static_cast<long>(b) * sh.T + t0 + r) * sh.C + c0 + pos.ch, dqv);
+          Io<TO>::store8(dqg + (static_cast<long>(b) * sh.T + t0 + r) * sh.C + c0 + pos.ch, dqv);
       }
     }
 
@@ -940,7 +953,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
         const int r = pos.row0 + i;
         if ((t0 + r) < sh.T) {
           float2 gh[4];
-          get_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
+          get_ghat_any(r, gh);
 #pragma unroll
           for (int q = 0; q < 4; ++q) hl[q] = mul2(gate_A<MODE>(Ar[i][q]), add2(gh[q], hl[q]));
         }
@@ -1006,7 +1019,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
         const int r = pos.row0 + i;
         if ((t0 + r) < sh.T) {
           float2 gh[4], dvv[4], dav[4];
-          get_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
+          get_ghat_any(r, gh);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const float2 G = add2(gh[q], h[q]);
@@ -1017,8 +1030,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
             h[q] = mul2(A, G);
           }
           if (ch_ok) {
-            Io<T>::store8(dvg + gbase + static_cast<long>(r) * sh.C, dvv);
-            Io<T>::store8(dag + gbase + static_cast<long>(r) * sh.C, dav);
+            Io<TO>::store8(dvg + gbase + static_cast<long>(r) * sh.C, dvv);
+            Io<TO>::store8(dag + gbase + static_cast<long>(r) * sh.C, dav);
           }
         }
       }

@@ -7,7 +7,7 @@ namespace esa {
 int launch_bwd_map(int dtype, int mode, int D, const CUtensorMap &ta, const CUtensorMap &tv,
                    const CUtensorMap &tq, const CUtensorMap &tdy, const BwdArgs &args, int ntiles,
                    cudaStream_t stream) {
-  return dispatch(dtype, mode, D, BwdLauncher<true>{ta, tv, tq, tdy, args, ntiles, stream});
+  return dispatch<true>(dtype, mode, D, BwdLauncher<true>{ta, tv, tq, tdy, args, ntiles, stream});
 }
 
 }  // namespace esa

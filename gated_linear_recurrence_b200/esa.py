@@ -15,8 +15,10 @@ The functions carry the C names:
 * :func:`esa_compose`   -- apply a sequence of segment maps to a state
 * :func:`esa_fused_fwd` -- forward scan with the a / v / q projections fused in
 
-Input dtypes: float32, float16, bfloat16, and float8_e4m3fn for the forward
-scans (esa_scan_fwd, esa_scan_map), whose outputs are then float16.
+Input dtypes: float32, float16, bfloat16, and float8_e4m3fn for the scans
+(esa_scan_fwd, esa_scan_bwd, esa_scan_map, esa_scan_bwd_map), whose outputs
+are then float16; the decode step and the fused forward take 16-bit or
+float32 inputs.
 * :func:`esa_check`     -- synchronise and read the device status of a workspace
 * :func:`esa_workspace_init` -- zero a new workspace and write its header
 * :func:`esa_workspace_size`, :func:`esa_strerror`, :func:`esa_version`
@@ -39,7 +41,7 @@ _DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2, torch.floa
 
 def out_dtype(dtype):
     """The dtype of a scan's outputs for inputs of `dtype`: the same, except
-    that fp8 (e4m3) inputs give fp16 outputs (forward scans only)."""
+    that fp8 (e4m3) inputs give fp16 outputs."""
     return torch.float16 if dtype == torch.float8_e4m3fn else dtype
 
 ESA_OK = 0
@@ -238,11 +240,14 @@ def esa_scan_bwd(a, v, q, dy, workspace, mode=CONTROLLED, E_init=None, dE_final=
     B, T, H, D = _dims(a)
     for name, t in (("v", v), ("q", q), ("dy", dy)):
         _check_seq(name, t, a)
-    da = torch.empty_like(a) if da is None else da
-    dv = torch.empty_like(a) if dv is None else dv
-    dq = torch.empty_like(a) if dq is None else dq
+    odt = out_dtype(a.dtype)
+    da = torch.empty(a.shape, dtype=odt, device=a.device) if da is None else da
+    dv = torch.empty(a.shape, dtype=odt, device=a.device) if dv is None else dv
+    dq = torch.empty(a.shape, dtype=odt, device=a.device) if dq is None else dq
     for name, t in (("da", da), ("dv", dv), ("dq", dq)):
-        _check_seq(name, t, a)
+        if not isinstance(t, torch.Tensor) or tuple(t.shape) != tuple(a.shape) or t.dtype != odt \
+                or t.device != a.device or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {odt} tensor of shape {tuple(a.shape)} on {a.device}")
     if dE_init is None and want_dE_init:
         dE_init = torch.empty((B, H, D), dtype=torch.float32, device=a.device)
     _check_state("dE_init", dE_init, B, H, D, a.device)

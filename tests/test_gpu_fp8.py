@@ -3,8 +3,9 @@
 a, v, q are e4m3 (torch.float8_e4m3fn); the state and the arithmetic are
 fp32 and y is fp16.  The oracle scans the same e4m3 values widened to fp64,
 so the comparison is the fp16 one (2e-3 (1 + |ref|) plus half an fp16 unit
-in the last place).  The backward, the decode step and the fused forward do
-not take fp8 inputs and must say so.
+in the last place).  The backward takes e4m3 dy too and returns fp16 gradients;
+the decode step and the fused forward do not take fp8 inputs and must say
+so.
 """
 import pytest
 import torch
@@ -57,16 +58,35 @@ def test_fp8_segment_map_matches_oracle(cuda_device):
     assert_close(S, S_r, TOL[torch.float16], "S")
 
 
-def test_fp8_is_refused_outside_the_forward(cuda_device):
+@pytest.mark.parametrize("case", CASES, ids=[f"B{c[0]}T{c[1]}H{c[2]}D{c[3]}m{c[4]}" for c in CASES])
+def test_fp8_backward_matches_oracle(cuda_device, case):
+    """e4m3 a, v, q and upstream gradient dy; fp16 gradients."""
+    B, T, H, D, mode = case
+    x = inputs.make_scan_inputs(B, T, H, D, "f32", 1.5, 430 + T)
+    xd = {k: x[k].to(F8).to(cuda_device) for k in ("a", "v", "q", "dy")}
+    E0 = inputs.make_state(B, H, D, seed=431, scale=0.5).to(cuda_device)
+    dEf = inputs.make_state(B, H, D, seed=432).to(cuda_device)
+    _, _, ws = esa.esa_scan_fwd(xd["a"], xd["v"], xd["q"], mode=mode, E_init=E0)
+    da, dv, dq, dE0 = esa.esa_scan_bwd(xd["a"], xd["v"], xd["q"], xd["dy"], ws, mode=mode, E_init=E0,
+                                       dE_final=dEf)
+    esa.esa_check(ws)
+    assert da.dtype == dv.dtype == dq.dtype == torch.float16
+    f64 = lambda t: t.to(torch.float32).to("cpu", torch.float64).numpy()  # noqa: E731
+    ref = oracle.scan_bwd(*(f64(xd[k]) for k in ("a", "v", "q", "dy")), mode, E_init=host64(E0),
+                          dE_final=host64(dEf))
+    for name, g, r in zip(("da", "dv", "dq", "dE_init"), (da, dv, dq, dE0), ref):
+        assert_close(g, r, TOL[torch.float16], name)
+
+
+def test_fp8_is_refused_by_the_step_and_the_fused_forward(cuda_device):
     B, T, H, D = 1, 64, 2, 32
     x = _fp8_inputs(B, T, H, D, 420, cuda_device)
-    _, _, ws = esa.esa_scan_fwd(x["a"], x["v"], x["q"], mode=1)
-    dy = torch.zeros_like(x["a"])
-    with pytest.raises(esa.EsaError) as err:
-        esa.esa_scan_bwd(x["a"], x["v"], x["q"], dy, ws, mode=1, da=torch.empty_like(x["a"]),
-                         dv=torch.empty_like(x["a"]), dq=torch.empty_like(x["a"]))
-    assert err.value.code == esa.ESA_ERR_UNSUPPORTED
     E = torch.zeros(B, H, D, device=cuda_device)
     with pytest.raises(esa.EsaError) as err:
         esa.esa_step(x["a"][:, 0].contiguous(), x["v"][:, 0].contiguous(), x["q"][:, 0].contiguous(), E, mode=1)
+    assert err.value.code == esa.ESA_ERR_UNSUPPORTED
+    xin = torch.zeros(B, T, 128, device=cuda_device).to(F8)
+    W = torch.zeros(3 * H * D, 128, device=cuda_device).to(F8)
+    with pytest.raises(esa.EsaError) as err:
+        esa.esa_fused_fwd(xin, W, H)
     assert err.value.code == esa.ESA_ERR_UNSUPPORTED
