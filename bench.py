@@ -708,17 +708,19 @@ def measure_layer(dev, reps=5, seq=None):
     return out
 
 
-def measure_fp8_forward(dev, a, v, q, mode, reps=10):
-    """The forward scan with fp8 (e4m3) inputs and fp16 output against the
-    fp16 forward, on the benchmark workload's inputs (rounded to e4m3).
-    Algorithmic bytes per element: 3 (e4m3 a, v, q) + 2 (fp16 y) = 5,
-    against 8 for fp16."""
+def measure_fp8_forward(dev, a, v, q, mode, reps=10, dy=None):
+    """The scans with fp8 (e4m3) inputs and fp16 outputs against fp16, on the
+    benchmark workload's inputs (rounded to e4m3).  Algorithmic bytes per
+    element: forward 3 (e4m3 a, v, q) + 2 (fp16 y) = 5, against 8 for fp16;
+    backward 4 (e4m3 a, v, q, dy) + 6 (fp16 da, dv, dq) = 10, against 14."""
     import torch
 
     from gated_linear_recurrence_b200 import esa
     B, T, H, D = (int(x) for x in a.shape)
     a8, v8, q8 = (t.to(torch.float8_e4m3fn) for t in (a, v, q))
+    dy8 = None if dy is None else dy.to(torch.float8_e4m3fn)
     y = torch.empty(a.shape, dtype=torch.float16, device=dev)
+    grads = [torch.empty(a.shape, dtype=torch.float16, device=dev) for _ in range(3)]
     ws = esa.new_workspace(B, T, H, D, torch.float8_e4m3fn, dev)
     stream = torch.cuda.current_stream(dev)
     out = {}
@@ -733,15 +735,32 @@ def measure_fp8_forward(dev, a, v, q, mode, reps=10):
         e1.record(stream)
         torch.cuda.synchronize()
         out[name + "_fwd_ms"] = e0.elapsed_time(e1) / reps
+        if dy is not None:   # backward on the same workspace (the forward just wrote its chunk states)
+            dyx = dy8 if name == "fp8" else dy
+            e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            tot = 0.0
+            for k in range(reps + 2):
+                esa.esa_scan_fwd(*args, y=y, mode=mode, workspace=ws, want_E_final=False)
+                e2.record(stream)
+                esa.esa_scan_bwd(*args, dyx, ws, mode=mode, da=grads[0], dv=grads[1], dq=grads[2],
+                                 want_dE_init=False)
+                e3.record(stream)
+                torch.cuda.synchronize()
+                if k >= 2:
+                    tot += e2.elapsed_time(e3)
+            out[name + "_bwd_ms"] = tot / reps
     esa.esa_check(ws)
     el = B * T * H * D
     peak, _ = measured_peak()
-    out.update({"workload": f"{WORKLOAD_NAME} forward, a/v/q rounded to e4m3, y fp16",
+    if dy is not None:
+        out["fp8_bwd_GBs"] = 10 * el / (out["fp8_bwd_ms"] / 1e3) / 1e9
+        out["fp8_fwd_bwd_tokens_per_s"] = B * T / ((out["fp8_fwd_ms"] + out["fp8_bwd_ms"]) / 1e3)
+    out.update({"workload": f"{WORKLOAD_NAME}, a/v/q/dy rounded to e4m3, outputs fp16",
                 "fp8_tokens_per_s": B * T / (out["fp8_fwd_ms"] / 1e3),
                 "fp16_tokens_per_s": B * T / (out["fp16_fwd_ms"] / 1e3),
                 "fp8_algorithmic_bytes": 5 * el, "fp8_GBs": 5 * el / (out["fp8_fwd_ms"] / 1e3) / 1e9,
                 "fp8_frac_of_measured_hbm": 5 * el / (out["fp8_fwd_ms"] / 1e3) / 1e9 / peak})
-    del a8, v8, q8, y, ws
+    del a8, v8, q8, dy8, y, ws, grads
     torch.cuda.empty_cache()
     return out
 
@@ -909,7 +928,7 @@ def run_ours(args):
     if not args.no_fused and args.batch is None and args.seq is None:
         fusedm = measure_fused(dev)
         layerm = measure_layer(dev)
-        fp8m = measure_fp8_forward(dev, a, v, q, mode)
+        fp8m = measure_fp8_forward(dev, a, v, q, mode, dy=dy)
 
     cpu = cpu_all = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
