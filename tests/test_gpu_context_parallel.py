@@ -11,7 +11,6 @@
   whole sequence.
 * The ESA layer with a one-rank NCCL group against the layer without one.
 """
-import numpy as np
 import pytest
 import torch
 
