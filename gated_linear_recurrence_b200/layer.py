@@ -204,3 +204,18 @@ class ESA(torch.nn.Module):
         """A zero state ``[batch, head, head_dim]`` (float32)."""
         return torch.zeros(batch, self.head, self.head_dim, dtype=torch.float32,
                            device=device if device is not None else self.W_A.weight.device)
+
+    # The generation interface of the pages (mlbricks-web.pages.dev/esa, Quick
+    # start: prefill returns the output and the state, decode_step advances
+    # one token), on the layer's input and output.
+    @torch.no_grad()
+    def prefill(self, x, state=None):
+        """``(out, state)`` after the whole prompt ``x`` [B, T, embd]."""
+        out, E = self.forward(x, state=state, return_state=True)
+        return out, E
+
+    @torch.no_grad()
+    def decode_step(self, x_t, state):
+        """``(out_t, state)`` for one token ``x_t`` [B, embd]; ``state`` is
+        updated in place and returned."""
+        return self.step(x_t, state), state

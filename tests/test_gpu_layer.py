@@ -144,3 +144,22 @@ def test_fused_layer_inference_matches_reference(cuda_device):
     ref = _reference_layer(x.cpu().double(), W["W_A"], W["W_V"], W["W_Q"], W["W_O"], H, "controlled")
     scale = float(ref.abs().max())
     assert_close(out.float() / scale, ref.numpy() / scale, 1e-2, "out")
+
+
+def test_prefill_and_decode_step_interface(cuda_device):
+    """prefill -> (out, state) and decode_step -> (out_t, state) agree with
+    one forward over prompt + tokens (fused 16-bit layer)."""
+    torch.manual_seed(11)
+    B, T, C, H, extra = 2, 150, 128, 4, 5
+    layer = ESA(C, H, mode="direct", device=cuda_device, dtype=torch.float16)
+    x = torch.randn(B, T + extra, C, device=cuda_device, dtype=torch.float16)
+    with torch.no_grad():
+        full = layer(x)
+    out, state = layer.prefill(x[:, :T])
+    steps = []
+    for i in range(extra):
+        y_t, state = layer.decode_step(x[:, T + i], state)
+        steps.append(y_t)
+    scale = float(full.float().abs().max())
+    assert_close(out.float() / scale, host64(full[:, :T].float()) / scale, 1e-2, "prefill")
+    assert_close(torch.stack(steps, dim=1).float() / scale, host64(full[:, T:].float()) / scale, 1e-2, "decode")
