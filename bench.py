@@ -765,6 +765,62 @@ def measure_fp8_forward(dev, a, v, q, mode, reps=10, dy=None):
     return out
 
 
+def measure_other_workloads(dev, reps=10):
+    """The two other throughput workloads of the specification, device-timed:
+    controlled bf16 B=64 T=4096 H=8 D=64 (C=512), forward + backward, inputs
+    (2.1 GB read per step) larger than the L2; and controlled fp16 B=16
+    T=1024 H=4 D=32, forward only, whose 16.8 MB of inputs would stay in the
+    126 MB L2, so a 256 MB buffer is written between iterations (the flush is
+    outside the timed events)."""
+    import torch
+
+    from gated_linear_recurrence_b200 import esa, inputs
+    stream = torch.cuda.current_stream(dev)
+    peak, _ = measured_peak()
+    out = {}
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    for name, with_bwd in (("controlled_bf16_B64_T4096_H8_D64", True), ("controlled_f16_B16_T1024_H4_D32", False)):
+        w = inputs.WORKLOADS[name]
+        B, T, H, D = w.B, w.T, w.H, w.D
+        x = inputs.make_scan_inputs(B, T, H, D, w.dtype, w.a_mean, w.seed, device=dev)
+        ws = esa.new_workspace(B, T, H, D, x["a"].dtype, dev)
+        y = torch.empty_like(x["a"])
+        g = [torch.empty_like(x["a"]) for _ in range(3)]
+        fwd_t = bwd_t = 0.0
+        for k in range(reps + 3):
+            if not with_bwd:
+                flush.fill_(k & 0xff)
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0.record(stream)
+            esa.esa_scan_fwd(x["a"], x["v"], x["q"], y=y, mode=w.mode, workspace=ws, want_E_final=False)
+            e1.record(stream)
+            if with_bwd:
+                esa.esa_scan_bwd(x["a"], x["v"], x["q"], x["dy"], ws, mode=w.mode, da=g[0], dv=g[1], dq=g[2],
+                                 want_dE_init=False)
+            e2.record(stream)
+            torch.cuda.synchronize()
+            if k >= 3:
+                fwd_t += e0.elapsed_time(e1)
+                bwd_t += e1.elapsed_time(e2)
+        esa.esa_check(ws)
+        fwd_ms, bwd_ms = fwd_t / reps, bwd_t / reps
+        el = B * T * H * D
+        s_ = x["a"].element_size()
+        r = {"fwd_ms": fwd_ms, "fwd_GBs": 4 * s_ * el / (fwd_ms / 1e3) / 1e9,
+             "fwd_tokens_per_s": B * T / (fwd_ms / 1e3)}
+        if with_bwd:
+            r.update({"bwd_ms": bwd_ms, "bwd_GBs": 7 * s_ * el / (bwd_ms / 1e3) / 1e9,
+                      "fwd_bwd_tokens_per_s": B * T / ((fwd_ms + bwd_ms) / 1e3),
+                      "fwd_bwd_frac_of_measured_hbm": 11 * s_ * el / ((fwd_ms + bwd_ms) / 1e3) / 1e9 / peak})
+        else:
+            r["note"] = "L2 flushed (256 MB written) before every iteration"
+        out[name] = r
+        del x, ws, y, g
+    del flush
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------------------
 # Our arm.
 # ---------------------------------------------------------------------------
@@ -924,11 +980,12 @@ def run_ours(args):
     cpar = None
     if not args.no_cp and args.batch is None and args.seq is None:
         cpar = measure_context_parallel(dev)
-    fusedm = layerm = fp8m = None
+    fusedm = layerm = fp8m = otherm = None
     if not args.no_fused and args.batch is None and args.seq is None:
         fusedm = measure_fused(dev)
         layerm = measure_layer(dev)
         fp8m = measure_fp8_forward(dev, a, v, q, mode, dy=dy)
+        otherm = measure_other_workloads(dev)
 
     cpu = cpu_all = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -949,7 +1006,7 @@ def run_ours(args):
                    "step_frac_of_measured_peak": step_gbs / peak, "step_frac_of_nominal_8TBs":
                    step_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes_per_step": fwd_bytes + bwd_bytes,
                    "decode": decode, "context_parallel": cpar, "fused_layer_forward": fusedm, "layer_train_step": layerm,
-                   "fp8_forward": fp8m, "cpu_baseline_all_cores": cpu_all},
+                   "fp8_forward": fp8m, "other_workloads": otherm, "cpu_baseline_all_cores": cpu_all},
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": 2 * K,
