@@ -422,7 +422,6 @@ int esa_step(const void *a_t, const void *v_t, const void *q_t, float *E, void *
              int mode, int dtype, void *stream) {
   int rc = check_shape(B, 1, H, D, mode, dtype);
   if (rc) return rc;
-  if (dtype == ESA_E4M3) return ESA_ERR_UNSUPPORTED;   // fp8 inputs: forward scans only
   if (B > 0 && (!a_t || !v_t || !q_t || !E || !y_t)) return ESA_ERR_ARG;
   for (const void *p : {a_t, v_t, q_t, static_cast<const void *>(E), static_cast<const void *>(y_t)})
     if (p && !aligned16(p)) return ESA_ERR_ALIGN;

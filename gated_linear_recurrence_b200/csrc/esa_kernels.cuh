@@ -1061,7 +1061,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
 template <typename T, int MODE, int LPH>
 __global__ void __launch_bounds__(256)
     esa_step_kernel(const T *__restrict__ a, const T *__restrict__ v, const T *__restrict__ q,
-                    float *__restrict__ E, T *__restrict__ y, long nvec, float inv_D) {
+                    float *__restrict__ E, typename OutOf<T>::type *__restrict__ y, long nvec, float inv_D) {
   const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const bool act = idx < nvec;
   float2 x[4], vv[4], qq[4], e[4];
@@ -1086,7 +1086,7 @@ __global__ void __launch_bounds__(256)
   for (int i = 0; i < 4; ++i) yv[i] = mul2(qq[i], mul2(e[i], splat(rr)));
   if (act) {
     Io<float>::store8(E + idx * 8, e);
-    Io<T>::store8(y + idx * 8, yv);
+    Io<typename OutOf<T>::type>::store8(y + idx * 8, yv);
   }
 }
 

@@ -18,7 +18,7 @@ struct StepLauncher {
     const long blocks = (nvec + kBlock - 1) / kBlock;
     esa_step_kernel<T, MODE, LPH><<<static_cast<unsigned>(blocks), kBlock, 0, stream>>>(
         static_cast<const T *>(a), static_cast<const T *>(v), static_cast<const T *>(q), E,
-        static_cast<T *>(y), nvec, inv_D);
+        static_cast<typename OutOf<T>::type *>(y), nvec, inv_D);
     return launch_status(cudaGetLastError());
   }
 };
@@ -38,7 +38,7 @@ int launch_ws_init(WsHeader *hdr, cudaStream_t stream) {
 
 int launch_step(int dtype, int mode, int D, const void *a, const void *v, const void *q, float *E,
                 void *y, long nvec, float inv_D, cudaStream_t stream) {
-  return dispatch(dtype, mode, D, StepLauncher{a, v, q, E, y, nvec, inv_D, stream});
+  return dispatch<true>(dtype, mode, D, StepLauncher{a, v, q, E, y, nvec, inv_D, stream});
 }
 
 }  // namespace esa

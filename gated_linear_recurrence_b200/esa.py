@@ -15,10 +15,8 @@ The functions carry the C names:
 * :func:`esa_compose`   -- apply a sequence of segment maps to a state
 * :func:`esa_fused_fwd` -- forward scan with the a / v / q projections fused in
 
-Input dtypes: float32, float16, bfloat16, and float8_e4m3fn for the scans
-(esa_scan_fwd, esa_scan_bwd, esa_scan_map, esa_scan_bwd_map), whose outputs
-are then float16; the decode step and the fused forward take 16-bit or
-float32 inputs.
+Input dtypes: float32, float16, bfloat16, and float8_e4m3fn (outputs then
+float16) for every call except the fused forward, which takes 16-bit inputs.
 * :func:`esa_check`     -- synchronise and read the device status of a workspace
 * :func:`esa_workspace_init` -- zero a new workspace and write its header
 * :func:`esa_workspace_size`, :func:`esa_strerror`, :func:`esa_version`
@@ -418,7 +416,10 @@ def esa_step(a_t, v_t, q_t, E, y_t=None, mode=CONTROLLED, stream=None):
     if E is None:
         raise ValueError("E (the recurrent state) is required")
     if y_t is None:
-        y_t = torch.empty_like(a_t)
+        y_t = torch.empty(a_t.shape, dtype=out_dtype(a_t.dtype), device=a_t.device)
+    if tuple(y_t.shape) != tuple(a_t.shape) or y_t.dtype != out_dtype(a_t.dtype) or y_t.device != a_t.device \
+            or not y_t.is_contiguous():
+        raise ValueError(f"y_t must be a contiguous {out_dtype(a_t.dtype)} tensor of shape {tuple(a_t.shape)}")
     lib = load_library()
     with _on(a_t.device):
         rc = lib.esa_step(_ptr(a_t), _ptr(v_t), _ptr(q_t), _ptr(E), _ptr(y_t), B, H, D, int(mode),

@@ -57,9 +57,7 @@ typedef enum { ESA_DIRECT = 0, ESA_CONTROLLED = 1 } esa_mode;
 /* I/O element type of the sequence tensors.  ESA_E4M3: the sequence inputs
  * (a, v, q, and dy for the backward) in fp8 e4m3 (1 sign, 4 exponent,
  * 3 mantissa bits, finite, largest 448) and the sequence outputs (y, da, dv,
- * dq) in fp16; accepted by the scans (esa_scan_fwd, esa_scan_fwd_noalloc,
- * esa_scan_bwd, esa_scan_map, esa_scan_bwd_map), not by esa_step or
- * esa_fused_fwd.  "Entangled State Attention v2.1" lists fp8 as an
+ * dq, y_t) in fp16; accepted by every call but esa_fused_fwd.  "Entangled State Attention v2.1" lists fp8 as an
  * experimental precision mode. */
 typedef enum { ESA_F32 = 0, ESA_F16 = 1, ESA_BF16 = 2, ESA_E4M3 = 3 } esa_dtype;
 

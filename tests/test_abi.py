@@ -215,12 +215,12 @@ def test_fp8_inputs_are_a_scan_dtype(lib):
     P = _fake
     # e4m3 inputs: 1-byte a, v, q; the workspace is sized like the 16-bit one (64-row slots)
     assert lib.esa_workspace_size(2, 1000, 4, 32, 3) == lib.esa_workspace_size(2, 1000, 4, 32, 1)
-    rc = lib.esa_step(P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000), 2, 2, 32, 1, 3, None)
-    assert rc == esa.ESA_ERR_UNSUPPORTED
     rc = lib.esa_fused_fwd(P(0x1000), P(0x2000), P(0x3000), None, None, None, None, 2, 8, 2, 32, 128, 1, None, 3,
                            P(0x10000), 1 << 30, None)
     assert rc == esa.ESA_ERR_UNSUPPORTED
     if not torch.cuda.is_available():   # the scans accept it: they get as far as the device check
         rc = lib.esa_scan_bwd(P(0x1000), P(0x2000), P(0x3000), P(0x4000), None, P(0x5000), P(0x6000), P(0x7000),
                               None, 2, 8, 2, 32, 1, None, 3, P(0x10000), 1 << 30, None)
+        assert rc == esa.ESA_ERR_DEVICE
+        rc = lib.esa_step(P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000), 2, 2, 32, 1, 3, None)
         assert rc == esa.ESA_ERR_DEVICE

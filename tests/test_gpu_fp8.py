@@ -4,8 +4,8 @@ a, v, q are e4m3 (torch.float8_e4m3fn); the state and the arithmetic are
 fp32 and y is fp16.  The oracle scans the same e4m3 values widened to fp64,
 so the comparison is the fp16 one (2e-3 (1 + |ref|) plus half an fp16 unit
 in the last place).  The backward takes e4m3 dy too and returns fp16 gradients;
-the decode step and the fused forward do not take fp8 inputs and must say
-so.
+the decode step takes e4m3 inputs and returns fp16; the fused forward does
+not take fp8 inputs and must say so.
 """
 import pytest
 import torch
@@ -78,13 +78,23 @@ def test_fp8_backward_matches_oracle(cuda_device, case):
         assert_close(g, r, TOL[torch.float16], name)
 
 
-def test_fp8_is_refused_by_the_step_and_the_fused_forward(cuda_device):
+def test_fp8_decode_steps_match_oracle(cuda_device):
+    B, H, D, n = 3, 4, 32, 8
+    E = inputs.make_state(B, H, D, seed=440, scale=0.5).to(cuda_device)
+    E_r = host64(E)
+    f64 = lambda t: t.to(torch.float32).to("cpu", torch.float64).numpy()  # noqa: E731
+    for i in range(n):
+        st = inputs.make_step_inputs(B, H, D, "f32", 1.0, seed=441 + i)
+        a, v, q = (st[k].to(F8).to(cuda_device) for k in ("a", "v", "q"))
+        y = esa.esa_step(a, v, q, E, mode=i % 2)
+        assert y.dtype == torch.float16
+        y_r, E_r = oracle.step(f64(a), f64(v), f64(q), E_r, i % 2)
+        assert_close(y, y_r, TOL[torch.float16], f"step{i}.y")
+    assert_close(E, E_r, TOL[torch.float16], "E")
+
+
+def test_fp8_is_refused_by_the_fused_forward(cuda_device):
     B, T, H, D = 1, 64, 2, 32
-    x = _fp8_inputs(B, T, H, D, 420, cuda_device)
-    E = torch.zeros(B, H, D, device=cuda_device)
-    with pytest.raises(esa.EsaError) as err:
-        esa.esa_step(x["a"][:, 0].contiguous(), x["v"][:, 0].contiguous(), x["q"][:, 0].contiguous(), E, mode=1)
-    assert err.value.code == esa.ESA_ERR_UNSUPPORTED
     xin = torch.zeros(B, T, 128, device=cuda_device).to(F8)
     W = torch.zeros(3 * H * D, 128, device=cuda_device).to(F8)
     with pytest.raises(esa.EsaError) as err:
