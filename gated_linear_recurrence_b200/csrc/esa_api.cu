@@ -125,8 +125,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [B][T][C] tensor in the I/O dtype, read in boxes of [rows][CT channels].
-int make_tmap(CUtensorMap *map, const void *ptr, int dtype, int B, int T, int C, const Layout &lo, int rows) {
+// [B][T][C] tensor in the I/O dtype, read in boxes of [rows][CT channels];
+// consecutive tokens' rows are `ld` elements apart (ld = C: contiguous).
+int make_tmap(CUtensorMap *map, const void *ptr, int dtype, int B, int T, int C, const Layout &lo, int rows,
+              long long ld = 0) {
+  if (ld == 0) ld = C;
   auto fn = encode_fn();
   if (fn == nullptr) return ESA_ERR_LAUNCH;
   const CUtensorMapDataType dt = dtype == ESA_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
@@ -136,8 +139,8 @@ int make_tmap(CUtensorMap *map, const void *ptr, int dtype, int B, int T, int C,
   const cuuint64_t s = elem_bytes(dtype);
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(T),
                               static_cast<cuuint64_t>(B)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(C) * s,
-                                 static_cast<cuuint64_t>(T) * static_cast<cuuint64_t>(C) * s};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * s,
+                                 static_cast<cuuint64_t>(T) * static_cast<cuuint64_t>(ld) * s};
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(lo.CT), static_cast<cuuint32_t>(rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   std::memset(map, 0, sizeof(*map));
@@ -195,6 +198,28 @@ int rt(cudaError_t e) {
   return ESA_ERR_LAUNCH;
 }
 
+// A row stride of `ld` elements of `bytes` each: at least C, a whole number
+// of 16-byte units (TMA strides and the kernels' 16-byte stores), and small
+// enough that T rows of a batch stay addressable.
+int check_ld(long long ld, int C, size_t bytes, int T) {
+  if (ld < C || ld > INT_MAX) return ESA_ERR_ARG;
+  if ((static_cast<unsigned long long>(ld) * bytes) % 16u != 0) return ESA_ERR_ALIGN;
+  if (static_cast<long double>(ld) * bytes * (T > 0 ? T : 1) > static_cast<long double>(1ull << 40))
+    return ESA_ERR_ARG;
+  return ESA_OK;
+}
+
+// Element size of the gradients and y: fp8 inputs give fp16 outputs.
+size_t out_bytes(int dtype) { return dtype == ESA_E4M3 ? 2 : elem_bytes(dtype); }
+
+int scan_fwd_impl(const void *a, const void *v, const void *q, long long ld_in, void *y, float *E_final, int B,
+                  int T, int H, int D, int mode, const float *E_init, int dtype, void *workspace,
+                  size_t workspace_bytes, void *stream);
+int scan_bwd_impl(const void *a, const void *v, const void *q, long long ld_in, const void *dy,
+                  const float *dE_final, void *da, void *dv, void *dq, long long ld_grad, float *dE_init, int B,
+                  int T, int H, int D, int mode, const float *E_init, int dtype, void *workspace,
+                  size_t workspace_bytes, void *stream);
+
 }  // namespace
 
 extern "C" {
@@ -208,8 +233,45 @@ size_t esa_workspace_size(int B, int T, int H, int D, int dtype) {
 int esa_scan_fwd(const void *a, const void *v, const void *q, void *y, float *E_final, int B, int T,
                  int H, int D, int mode, const float *E_init, int dtype, void *workspace,
                  size_t workspace_bytes, void *stream) {
+  return scan_fwd_impl(a, v, q, 0, y, E_final, B, T, H, D, mode, E_init, dtype, workspace, workspace_bytes,
+                       stream);
+}
+
+int esa_scan_fwd_ld(const void *a, const void *v, const void *q, long long ld_in, void *y, float *E_final, int B,
+                    int T, int H, int D, int mode, const float *E_init, int dtype, void *workspace,
+                    size_t workspace_bytes, void *stream) {
+  if (ld_in <= 0) return ESA_ERR_ARG;
+  return scan_fwd_impl(a, v, q, ld_in, y, E_final, B, T, H, D, mode, E_init, dtype, workspace, workspace_bytes,
+                       stream);
+}
+
+int esa_scan_bwd_ld(const void *a, const void *v, const void *q, long long ld_in, const void *dy,
+                    const float *dE_final, void *da, void *dv, void *dq, long long ld_grad, float *dE_init, int B,
+                    int T, int H, int D, int mode, const float *E_init, int dtype, void *workspace,
+                    size_t workspace_bytes, void *stream) {
+  if (ld_in <= 0 || ld_grad <= 0) return ESA_ERR_ARG;
+  return scan_bwd_impl(a, v, q, ld_in, dy, dE_final, da, dv, dq, ld_grad, dE_init, B, T, H, D, mode, E_init,
+                       dtype, workspace, workspace_bytes, stream);
+}
+
+int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy, const float *dE_final,
+                 void *da, void *dv, void *dq, float *dE_init, int B, int T, int H, int D, int mode,
+                 const float *E_init, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+  return scan_bwd_impl(a, v, q, 0, dy, dE_final, da, dv, dq, 0, dE_init, B, T, H, D, mode, E_init, dtype,
+                       workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// ld_in / ld_grad = 0: contiguous rows (C elements apart).
+int scan_fwd_impl(const void *a, const void *v, const void *q, long long ld_in, void *y, float *E_final, int B,
+                  int T, int H, int D, int mode, const float *E_init, int dtype, void *workspace,
+                  size_t workspace_bytes, void *stream) {
   int rc = check_shape(B, T, H, D, mode, dtype);
   if (rc) return rc;
+  if (ld_in != 0 && (rc = check_ld(ld_in, H * D, elem_bytes(dtype), T))) return rc;
   const bool has_tokens = B > 0 && T > 0;   // empty tensors may carry NULL pointers
   if (has_tokens && (!a || !v || !q || !y)) return ESA_ERR_ARG;
   for (const void *p : {a, v, q, static_cast<const void *>(y), static_cast<const void *>(E_final),
@@ -230,9 +292,9 @@ int esa_scan_fwd(const void *a, const void *v, const void *q, void *y, float *E_
   }
   const int sub = fwd_slots_per_tile(dtype, D);
   CUtensorMap ta, tv, tq;
-  if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo, lo.L * sub))) return rc;
-  if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo, lo.L * sub))) return rc;
-  if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo, lo.L * sub))) return rc;
+  if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo, lo.L * sub, ld_in))) return rc;
+  if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo, lo.L * sub, ld_in))) return rc;
+  if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo, lo.L * sub, ld_in))) return rc;
   esa::FwdArgs args;
   args.s = scan_shape(B, T, H, D, lo, sub);
   args.y = y;
@@ -242,11 +304,14 @@ int esa_scan_fwd(const void *a, const void *v, const void *q, void *y, float *E_
   return esa::launch_fwd(dtype, mode, D, ta, tv, tq, args, args.s.ntiles, st);
 }
 
-int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy, const float *dE_final,
-                 void *da, void *dv, void *dq, float *dE_init, int B, int T, int H, int D, int mode,
-                 const float *E_init, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+int scan_bwd_impl(const void *a, const void *v, const void *q, long long ld_in, const void *dy,
+                  const float *dE_final, void *da, void *dv, void *dq, long long ld_grad, float *dE_init, int B,
+                  int T, int H, int D, int mode, const float *E_init, int dtype, void *workspace,
+                  size_t workspace_bytes, void *stream) {
   int rc = check_shape(B, T, H, D, mode, dtype);
   if (rc) return rc;
+  if (ld_in != 0 && (rc = check_ld(ld_in, H * D, elem_bytes(dtype), T))) return rc;
+  if (ld_grad != 0 && (rc = check_ld(ld_grad, H * D, out_bytes(dtype), T))) return rc;
   const bool has_tokens = B > 0 && T > 0;   // empty tensors may carry NULL pointers
   if (has_tokens && (!a || !v || !q || !dy || !da || !dv || !dq)) return ESA_ERR_ARG;
   for (const void *p : {a, v, q, dy, static_cast<const void *>(dE_final), static_cast<const void *>(da),
@@ -269,21 +334,26 @@ int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy, co
   }
   const int sub = esa::bwd_slots_per_tile(dtype, D);
   CUtensorMap ta, tv, tq, tdy;
-  if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo, lo.L * sub))) return rc;
-  if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo, lo.L * sub))) return rc;
-  if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo, lo.L * sub))) return rc;
+  if ((rc = make_tmap(&ta, a, dtype, B, T, C, lo, lo.L * sub, ld_in))) return rc;
+  if ((rc = make_tmap(&tv, v, dtype, B, T, C, lo, lo.L * sub, ld_in))) return rc;
+  if ((rc = make_tmap(&tq, q, dtype, B, T, C, lo, lo.L * sub, ld_in))) return rc;
   if ((rc = make_tmap(&tdy, dy, dtype, B, T, C, lo, lo.L * sub))) return rc;
   esa::BwdArgs args;
   args.s = scan_shape(B, T, H, D, lo, sub);
   args.da = da;
   args.dv = dv;
   args.dq = dq;
+  args.ldg = ld_grad != 0 ? ld_grad : C;
   args.dE_final = dE_final;
   args.dE_init = dE_init;
   args.E_init = E_init;
   args.ws = workspace_view(workspace, lo);
   return esa::launch_bwd(dtype, mode, D, ta, tv, tq, tdy, args, args.s.ntiles, st);
 }
+
+}  // namespace
+
+extern "C" {
 
 int esa_scan_map(const void *a, const void *v, float *P, float *S, int B, int T, int H, int D, int mode,
                  int dtype, void *workspace, size_t workspace_bytes, void *stream) {
@@ -338,6 +408,7 @@ int esa_scan_bwd_map(const void *a, const void *v, const void *q, const void *dy
   esa::BwdArgs args;
   args.s = scan_shape(B, T, H, D, lo, sub);
   args.da = args.dv = args.dq = nullptr;
+  args.ldg = C;
   args.dE_final = nullptr;
   args.dE_init = nullptr;
   args.E_init = E_init;

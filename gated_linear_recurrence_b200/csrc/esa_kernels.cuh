@@ -66,6 +66,7 @@ struct FwdArgs {
 struct BwdArgs {
   ScanShape s;
   void *da, *dv, *dq;
+  long ldg;   // elements between consecutive tokens' rows of da, dv, dq (C when contiguous)
   const float *dE_final;
   float *dE_init;
   const float *E_init;
@@ -931,7 +932,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
         if constexpr (Cfg::kSeparateScratch) put_ghat<float>(gh_s + r * CT + pos.ch, nullptr, gh);
         else put_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
         if (!MAP && valid && (c0 + pos.ch) < sh.C)
-          Io<TO>::store8(dqg + (static_cast<long>(b) * sh.T + t0 + r) * sh.C + c0 + pos.ch, dqv);
+          Io<TO>::store8(dqg + (static_cast<long>(b) * sh.T + t0 + r) * args.ldg + c0 + pos.ch, dqv);
       }
     }
 
@@ -1010,7 +1011,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     // ---- B: total gradient G_t (latest step first): dv and
     //      da = G A (1 - A) (E_{t-1} - v_t)  (direct mode: times E_{t-1}).
     const bool ch_ok = (c0 + pos.ch) < sh.C;
-    const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
+    const long gbase = (static_cast<long>(b) * sh.T + t0) * args.ldg + c0 + pos.ch;
     if constexpr (!MAP) {
       float2 h[4];
       run_carry<CT>(scan_s, es_s, pos.run, pos.ch, h);
@@ -1030,8 +1031,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
             h[q] = mul2(A, G);
           }
           if (ch_ok) {
-            Io<TO>::store8(dvg + gbase + static_cast<long>(r) * sh.C, dvv);
-            Io<TO>::store8(dag + gbase + static_cast<long>(r) * sh.C, dav);
+            Io<TO>::store8(dvg + gbase + static_cast<long>(r) * args.ldg, dvv);
+            Io<TO>::store8(dag + gbase + static_cast<long>(r) * args.ldg, dav);
           }
         }
       }

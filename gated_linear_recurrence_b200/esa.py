@@ -9,6 +9,9 @@ The functions carry the C names:
 
 * :func:`esa_scan_fwd`  -- forward scan (+ E_final, + checkpoints in the workspace)
 * :func:`esa_scan_bwd`  -- backward scan (da, dv, dq, dE_init)
+
+  Both also take row-strided a, v, q (and da, dv, dq): column blocks of one
+  ``[B, T, 3 H D]`` buffer, through ``esa_scan_fwd_ld`` / ``esa_scan_bwd_ld``.
 * :func:`esa_step`      -- one-token decode update (in place on E)
 * :func:`esa_scan_map`, :func:`esa_scan_bwd_map` -- forward / backward segment
   maps ``(P, S)`` of a time slice (context parallelism)
@@ -81,6 +84,11 @@ def load_library():
         lib.esa_scan_fwd.restype = I
         lib.esa_scan_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, P, I, P, S, P]
         lib.esa_scan_bwd.restype = I
+        L = ctypes.c_longlong
+        lib.esa_scan_fwd_ld.argtypes = [P, P, P, L, P, P, I, I, I, I, I, P, I, P, S, P]
+        lib.esa_scan_fwd_ld.restype = I
+        lib.esa_scan_bwd_ld.argtypes = [P, P, P, L, P, P, P, P, P, L, P, I, I, I, I, I, P, I, P, S, P]
+        lib.esa_scan_bwd_ld.restype = I
         lib.esa_scan_map.argtypes = [P, P, P, P, I, I, I, I, I, I, P, S, P]
         lib.esa_scan_map.restype = I
         lib.esa_scan_bwd_map.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, I, P, S, P]
@@ -154,6 +162,42 @@ def _check_seq(name, t, ref):
         raise ValueError(f"{name} must be contiguous [B, T, H, D]")
 
 
+def row_stride(t):
+    """Elements between consecutive tokens' rows of a ``[B, T, H, D]`` tensor
+    whose H * D channels per token are contiguous (e.g. a column block of a
+    ``[B, T, 3 H D]`` projection output); None for any other layout."""
+    B, T, H, D = (int(x) for x in t.shape)
+    st = t.stride()
+    if (D > 1 and st[3] != 1) or (H > 1 and st[2] != D):
+        return None
+    if T > 1:
+        ld = st[1]
+        if B > 1 and st[0] != T * ld:
+            return None
+    elif B > 1:
+        ld = st[0]
+    else:
+        ld = H * D
+    return ld if ld >= H * D else None
+
+
+def _strided_seq(names, ts, ref):
+    """Common row stride of same-shaped sequence tensors (checked)."""
+    lds = set()
+    for name, t in zip(names, ts):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor (the ESA library has no CPU path)")
+        if t.shape != ref.shape or t.device != ref.device:
+            raise ValueError(f"{name} must have shape {tuple(ref.shape)} on {ref.device}")
+        ld = row_stride(t)
+        if ld is None:
+            raise ValueError(f"{name} must be [B, T, H, D] with each token's H*D channels contiguous")
+        lds.add(ld)
+    if len(lds) != 1:
+        raise ValueError(f"{', '.join(names)} must share one row stride (got {sorted(lds)})")
+    return lds.pop()
+
+
 def _check_state(name, t, B, H, D, device):
     if t is None:
         return
@@ -163,14 +207,14 @@ def _check_state(name, t, B, H, D, device):
         raise ValueError(f"{name} must be a contiguous float32 tensor of shape {(B, H, D)}")
 
 
-def _dims(a):
+def _dims(a, strided=False):
     if not isinstance(a, torch.Tensor) or not a.is_cuda:
         raise TypeError("a must be a CUDA tensor (the ESA library has no CPU path)")
     if a.dim() != 4:
         raise ValueError("sequence tensors must be [B, T, H, D]")
     if a.dtype not in _DTYPE_CODE:
         raise TypeError(f"unsupported dtype {a.dtype}")
-    if not a.is_contiguous():
+    if not strided and not a.is_contiguous():
         raise ValueError("a must be contiguous [B, T, H, D]")
     return tuple(int(s) for s in a.shape)
 
@@ -202,11 +246,16 @@ def esa_scan_fwd(a, v, q, y=None, E_final=None, mode=CONTROLLED, E_init=None, wo
 
     ``workspace`` (uint8 CUDA tensor) is allocated when not given; keep it for
     :func:`esa_scan_bwd`.  ``E_final`` is allocated when not given unless
-    ``want_E_final`` is False.
+    ``want_E_final`` is False.  a, v, q may be row-strided views (each
+    token's channels contiguous, one row stride for the three, e.g. column
+    blocks of one projection output): they then go through
+    ``esa_scan_fwd_ld``.
     """
-    B, T, H, D = _dims(a)
-    _check_seq("v", v, a)
-    _check_seq("q", q, a)
+    B, T, H, D = _dims(a, strided=True)
+    ld = _strided_seq(("a", "v", "q"), (a, v, q), a)
+    for name, t in (("v", v), ("q", q)):
+        if t.dtype != a.dtype:
+            raise ValueError(f"{name} must match a: dtype {a.dtype}")
     ydt = out_dtype(a.dtype)
     if y is None:
         y = torch.empty(a.shape, dtype=ydt, device=a.device)
@@ -221,11 +270,16 @@ def esa_scan_fwd(a, v, q, y=None, E_final=None, mode=CONTROLLED, E_init=None, wo
         workspace = new_workspace(B, T, H, D, a.dtype, a.device)
     lib = load_library()
     with _on(a.device):
-        rc = lib.esa_scan_fwd(_ptr(a), _ptr(v), _ptr(q), _ptr(y), _ptr(E_final), B, T, H, D, int(mode),
-                              _ptr(E_init), _DTYPE_CODE[a.dtype], _ptr(workspace),
-                              workspace.numel() * workspace.element_size(), _stream(a.device, stream))
+        if ld == H * D:
+            rc = lib.esa_scan_fwd(_ptr(a), _ptr(v), _ptr(q), _ptr(y), _ptr(E_final), B, T, H, D, int(mode),
+                                  _ptr(E_init), _DTYPE_CODE[a.dtype], _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(a.device, stream))
+        else:
+            rc = lib.esa_scan_fwd_ld(_ptr(a), _ptr(v), _ptr(q), ld, _ptr(y), _ptr(E_final), B, T, H, D,
+                                     int(mode), _ptr(E_init), _DTYPE_CODE[a.dtype], _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(a.device, stream))
     if rc != 0:
-        raise EsaError("esa_scan_fwd", rc)
+        raise EsaError("esa_scan_fwd" if ld == H * D else "esa_scan_fwd_ld", rc)
     return y, E_final, workspace
 
 
@@ -233,19 +287,26 @@ def esa_scan_bwd(a, v, q, dy, workspace, mode=CONTROLLED, E_init=None, dE_final=
                  dq=None, dE_init=None, stream=None, want_dE_init=True):
     """Backward scan.  ``workspace`` must be the one the matching forward wrote.
 
-    Returns ``(da, dv, dq, dE_init)``.
+    Returns ``(da, dv, dq, dE_init)``.  a, v, q (one row stride) and the
+    given da, dv, dq (another) may be row-strided views, e.g. column blocks
+    of one ``[B, T, 3 H D]`` buffer; dy is contiguous.  Strided rows go
+    through ``esa_scan_bwd_ld``.
     """
-    B, T, H, D = _dims(a)
-    for name, t in (("v", v), ("q", q), ("dy", dy)):
-        _check_seq(name, t, a)
+    B, T, H, D = _dims(a, strided=True)
+    ld_in = _strided_seq(("a", "v", "q"), (a, v, q), a)
+    for name, t in (("v", v), ("q", q)):
+        if t.dtype != a.dtype:
+            raise ValueError(f"{name} must match a: dtype {a.dtype}")
+    _check_seq("dy", dy, a)
     odt = out_dtype(a.dtype)
     da = torch.empty(a.shape, dtype=odt, device=a.device) if da is None else da
     dv = torch.empty(a.shape, dtype=odt, device=a.device) if dv is None else dv
     dq = torch.empty(a.shape, dtype=odt, device=a.device) if dq is None else dq
     for name, t in (("da", da), ("dv", dv), ("dq", dq)):
         if not isinstance(t, torch.Tensor) or tuple(t.shape) != tuple(a.shape) or t.dtype != odt \
-                or t.device != a.device or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous {odt} tensor of shape {tuple(a.shape)} on {a.device}")
+                or t.device != a.device:
+            raise ValueError(f"{name} must be a {odt} tensor of shape {tuple(a.shape)} on {a.device}")
+    ld_g = _strided_seq(("da", "dv", "dq"), (da, dv, dq), a)
     if dE_init is None and want_dE_init:
         dE_init = torch.empty((B, H, D), dtype=torch.float32, device=a.device)
     _check_state("dE_init", dE_init, B, H, D, a.device)
@@ -254,13 +315,20 @@ def esa_scan_bwd(a, v, q, dy, workspace, mode=CONTROLLED, E_init=None, dE_final=
     if workspace is None or not workspace.is_cuda:
         raise ValueError("esa_scan_bwd needs the CUDA workspace written by the matching esa_scan_fwd")
     lib = load_library()
+    plain = ld_in == H * D and ld_g == H * D
     with _on(a.device):
-        rc = lib.esa_scan_bwd(_ptr(a), _ptr(v), _ptr(q), _ptr(dy), _ptr(dE_final), _ptr(da), _ptr(dv),
-                              _ptr(dq), _ptr(dE_init), B, T, H, D, int(mode), _ptr(E_init),
-                              _DTYPE_CODE[a.dtype], _ptr(workspace),
-                              workspace.numel() * workspace.element_size(), _stream(a.device, stream))
+        if plain:
+            rc = lib.esa_scan_bwd(_ptr(a), _ptr(v), _ptr(q), _ptr(dy), _ptr(dE_final), _ptr(da), _ptr(dv),
+                                  _ptr(dq), _ptr(dE_init), B, T, H, D, int(mode), _ptr(E_init),
+                                  _DTYPE_CODE[a.dtype], _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(a.device, stream))
+        else:
+            rc = lib.esa_scan_bwd_ld(_ptr(a), _ptr(v), _ptr(q), ld_in, _ptr(dy), _ptr(dE_final), _ptr(da),
+                                     _ptr(dv), _ptr(dq), ld_g, _ptr(dE_init), B, T, H, D, int(mode),
+                                     _ptr(E_init), _DTYPE_CODE[a.dtype], _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(a.device, stream))
     if rc != 0:
-        raise EsaError("esa_scan_bwd", rc)
+        raise EsaError("esa_scan_bwd" if plain else "esa_scan_bwd_ld", rc)
     return da, dv, dq, dE_init
 
 

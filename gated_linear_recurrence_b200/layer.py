@@ -15,9 +15,12 @@ When the shapes allow it (16-bit weights and input, no bias, head dimension
 <= 64, input width 64 or 128) the input projections run inside the scan
 kernel on the tensor cores (``esa_fused_fwd``); in training that call also
 writes a, v, q for the library backward, and the projections' own gradients
-(dx, dW) are ordinary GEMMs.  Otherwise the projections are
-``torch.nn.Linear`` layers feeding ``esa_scan``.  W_O is always a linear
-layer.  Every step of the recurrence and its readout runs in the CUDA
+(dx, dW) are ordinary GEMMs.  Otherwise the three input projections are one
+GEMM whose ``[B, T, 3 C]`` output the scan reads in place (a, v, q are its
+column blocks, row stride 3 C); the backward writes da, dv, dq into one such
+buffer, so dx and dW are single GEMMs over K = 3 C as well.  With a
+context-parallel group the projections are separate linear layers feeding
+the context-parallel scan.  W_O is always a linear layer.  Every step of the recurrence and its readout runs in the CUDA
 library; there is no CPU path.
 """
 from __future__ import annotations
@@ -85,17 +88,73 @@ class _FusedProjScanFn(torch.autograd.Function):
         E0 = E0 if ctx.has_E_init else None
         dy = torch.zeros_like(a) if dy is None else dy.to(a.dtype).contiguous()
         dEf = None if dE_final is None else dE_final.float().contiguous()
-        da, dv, dq, dE0 = _esa.esa_scan_bwd(a, v, q, dy, ctx.ws, mode=ctx.mode, E_init=E0, dE_final=dEf,
-                                            want_dE_init=ctx.has_E_init)
+        G, dE0 = _grads_into_one_buffer(a, v, q, dy, ctx.ws, ctx.mode, E0, dEf, ctx.has_E_init)
         ctx.ws = None
-        B, T = x.shape[:2]
+        dx, dW, _ = _projection_grads(G, x, W, ctx.needs_input_grad[0], False)
+        return dx, dW, (dE0 if ctx.has_E_init else None), None, None
+
+
+def _grads_into_one_buffer(a, v, q, dy, ws, mode, E0, dEf, want_dE_init):
+    """esa_scan_bwd writing da, dv, dq as the column blocks of one
+    ``[B, T, 3 C]`` buffer (row stride 3 C), so that the projections'
+    gradients are single GEMMs over K = 3 C."""
+    B, T, H, D = a.shape
+    G = torch.empty(B, T, 3, H, D, dtype=_esa.out_dtype(a.dtype), device=a.device)
+    da, dv, dq = G.unbind(2)
+    _, _, _, dE0 = _esa.esa_scan_bwd(a, v, q, dy, ws, mode=mode, E_init=E0, dE_final=dEf, da=da, dv=dv, dq=dq,
+                                     want_dE_init=want_dE_init)
+    return G, dE0
+
+
+def _projection_grads(G, x, W, want_dx, want_db):
+    """dx = G W, dW = G^T x (and db = column sums of G) for the projection
+    P = x W^T (+ b), G = dL/dP as ``[B, T, 3 C]``."""
+    B, T = x.shape[:2]
+    G2 = G.reshape(B * T, -1)
+    if G2.dtype != W.dtype:
+        G2 = G2.to(W.dtype)
+    x2 = x.reshape(B * T, -1)
+    dx = (G2 @ W).reshape(x.shape) if want_dx else None
+    dW = G2.t() @ x2
+    db = G2.sum(0) if want_db else None
+    return dx, dW, db
+
+
+class _ProjScanFn(torch.autograd.Function):
+    """(x, W = [W_A; W_V; W_Q], b) -> (y, E_final) with the three input
+    projections as one GEMM: P = x W^T + b is ``[B, T, 3 C]`` and a, v, q are
+    its column blocks, scanned in place (row stride 3 C, esa_scan_fwd_ld).
+    The backward writes da, dv, dq into one ``[B, T, 3 C]`` buffer
+    (esa_scan_bwd_ld), so dx = G W and dW = G^T x are single GEMMs."""
+
+    @staticmethod
+    def forward(ctx, x, W, b, E_init, mode, H, scan_dtype):
+        B, T, _ = x.shape
         C = W.shape[0] // 3
-        x2 = x.reshape(B * T, -1)
-        gs = [t.reshape(B * T, C) for t in (da, dv, dq)]
-        dx = gs[0] @ W[:C]
-        dx.addmm_(gs[1], W[C:2 * C]).addmm_(gs[2], W[2 * C:])
-        dW = torch.cat([g.t() @ x2 for g in gs], dim=0)
-        return dx.reshape(x.shape), dW, (dE0 if ctx.has_E_init else None), None, None
+        P = torch.nn.functional.linear(x, W, b)
+        if scan_dtype is not None and P.dtype != scan_dtype:
+            P = P.to(scan_dtype)
+        a, v, q = P.view(B, T, 3, H, C // H).unbind(2)
+        E0 = None if E_init is None else E_init.detach().contiguous().float()
+        y, E_final, ws = _esa.esa_scan_fwd(a, v, q, mode=mode, E_init=E0)
+        ctx.mode, ctx.has_E_init, ctx.has_b, ctx.H = mode, E_init is not None, b is not None, H
+        ctx.ws = ws
+        ctx.save_for_backward(x, W, P, E0 if E0 is not None else torch.empty(0, device=x.device))
+        return y, E_final
+
+    @staticmethod
+    def backward(ctx, dy, dE_final):
+        x, W, P, E0 = ctx.saved_tensors
+        E0 = E0 if ctx.has_E_init else None
+        B, T, _ = x.shape
+        C = W.shape[0] // 3
+        a, v, q = P.view(B, T, 3, ctx.H, C // ctx.H).unbind(2)
+        dy = torch.zeros(a.shape, dtype=a.dtype, device=a.device) if dy is None else dy.to(a.dtype).contiguous()
+        dEf = None if dE_final is None else dE_final.float().contiguous()
+        G, dE0 = _grads_into_one_buffer(a, v, q, dy, ctx.ws, ctx.mode, E0, dEf, ctx.has_E_init)
+        ctx.ws = None
+        dx, dW, db = _projection_grads(G, x, W, ctx.needs_input_grad[0], ctx.has_b)
+        return dx, dW, db, (dE0 if ctx.has_E_init else None), None, None, None
 
 
 def esa_scan(a, v, q, mode="controlled", E_init=None):
@@ -182,12 +241,14 @@ class ESA(torch.nn.Module):
             y, E = _FusedProjScanFn.apply(x, W, state, m, self.head)
             out = self.W_O(y.reshape(B, T, C).to(self.W_O.weight.dtype))
             return (out, E) if return_state else out
-        a, v, q = self._proj(x, (B, T, self.head, self.head_dim))
         if self.cp_group is not None:
             from .context_parallel import cp_esa_scan
+            a, v, q = self._proj(x, (B, T, self.head, self.head_dim))
             y, E = cp_esa_scan(a, v, q, self.mode, E_init=state, group=self.cp_group)
         else:
-            y, E = esa_scan(a, v, q, self.mode, E_init=state)
+            W = torch.cat([self.W_A.weight, self.W_V.weight, self.W_Q.weight], dim=0)
+            b = None if self.W_A.bias is None else torch.cat([self.W_A.bias, self.W_V.bias, self.W_Q.bias])
+            y, E = _ProjScanFn.apply(x, W, b, state, _MODES[self.mode], self.head, self.scan_dtype)
         out = self.W_O(y.reshape(B, T, C).to(self.W_O.weight.dtype))
         return (out, E) if return_state else out
 

@@ -144,6 +144,29 @@ int esa_scan_bwd(const void *a, const void *v, const void *q, const void *dy,
                  int dtype, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * The two scans on token rows with a stride, so that a, v, q can be column
+ * blocks of one projection output [B,T,ld_in] (e.g. ld_in = 3C, a at column
+ * 0, v at C, q at 2C) and da, dv, dq column blocks of one gradient buffer
+ * [B,T,ld_grad], which the projections' backward then multiplies in a
+ * single GEMM.  Element (b, t, c) of a, v, q (and of a gradient) is at
+ * ptr[(b T + t) ld + c].  y and dy stay contiguous [B,T,H,D].
+ *   ld_in     row stride of a, v, q, in elements: >= C, and ld_in times the
+ *             element size a multiple of 16 bytes (else ESA_ERR_ARG /
+ *             ESA_ERR_ALIGN).
+ *   ld_grad   row stride of da, dv, dq, in elements of the output type (fp16
+ *             for ESA_E4M3): the same rules.  Their rows must not overlap.
+ * Every other argument, the results and the workspace rules are those of
+ * esa_scan_fwd / esa_scan_bwd, which are these calls with ld_in = ld_grad = C.
+ */
+int esa_scan_fwd_ld(const void *a, const void *v, const void *q, long long ld_in, void *y, float *E_final,
+                    int B, int T, int H, int D, int mode, const float *E_init,
+                    int dtype, void *workspace, size_t workspace_bytes, void *stream);
+int esa_scan_bwd_ld(const void *a, const void *v, const void *q, long long ld_in, const void *dy,
+                    const float *dE_final, void *da, void *dv, void *dq, long long ld_grad, float *dE_init,
+                    int B, int T, int H, int D, int mode, const float *E_init,
+                    int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Forward scan that allocates nothing.  The pages have no counterpart of this
  * entry point; it exists for callers that cannot allocate device memory at
  * the point where they run the scan -- serving loops whose device-memory

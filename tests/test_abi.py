@@ -224,3 +224,49 @@ def test_fp8_inputs_are_a_scan_dtype(lib):
         assert rc == esa.ESA_ERR_DEVICE
         rc = lib.esa_step(P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000), 2, 2, 32, 1, 3, None)
         assert rc == esa.ESA_ERR_DEVICE
+
+
+def test_row_strided_entry_points_check_their_strides(lib):
+    """esa_scan_fwd_ld / esa_scan_bwd_ld: a row stride below C is an argument
+    error, one that is not a whole number of 16-byte units an alignment
+    error; a well-formed call on a machine without a device reports that."""
+    from gated_linear_recurrence_b200 import esa
+    P = _fake
+    C = 64   # H = 2, D = 32
+
+    def fwd(ld, dtype=1):
+        return lib.esa_scan_fwd_ld(P(0x1000), P(0x2000), P(0x3000), ld, P(0x4000), None, 2, 8, 2, 32, 1, None,
+                                   dtype, P(0x10000), 1 << 30, None)
+
+    def bwd(ld_in, ld_g, dtype=1):
+        return lib.esa_scan_bwd_ld(P(0x1000), P(0x2000), P(0x3000), ld_in, P(0x4000), None, P(0x5000),
+                                   P(0x6000), P(0x7000), ld_g, None, 2, 8, 2, 32, 1, None, dtype, P(0x10000),
+                                   1 << 30, None)
+
+    assert fwd(0) == esa.ESA_ERR_ARG
+    assert fwd(C - 8) == esa.ESA_ERR_ARG
+    assert fwd(3 * C + 1) == esa.ESA_ERR_ALIGN       # 16-bit: 386 bytes
+    assert fwd(3 * C + 2, dtype=0) == esa.ESA_ERR_ALIGN   # fp32: 776 bytes
+    assert fwd(3 * C + 8, dtype=3) == esa.ESA_ERR_ALIGN   # e4m3: 200 bytes
+    assert bwd(3 * C, C - 1) == esa.ESA_ERR_ARG
+    assert bwd(3 * C, 3 * C + 4) == esa.ESA_ERR_ALIGN
+    import torch
+    if not torch.cuda.is_available():
+        assert fwd(3 * C) == esa.ESA_ERR_DEVICE
+        assert bwd(3 * C, 3 * C) == esa.ESA_ERR_DEVICE
+        assert bwd(3 * C, 3 * C + 8, dtype=3) == esa.ESA_ERR_DEVICE   # e4m3 grads are fp16: 400-byte rows
+
+
+def test_row_stride_of_views():
+    import torch
+    from gated_linear_recurrence_b200.esa import row_stride
+    B, T, H, D = 2, 5, 4, 8
+    C = H * D
+    P = torch.empty(B, T, 3 * C)
+    a, v, q = P.view(B, T, 3, H, D).unbind(2)
+    assert row_stride(a) == row_stride(q) == 3 * C
+    assert row_stride(torch.empty(B, T, H, D)) == C
+    assert row_stride(torch.empty(B, T, D, H).transpose(2, 3)) is None          # channels not contiguous
+    assert row_stride(torch.empty(T, B, H, D).transpose(0, 1)) is None          # batch inside time
+    assert row_stride(torch.empty(1, 1, H, D)) == C
+    assert row_stride(P.view(B, T, 3, H, D)[:, :1].unbind(2)[1]) == T * 3 * C   # T = 1: rows are batch rows

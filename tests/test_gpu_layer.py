@@ -163,3 +163,44 @@ def test_prefill_and_decode_step_interface(cuda_device):
     scale = float(full.float().abs().max())
     assert_close(out.float() / scale, host64(full[:, :T].float()) / scale, 1e-2, "prefill")
     assert_close(torch.stack(steps, dim=1).float() / scale, host64(full[:, T:].float()) / scale, 1e-2, "decode")
+
+
+@pytest.mark.parametrize("bias,wdt,sdt", [(True, torch.float32, torch.float16), (False, torch.bfloat16, None),
+                                          (True, torch.float32, None)])
+def test_layer_one_projection_gemm_matches_separate_projections(cuda_device, bias, wdt, sdt):
+    """The unfused layer runs its three input projections as one GEMM and
+    scans the column blocks of its output in place; its backward writes da,
+    dv, dq into one buffer.  Against the same layer written with three
+    separate projections feeding esa_scan: output, final state and every
+    gradient (input, initial state, weights, biases)."""
+    torch.manual_seed(11)
+    B, T, C, H = 2, 257, 128, 4
+    layer = ESA(C, H, mode="controlled", bias=bias, scan_dtype=sdt, device=cuda_device, dtype=wdt, fused=False)
+    x = torch.randn(B, T, C, device=cuda_device, dtype=wdt)
+    E0 = torch.randn(B, H, C // H, device=cuda_device) * 0.3
+    g = torch.randn(B, T, C, device=cuda_device, dtype=wdt)
+
+    def separate(xi, Ei):
+        proj = [lin(xi).reshape(B, T, H, C // H) for lin in (layer.W_A, layer.W_V, layer.W_Q)]
+        if sdt is not None:
+            proj = [p.to(sdt) for p in proj]
+        y, E = esa_scan(*proj, "controlled", E_init=Ei)
+        return layer.W_O(y.reshape(B, T, C).to(wdt)), E
+
+    res = []
+    for run in (lambda xi, Ei: layer(xi, state=Ei, return_state=True), separate):
+        layer.zero_grad(set_to_none=True)
+        xi = x.clone().requires_grad_(True)
+        Ei = E0.clone().requires_grad_(True)
+        out, E = run(xi, Ei)
+        ((out.float() * g.float()).sum() + E.sum()).backward()
+        grads = [getattr(layer, n).weight.grad for n in ("W_A", "W_V", "W_Q", "W_O")]
+        if bias:
+            grads += [getattr(layer, n).bias.grad for n in ("W_A", "W_V", "W_Q")]
+        res.append([out.detach(), E.detach(), xi.grad, Ei.grad] + grads)
+    names = ["out", "E_final", "dx", "dE0", "dW_A", "dW_V", "dW_Q", "dW_O"] + (["db_A", "db_V", "db_Q"] if bias else [])
+    # The GEMMs accumulate in different orders; 16-bit roundings may then differ by one unit.
+    tol = 1e-2 if torch.bfloat16 in (wdt, sdt) else 5e-3
+    for name, one, sep in zip(names, res[0], res[1]):
+        scale = float(sep.float().abs().max()) or 1.0
+        assert_close(one.float() / scale, host64(sep.float()) / scale, tol, name)
