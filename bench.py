@@ -669,8 +669,10 @@ def measure_layer(dev, reps=5, seq=None):
     activations, no bias) on the benchmark workload's shape: B = 64,
     T = 65536, embd = 128, 4 heads, controlled.  Fused: the input
     projections inside the scan kernel (esa_fused_fwd writing a, v, q for
-    esa_scan_bwd); unfused: linear projections + esa_scan.  W_O and the
-    projections' gradients are cuBLAS GEMMs in both."""
+    esa_scan_bwd); unfused: the three projections as one GEMM whose
+    [B, T, 3C] output the scan reads in place (row stride 3C).  W_O and the
+    projections' gradients (single GEMMs over K = 3C: the backward writes
+    da, dv, dq into one buffer) are cuBLAS GEMMs in both."""
     import torch
 
     from gated_linear_recurrence_b200 import ESA
