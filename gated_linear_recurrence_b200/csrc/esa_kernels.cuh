@@ -874,7 +874,16 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
       }
     }
     // The gate rows are free from here on (only this warp read its own rows).
-    if constexpr (Cfg::kWarpScratch) __syncwarp(); else __syncthreads();
+    // A separate scratch region needs no wait: each thread writes only the
+    // entries of its own run and channels, which only it reads again (the
+    // previous tile's B phase); the run scans that read every entry are
+    // fenced by the barriers of their own tiles.
+    if constexpr (Cfg::kSeparateScratch) {
+    } else if constexpr (Cfg::kWarpScratch) {
+      __syncwarp();
+    } else {
+      __syncthreads();
+    }
     scan_store8<CT>(scan_s, pos.run, pos.ch, P, S);
     __syncthreads();
     // The checkpoint carry goes in only now: every warp has left the previous
