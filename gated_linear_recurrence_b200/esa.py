@@ -9,20 +9,21 @@ The functions carry the C names:
 
 * :func:`esa_scan_fwd`  -- forward scan (+ E_final, + checkpoints in the workspace)
 * :func:`esa_scan_bwd`  -- backward scan (da, dv, dq, dE_init)
-
-  Both also take row-strided a, v, q (and da, dv, dq): column blocks of one
-  ``[B, T, 3 H D]`` buffer, through ``esa_scan_fwd_ld`` / ``esa_scan_bwd_ld``.
 * :func:`esa_step`      -- one-token decode update (in place on E)
 * :func:`esa_scan_map`, :func:`esa_scan_bwd_map` -- forward / backward segment
   maps ``(P, S)`` of a time slice (context parallelism)
 * :func:`esa_compose`   -- apply a sequence of segment maps to a state
 * :func:`esa_fused_fwd` -- forward scan with the a / v / q projections fused in
-
-Input dtypes: float32, float16, bfloat16, and float8_e4m3fn (outputs then
-float16) for every call except the fused forward, which takes 16-bit inputs.
 * :func:`esa_check`     -- synchronise and read the device status of a workspace
 * :func:`esa_workspace_init` -- zero a new workspace and write its header
 * :func:`esa_workspace_size`, :func:`esa_strerror`, :func:`esa_version`
+
+The two scans also take row-strided a, v, q (and da, dv, dq): column blocks
+of one ``[B, T, 3 H D]`` buffer, passed to ``esa_scan_fwd_ld`` /
+``esa_scan_bwd_ld`` with their row stride.
+
+Input dtypes: float32, float16, bfloat16, and float8_e4m3fn (outputs then
+float16) for every call except the fused forward, which takes 16-bit inputs.
 """
 from __future__ import annotations
 
