@@ -67,6 +67,9 @@ def parse_args(argv=None):
                          "segment maps) instead of giving every rank its own batch: strong scaling")
     ap.add_argument("--cp-only", action="store_true",
                     help="run only the context-parallel phase timing (one JSON line; for profiling its kernels)")
+    ap.add_argument("--fp8-only", action="store_true",
+                    help="run only the fp8 (e4m3) forward + backward timing against fp16 on the workload's inputs "
+                         "(one JSON line; for profiling its kernels; --seq shortens the sequence)")
     ap.add_argument("--batch", type=int, default=None,
                     help="run a smaller batch of the same workload (profiling cases only)")
     ap.add_argument("--seq", type=int, default=None,
@@ -1029,12 +1032,18 @@ def main(argv=None):
         return run_reference(args)
     if args.context_parallel:
         return run_context_parallel(args)
-    if args.cp_only or args.fused_only:
+    if args.cp_only or args.fused_only or args.fp8_only:
         import torch
         dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
         torch.cuda.set_device(dev)
         if args.cp_only:
             print(json.dumps({"context_parallel": measure_context_parallel(dev)}), flush=True)
+        elif args.fp8_only:
+            from gated_linear_recurrence_b200 import inputs
+            w = workload(args.batch, args.seq)
+            x = inputs.make_scan_inputs(w.B, w.T, w.H, w.D, w.dtype, w.a_mean, w.seed, device=dev)
+            print(json.dumps({"fp8_forward": measure_fp8_forward(dev, x["a"], x["v"], x["q"], w.mode, dy=x["dy"]),
+                              "T": w.T}), flush=True)
         else:
             print(json.dumps({"fused_layer_forward": measure_fused(dev, seq=args.seq),
                               "layer_train_step": measure_layer(dev, seq=args.seq)}), flush=True)
