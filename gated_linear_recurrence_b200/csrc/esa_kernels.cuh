@@ -818,8 +818,13 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
 
   const ThreadPos<Cfg> pos(tid);
   // ghat of row r of this thread: in its q / dy slots, or (1-byte inputs) its own region.
+  // The separate region keeps row r as two halves of CT / 2 floats: the first
+  // four values of every thread's 8 channels, then the last four, so the
+  // 16-byte accesses of the eight lanes that share a row are contiguous.
   auto get_ghat_any = [&](int r, float2 (&g)[4]) {
-    if constexpr (Cfg::kSeparateScratch) get_ghat<float>(gh_s + r * CT + pos.ch, nullptr, g);
+    if constexpr (Cfg::kSeparateScratch)
+      get_ghat<__half>(reinterpret_cast<const __half *>(gh_s + r * CT + pos.ch / 2),
+                       reinterpret_cast<const __half *>(gh_s + r * CT + CT / 2 + pos.ch / 2), g);
     else get_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, g);
   };
   using TO = typename OutOf<T>::type;
@@ -938,7 +943,9 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
         float2 gh[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) gh[q] = mul2(splat(rr), fma2(nn[q], splat(-dot), dn[q]));
-        if constexpr (Cfg::kSeparateScratch) put_ghat<float>(gh_s + r * CT + pos.ch, nullptr, gh);
+        if constexpr (Cfg::kSeparateScratch)
+          put_ghat<__half>(reinterpret_cast<__half *>(gh_s + r * CT + pos.ch / 2),
+                           reinterpret_cast<__half *>(gh_s + r * CT + CT / 2 + pos.ch / 2), gh);
         else put_ghat<T>(q_s + r * CT + pos.ch, dy_s + r * CT + pos.ch, gh);
         if (!MAP && valid && (c0 + pos.ch) < sh.C)
           Io<TO>::store8(dqg + (static_cast<long>(b) * sh.T + t0 + r) * args.ldg + c0 + pos.ch, dqv);
