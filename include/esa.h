@@ -181,19 +181,50 @@ int esa_scan_bwd_ld(const void *a, const void *v, const void *q, long long ld_in
  *   - A shape whose esa_workspace_size() exceeds ESA_NOALLOC_SCRATCH_BYTES is
  *     rejected with ESA_ERR_NOALLOC_LIMIT before anything is enqueued (for
  *     example B=64, T=8192, C=128 in 16-bit I/O needs 33.6 MB and fits).
- *   - The first call on a device sets the array up with that device current
- *     (looks up its device address, zeroes it) and synchronises `stream`
- *     once; make that first call before any stream capture.
+ *     Other argument errors are reported as by esa_scan_fwd, also before
+ *     anything is enqueued.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current (once per device); make that first call before any
+ *     stream capture.  A cudaDeviceReset() invalidates the looked-up address:
+ *     do not use this entry point on a device after resetting it.
+ *   - Each call enqueues two kernels on `stream`: a one-block guard, then the
+ *     scan.  The guard initialises the array the first time it is used on a
+ *     device, and clears it and starts its call counter (the 32-bit epoch
+ *     that tags the chunk carries) afresh every 2^32 - 256 calls, so the
+ *     counter never runs out.  Those two cases take a fraction of a
+ *     millisecond; otherwise the guard only reads the array's header.
  *   - All calls share the one array, which keeps the last call's contents
- *     (the chunk carries are tagged with a per-call epoch, so nothing needs
- *     clearing between calls).  Calls whose executions overlap on the GPU,
- *     from any stream or thread, race on it: order them.  The chunk-end
- *     states it holds are not kept for a backward pass.
+ *     (the carries are tagged with the call's epoch, so nothing needs clearing
+ *     between calls).  Calls whose executions overlap on the GPU, from any
+ *     stream or thread, race on it: order them.  The chunk-end states it holds
+ *     are not kept for a backward pass.
+ *   - Device-side failures (a bounded wait inside the scan that gave up) are
+ *     recorded in the array and reported by esa_check_noalloc().
  */
 #define ESA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 int esa_scan_fwd_noalloc(const void *a, const void *v, const void *q, void *y, float *E_final,
                          int B, int T, int H, int D, int mode, const float *E_init,
                          int dtype, void *stream);
+
+/*
+ * Status of esa_scan_fwd_noalloc on the current device (no counterpart on the
+ * pages): synchronise `stream`, then read and clear the status recorded in
+ * the built-in array.  Returns ESA_OK (also when no call has used the array
+ * on this device yet), ESA_ERR_TIMEOUT if a bounded wait inside one of its
+ * scans gave up since the last check (that call's outputs are invalid), or
+ * ESA_ERR_LAUNCH if the stream reports a CUDA error.  Allocates nothing.
+ */
+int esa_check_noalloc(void *stream);
+
+/*
+ * Device address and size of the built-in array of esa_scan_fwd_noalloc on
+ * the current device (no counterpart on the pages), for inspection and
+ * tests: its first 256 bytes are the header esa_check reads, the rest the
+ * chunk carries.  Looks the address up if no call has done so yet (with the
+ * device current); `bytes` may be NULL.  Writing to the array other than
+ * through this library's calls leaves the results of later calls undefined.
+ */
+int esa_noalloc_scratch(void **device_ptr, size_t *bytes);
 
 /*
  * Segment maps, for splitting one sequence over several GPUs along time
