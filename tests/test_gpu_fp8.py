@@ -2,8 +2,7 @@
 
 a, v, q are e4m3 (torch.float8_e4m3fn); the state and the arithmetic are
 fp32 and y is fp16.  The oracle scans the same e4m3 values widened to fp64,
-so the comparison is the fp16 one (2e-3 (1 + |ref|) plus half an fp16 unit
-in the last place).  The backward takes e4m3 dy too and returns fp16 gradients;
+so the comparison is the fp16 one (2e-3 (1 + |ref|)).  The backward takes e4m3 dy too and returns fp16 gradients;
 the decode step takes e4m3 inputs and returns fp16; the fused forward does
 not take fp8 inputs and must say so.
 """
