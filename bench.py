@@ -54,6 +54,9 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sustained-s", type=float, default=1.2,
+                    help="length of the sustained run (detail.sustained; 0 = skip): steps back to back for at "
+                         "least this many seconds, after the burst timing, with its own clock record")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the prefill + decode (esa_step) measurement reported under detail.decode")
     ap.add_argument("--no-cp", action="store_true",
@@ -335,86 +338,105 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 
 def measure_decode(dev, reps=5):
-    """Prefill tokens/s and per-step decode time, eager and as a CUDA graph.
+    """Prefill, then decode, for each prompt length of the decode workload.
 
-    Each decode step moves B*C*(4s + 8) bytes (read a_t, v_t, q_t and the
+    Prefill: esa_scan_fwd over the prompt, L2 flushed (256 MB written) before
+    every launch, so the short prompts are read from HBM like the long ones;
+    algorithmic bytes 4 s C per token.  Decode: the workload's 256 one-token
+    steps after the prompt, timed three ways -- eagerly through ``esa_step``
+    (argument checks and pointer marshalling on every call), eagerly through
+    ``PreparedStep`` objects (one per step, arguments resolved up front, as a
+    decode loop over fixed buffers would hold them), and as one captured CUDA
+    graph.  Each step moves B C (4 s + 8) bytes (read a_t, v_t, q_t and the
     float32 state; write y_t and the state): 131 KB here, so a step is bound
-    by launch and latency, not by HBM; the graph removes the host launch cost.
+    by launch and latency, not by HBM.
     """
     import torch
 
     from gated_linear_recurrence_b200 import esa, inputs
     w = inputs.WORKLOADS["direct_f16_B64_H4_D32_prefill_decode"]
-    B, H, D, T, n = w.B, w.H, w.D, max(w.prompts), w.steps
-    x = inputs.make_scan_inputs(B, T, H, D, w.dtype, w.a_mean, w.seed, with_dy=False, device=dev)
-    g = x["generator"]
-    steps = [inputs.make_step_inputs(B, H, D, w.dtype, w.a_mean, generator=g, device=dev) for _ in range(n)]
-    y = torch.empty_like(x["a"])
-    Ef = torch.empty(B, H, D, dtype=torch.float32, device=dev)
-    ws = esa.new_workspace(B, T, H, D, x["a"].dtype, dev)
+    B, H, D, n = w.B, w.H, w.D, w.steps
     stream = torch.cuda.current_stream(dev)
+    peak, _ = measured_peak()
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    out = {"workload": w.name, "B": B, "H": H, "D": D, "mode": "direct", "io_dtype": w.dtype, "decode_steps": n,
+           "prompts": {}}
 
-    def prefill():
-        esa.esa_scan_fwd(x["a"], x["v"], x["q"], y=y, E_final=Ef, mode=w.mode, workspace=ws)
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
 
-    for _ in range(3):
-        prefill()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(reps):
-        prefill()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    prefill_ms = e0.elapsed_time(e1) / reps
-    esa.esa_check(ws)
+    # The first prompt length is measured twice and the first pass dropped:
+    # the first decode loops of a process run slower (host-side warm-up).
+    for T in (w.prompts[0],) + tuple(w.prompts):
+        x = inputs.make_scan_inputs(B, T, H, D, w.dtype, w.a_mean, w.seed, with_dy=False, device=dev)
+        g = x["generator"]
+        steps = [inputs.make_step_inputs(B, H, D, w.dtype, w.a_mean, generator=g, device=dev) for _ in range(n)]
+        y = torch.empty_like(x["a"])
+        Ef = torch.empty(B, H, D, dtype=torch.float32, device=dev)
+        ws = esa.new_workspace(B, T, H, D, x["a"].dtype, dev)
+        s = x["a"].element_size()
+        times = []
+        for k in range(reps + 3):
+            flush.fill_(k & 0xff)
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            esa.esa_scan_fwd(x["a"], x["v"], x["q"], y=y, E_final=Ef, mode=w.mode, workspace=ws)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if k >= 3:
+                times.append(e0.elapsed_time(e1))
+        esa.esa_check(ws)
+        prefill_ms = statistics.median(times)
+        prefill_gbs = 4 * s * H * D * B * T / (prefill_ms / 1e3) / 1e9
 
-    E = Ef.clone()
-    ys = [torch.empty_like(st["a"]) for st in steps]
+        E = Ef.clone()
+        ys = [torch.empty_like(st["a"]) for st in steps]
+        prepared = [esa.PreparedStep(st["a"], st["v"], st["q"], E, y_t=yt, mode=w.mode) for st, yt in zip(steps, ys)]
 
-    def decode():
-        for st, yt in zip(steps, ys):
-            esa.esa_step(st["a"], st["v"], st["q"], E, y_t=yt, mode=w.mode)
+        def decode():
+            for st, yt in zip(steps, ys):
+                esa.esa_step(st["a"], st["v"], st["q"], E, y_t=yt, mode=w.mode)
 
-    decode()   # warm-up (also fills the library's per-device caches before capture)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(reps):
-        decode()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    eager_us = 1e3 * e0.elapsed_time(e1) / (reps * n)
+        def decode_prepared():
+            for p_ in prepared:
+                p_()
 
-    graph = torch.cuda.CUDAGraph()
-    side = torch.cuda.Stream(dev)
-    side.wait_stream(stream)
-    with torch.cuda.stream(side):
-        decode()
-    stream.wait_stream(side)
-    torch.cuda.synchronize()
-    with torch.cuda.graph(graph):
-        decode()
-    graph.replay()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(reps):
-        graph.replay()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    graph_us = 1e3 * e0.elapsed_time(e1) / (reps * n)
-    del graph
+        def per_step_us(fn):
+            fn()   # warm-up
+            torch.cuda.synchronize()
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return 1e3 * e0.elapsed_time(e1) / (reps * n)
 
-    s = x["a"].element_size()
-    step_bytes = B * H * D * (4 * s + 8)
-    return {"workload": w.name, "B": B, "H": H, "D": D, "mode": "direct", "io_dtype": w.dtype,
-            "prefill_T": T, "prefill_ms": prefill_ms, "prefill_tokens_per_s": B * T / (prefill_ms / 1e3),
-            "prefill_GBs": 4 * s * H * D * B * T / (prefill_ms / 1e3) / 1e9,
-            "decode_steps": n, "bytes_per_step": step_bytes,
-            "eager_us_per_step": eager_us, "graph_us_per_step": graph_us,
-            "graph_tokens_per_s": B / (graph_us / 1e6),
-            "graph_GBs": step_bytes / (graph_us / 1e6) / 1e9,
-            "note": "decode steps are launch/latency bound (131 KB per step); eager time includes the "
-                    "Python binding's launch cost"}
+        eager_us = per_step_us(decode)
+        prepared_us = per_step_us(decode_prepared)
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            decode()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph):
+            decode()
+        graph_us = per_step_us(graph.replay)
+        del graph
+        step_bytes = B * H * D * (4 * s + 8)
+        out["prompts"][str(T)] = {
+            "prefill_ms": prefill_ms, "prefill_tokens_per_s": B * T / (prefill_ms / 1e3), "prefill_GBs": prefill_gbs,
+            "prefill_frac_of_measured_hbm": prefill_gbs / peak,
+            "eager_us_per_step": eager_us, "prepared_us_per_step": prepared_us, "graph_us_per_step": graph_us,
+            "graph_tokens_per_s": B / (graph_us / 1e6), "bytes_per_step": step_bytes}
+        del x, steps, y, ws, ys, prepared
+    del flush
+    torch.cuda.empty_cache()
+    out["note"] = ("prefill: L2 flushed before each launch; decode steps are launch/latency bound (131 KB per "
+                   "step); eager times include the Python binding's cost per call")
+    return out
 
 
 def measure_context_parallel(dev, n_slices=8, reps=5):
@@ -818,6 +840,7 @@ def measure_other_workloads(dev, reps=10):
                       "fwd_bwd_tokens_per_s": B * T / ((fwd_ms + bwd_ms) / 1e3),
                       "fwd_bwd_frac_of_measured_hbm": 11 * s_ * el / ((fwd_ms + bwd_ms) / 1e3) / 1e9 / peak})
         else:
+            r["fwd_frac_of_measured_hbm"] = r["fwd_GBs"] / peak
             r["note"] = "L2 flushed (256 MB written) before every iteration"
         out[name] = r
         del x, ws, y, g
@@ -973,6 +996,30 @@ def run_ours(args):
     achieved = dom_bytes / (dom_ms / 1e3) / 1e9
     step_gbs = (fwd_bytes + bwd_bytes) * K / (elapsed_ms / 1e3) / 1e9
 
+    # ---- sustained: the same step back to back for >= args.sustained_s ------
+    sustained = None
+    if args.sustained_s > 0:
+        n_sus = max(1, int(args.sustained_s * 1e3 / (elapsed_ms / K)) + 1)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clocks_s = ClockSampler(local).start()
+        barrier()
+        torch.cuda.synchronize()
+        s0.record(stream)
+        for _ in range(n_sus):
+            step()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        clk_s = clocks_s.stop()
+        esa.esa_check(ws)
+        sus_ms = max_over_ranks(s0.elapsed_time(s1), world, dev)
+        sustained = {"steps": n_sus, "seconds": sus_ms / 1e3, "ms_per_step": sus_ms / n_sus,
+                     "tokens_per_s": tokens_per_second(world, B, T, n_sus, sus_ms),
+                     "step_GBs": (fwd_bytes + bwd_bytes) * n_sus / (sus_ms / 1e3) / 1e9,
+                     "clocks": clk_s,
+                     "note": "the burst step back to back for over a second: the 1 kW power cap engages and "
+                             "lowers the SM clock"}
+
     # ---- end to end through the binding, with pinned host buffers ----------
     e2e = None
     if not args.no_e2e:
@@ -1010,11 +1057,11 @@ def run_ours(args):
                    "bwd_GBs": bwd_bytes / (bwd_ms / 1e3) / 1e9, "step_GBs": step_gbs,
                    "step_frac_of_measured_peak": step_gbs / peak, "step_frac_of_nominal_8TBs":
                    step_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes_per_step": fwd_bytes + bwd_bytes,
-                   "decode": decode, "context_parallel": cpar, "fused_layer_forward": fusedm, "layer_train_step": layerm,
+                   "sustained": sustained, "decode": decode, "context_parallel": cpar, "fused_layer_forward": fusedm, "layer_train_step": layerm,
                    "fp8_forward": fp8m, "other_workloads": otherm, "cpu_baseline_all_cores": cpu_all},
         "clocks": clk,
         "e2e": e2e,
-        "gpu_launches": 2 * K,
+        "gpu_launches": 2 * K,   # kernels of ours in the timed region (one forward, one backward per step)
         "cpu_baseline": cpu,
     }
     if rank == 0:

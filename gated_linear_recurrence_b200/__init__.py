@@ -11,6 +11,7 @@ from .esa import (  # noqa: F401
     DIRECT,
     EsaError,
     LIB_PATH,
+    PreparedStep,
     esa_check,
     esa_compose,
     esa_fused_fwd,
@@ -29,7 +30,7 @@ from .esa import (  # noqa: F401
 from .layer import ESA, esa_scan  # noqa: F401
 
 __all__ = [
-    "CONTROLLED", "DIRECT", "EsaError", "LIB_PATH", "esa_check", "esa_compose", "esa_fused_fwd", "esa_scan_bwd",
+    "CONTROLLED", "DIRECT", "EsaError", "LIB_PATH", "PreparedStep", "esa_check", "esa_compose", "esa_fused_fwd", "esa_scan_bwd",
     "esa_scan_bwd_map", "esa_scan_fwd", "esa_scan_map", "esa_step", "esa_strerror", "esa_version",
     "esa_workspace_init", "esa_workspace_size", "load_library", "new_workspace", "ESA", "esa_scan",
 ]

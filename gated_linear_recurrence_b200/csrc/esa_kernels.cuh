@@ -25,7 +25,10 @@
 //   * CTAs are persistent and software-pipelined: tiles are numbered by an
 //     atomic ticket (taken one tile ahead, chain as the fast index, so a
 //     tile's predecessor always belongs to a running CTA), and the TMA loads
-//     of the next tile are in flight while the current one is processed.
+//     of the next tile are in flight while the current one is processed.  A
+//     CTA takes its first ticket at its start and its second once its first
+//     tile's pass 1 is done, so a problem with fewer tiles than resident CTAs
+//     gives every CTA one tile.
 //     The last CTA to finish resets the ticket counter and advances the
 //     workspace epoch, so a call needs no separate reset launch.
 //     Every wait is bounded (iteration cap, then an error status).
@@ -37,8 +40,9 @@
 //     publishes its own (reverse) map at its first slot and skips the
 //     look-back, checkpoints, readout and outputs; a fold kernel then
 //     composes a chain's tile maps into the map of the whole slice.
-//   * fp8 (e4m3) inputs (forward only): 1-byte boxes are too small for the
-//     run-scan scratch, which gets its own region per stage.
+//   * fp8 (e4m3) inputs (both scans): 1-byte boxes are too small for the
+//     run-scan scratch, which gets its own region (per stage in the forward),
+//     and for the backward's ghat, which gets one too.
 #pragma once
 
 #include "esa_common.cuh"
@@ -350,33 +354,38 @@ __device__ __forceinline__ float head_sum2(float2 s) { return head_sum<LPH>(s.x 
 // `incl` and `agg`) whose chunk-end carry carries the current tag, with the
 // chunk maps of every tile in between applied oldest first -- the same fused
 // multiply-adds those tiles used for their own carries, so the value does not
-// depend on how far the search went.  Distances 1..4 are read in one round
-// trip; deeper searches walk one tile at a time.  Bounded: gives up (returns
-// 0, records a timeout, raises the abort flag) after kSpinLimit polls or when
-// another CTA raised the flag.
+// depend on how far the search went.  Predecessors are read four per round
+// trip; the search moves on past tiles that have published only their map,
+// and polls again (with back-off) where a tile has published neither.
+// Bounded: gives up (returns 0, records a timeout, raises the abort flag)
+// after kSpinLimit polls or when another CTA raised the flag.
 __device__ __forceinline__ float carry_in(const unsigned long long *incl, const ulonglong2 *agg, long me, long step,
                                        int avail, unsigned tag, unsigned *abort_flag, unsigned *status) {
   unsigned ns = 16;
+  int far = 0;    // distances 1..far have published their chunk maps and no carry
+  int polls = 0;  // rounds that found nothing new
   for (unsigned it = 0; it < kSpinLimit; ++it) {
     unsigned long long iw[4];
     ulonglong2 aw[4];
 #pragma unroll
     for (int d = 0; d < 4; ++d) {
-      if (d < avail) {
-        iw[d] = ld_relaxed_b64(&incl[me + (d + 1) * step]);
-        aw[d] = ld_relaxed_v2b64(&agg[me + (d + 1) * step]);
+      const long at = me + static_cast<long>(far + 1 + d) * step;
+      if (far + 1 + d <= avail) {
+        iw[d] = ld_relaxed_b64(&incl[at]);
+        aw[d] = ld_relaxed_v2b64(&agg[at]);
       } else {
         iw[d] = 0ull;
         aw[d] = make_ulonglong2(0ull, 0ull);
       }
     }
-    int found = -1;
+    int found = -1, maps = 0;
     bool blocked = false;
 #pragma unroll
     for (int d = 0; d < 4; ++d) {
-      if (found < 0 && !blocked && d < avail) {
+      if (found < 0 && !blocked && far + 1 + d <= avail) {
         if (tag_of(iw[d]) == tag) found = d;
-        else if (tag_of(aw[d].x) != tag || tag_of(aw[d].y) != tag) blocked = true;
+        else if (tag_of(aw[d].x) == tag && tag_of(aw[d].y) == tag) ++maps;
+        else blocked = true;
       }
     }
     if (found >= 0) {
@@ -384,35 +393,16 @@ __device__ __forceinline__ float carry_in(const unsigned long long *incl, const 
 #pragma unroll
       for (int d = 3; d >= 0; --d)
         if (d < found) E = __fmaf_rn(val_of(aw[d].x), E, val_of(aw[d].y));
+      for (int d = far; d >= 1; --d) {   // maps read in earlier rounds, oldest first
+        const ulonglong2 m = ld_relaxed_v2b64(&agg[me + static_cast<long>(d) * step]);
+        E = __fmaf_rn(val_of(m.x), E, val_of(m.y));
+      }
       return E;
     }
-    if (!blocked && avail > 4) {
-      // Four chunk maps in a row and no carry yet: walk further back.
-      int far = 4;   // distances 1..far have published maps
-      for (; it < kSpinLimit; ++it) {
-        const long at = me + static_cast<long>(far + 1) * step;
-        const unsigned long long w = ld_relaxed_b64(&incl[at]);
-        if (tag_of(w) == tag) {
-          float E = val_of(w);
-          for (int d = far; d >= 1; --d) {
-            const ulonglong2 m = ld_relaxed_v2b64(&agg[me + static_cast<long>(d) * step]);
-            E = __fmaf_rn(val_of(m.x), E, val_of(m.y));
-          }
-          return E;
-        }
-        const ulonglong2 m = ld_relaxed_v2b64(&agg[at]);
-        if (tag_of(m.x) == tag && tag_of(m.y) == tag && far + 1 < avail) {
-          ++far;
-          continue;
-        }
-        if ((it & 63u) == 63u && ld_relaxed(abort_flag)) break;
-        __nanosleep(ns);
-        ns = ns < 256 ? ns * 2 : 256;
-      }
-      break;
-    }
+    far += maps;
+    if (maps == 4) continue;   // four maps and no carry: read the next four at once
     if ((it & 63u) == 63u && ld_relaxed(abort_flag)) break;
-    if (it >= 2) {   // the first re-polls go straight out: a round trip is already ~1 us
+    if (++polls >= 2) {   // the first re-polls go straight out: a round trip is already ~1 us
       __nanosleep(ns);
       ns = ns < 256 ? ns * 2 : 256;
     }
@@ -536,10 +526,10 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     const unsigned tag = scan_prologue(hdr);
     *tag_s = tag;
     done_s[0] = done_s[1] = 0u;
-    const int t0 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[0], 1u)) : sh.ntiles;
-    const int t1 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[0], 1u)) : sh.ntiles;
-    issue(0, t0);
-    issue(1, t1);
+    // One ticket now; stage 1's is taken once the first tile's pass 1 is done,
+    // so that on a small problem every CTA holds a tile before any CTA takes a
+    // second one.
+    issue(0, tag ? static_cast<int>(atomicAdd(&hdr->ticket[0], 1u)) : sh.ntiles);
   }
   __syncthreads();
 
@@ -620,6 +610,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
       __syncthreads();
     }
     scan_store8<CT>(scan_s, pos.run, pos.ch, P, S);
+    if (it == 0 && tid == 0)   // stage 1's first tile (published to the CTA by the barrier below)
+      issue(1, tag ? static_cast<int>(atomicAdd(&hdr->ticket[0], 1u)) : sh.ntiles);
     __syncthreads();
 
     // ---- scan over runs, look-back, publish --------------------------------
@@ -808,11 +800,10 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     const unsigned tag = scan_prologue(hdr);
     *tag_s = tag;
     done_s[0] = done_s[1] = 0u;
+    // One ticket now, stage 1's after the first tile's F1 (see the forward).
     const int t0 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[1], 1u)) : sh.ntiles;
-    const int t1 = tag ? static_cast<int>(atomicAdd(&hdr->ticket[1], 1u)) : sh.ntiles;
     issue_av(0, t0);
     if (t0 < sh.ntiles) issue_qdy(info_s[0]);
-    issue_av(1, t1);
   }
   __syncthreads();
 
@@ -890,6 +881,8 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
       __syncthreads();
     }
     scan_store8<CT>(scan_s, pos.run, pos.ch, P, S);
+    if (it == 0 && tid == 0)   // stage 1's first tile (published to the CTA by the barrier below)
+      issue_av(1, tag ? static_cast<int>(atomicAdd(&hdr->ticket[1], 1u)) : sh.ntiles);
     __syncthreads();
     // The checkpoint carry goes in only now: every warp has left the previous
     // tile (whose B phase read the array) by the barrier above.

@@ -9,7 +9,8 @@ The functions carry the C names:
 
 * :func:`esa_scan_fwd`  -- forward scan (+ E_final, + checkpoints in the workspace)
 * :func:`esa_scan_bwd`  -- backward scan (da, dv, dq, dE_init)
-* :func:`esa_step`      -- one-token decode update (in place on E)
+* :func:`esa_step`      -- one-token decode update (in place on E); :class:`PreparedStep`
+  is the same call on fixed buffers with its arguments resolved once (decode loops)
 * :func:`esa_scan_map`, :func:`esa_scan_bwd_map` -- forward / backward segment
   maps ``(P, S)`` of a time slice (context parallelism)
 * :func:`esa_compose`   -- apply a sequence of segment maps to a state
@@ -496,6 +497,52 @@ def esa_step(a_t, v_t, q_t, E, y_t=None, mode=CONTROLLED, stream=None):
     if rc != 0:
         raise EsaError("esa_step", rc)
     return y_t
+
+
+class PreparedStep:
+    """``esa_step`` on fixed buffers, with the argument checks, the device
+    pointers and the stream resolved once, at construction.
+
+    A decode loop usually writes each new token's a_t, v_t, q_t into the same
+    buffers (the projections' outputs) and keeps one state E; for it each
+    call of this object is a single C call with prebuilt arguments, which
+    removes most of the host cost of :func:`esa_step` (the kernel itself
+    moves a few hundred KB at most and is launch-bound).  Work is enqueued on
+    the stream given here, or on the stream that was current at construction;
+    the buffers must outlive the object.  Calling it returns ``y_t``.
+    """
+
+    def __init__(self, a_t, v_t, q_t, E, y_t=None, mode=CONTROLLED, stream=None):
+        if not isinstance(a_t, torch.Tensor) or not a_t.is_cuda or a_t.dim() != 3:
+            raise TypeError("a_t must be a CUDA tensor [B, H, D] (the ESA library has no CPU path)")
+        if a_t.dtype not in _DTYPE_CODE or not a_t.is_contiguous():
+            raise ValueError("a_t must be contiguous with dtype float32, float16, bfloat16 or float8_e4m3fn")
+        B, H, D = (int(s) for s in a_t.shape)
+        for name, t in (("v_t", v_t), ("q_t", q_t)):
+            if t.shape != a_t.shape or t.dtype != a_t.dtype or t.device != a_t.device or not t.is_contiguous():
+                raise ValueError(f"{name} must match a_t")
+        if E is None:
+            raise ValueError("E (the recurrent state) is required")
+        _check_state("E", E, B, H, D, a_t.device)
+        if y_t is None:
+            y_t = torch.empty(a_t.shape, dtype=out_dtype(a_t.dtype), device=a_t.device)
+        if tuple(y_t.shape) != tuple(a_t.shape) or y_t.dtype != out_dtype(a_t.dtype) or \
+                y_t.device != a_t.device or not y_t.is_contiguous():
+            raise ValueError(f"y_t must be a contiguous {out_dtype(a_t.dtype)} tensor of shape {tuple(a_t.shape)}")
+        self.device = a_t.device
+        self.y_t = y_t
+        self._keep = (a_t, v_t, q_t, E, y_t)   # the buffers stay alive as long as this object
+        self._fn = load_library().esa_step
+        self._args = (_ptr(a_t), _ptr(v_t), _ptr(q_t), _ptr(E), _ptr(y_t), B, H, D, int(mode),
+                      _DTYPE_CODE[a_t.dtype], _stream(a_t.device, stream))
+        if self.device.index is not None and self.device.index != torch.cuda.current_device():
+            raise ValueError("make the tensors' device current before preparing and calling the step")
+
+    def __call__(self):
+        rc = self._fn(*self._args)
+        if rc != 0:
+            raise EsaError("esa_step", rc)
+        return self.y_t
 
 
 def esa_check(workspace, stream=None):

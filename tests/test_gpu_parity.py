@@ -183,3 +183,26 @@ def test_workload_prefill_then_256_decode_steps(cuda_device):
         assert_close(y, y_ref[:, :T], tol, f"prefill T={T} y")
         assert_close(torch.stack(ys, dim=1), y_ref[:, T:], tol, f"decode after T={T} y")
         assert_close(E, E_ref, tol, f"decode after T={T} E")
+
+
+def test_prepared_step_matches_esa_step_and_the_oracle(cuda_device):
+    """PreparedStep (arguments resolved once) is the same C call as esa_step:
+    bitwise-equal outputs and state, and both match the oracle's step."""
+    B, H, D = 8, 4, 32
+    g = torch.Generator().manual_seed(77)
+    E0 = inputs.make_state(B, H, D, seed=78).to(cuda_device)
+    E1, E2 = E0.clone(), E0.clone()
+    E_ref = host64(E0)
+    bufs = {k: torch.empty(B, H, D, dtype=torch.float16, device=cuda_device) for k in ("a", "v", "q")}
+    step = esa.PreparedStep(bufs["a"], bufs["v"], bufs["q"], E2, mode=esa.CONTROLLED)
+    for t in range(5):
+        s = inputs.make_step_inputs(B, H, D, "f16", 1.0, generator=g)
+        for k in ("a", "v", "q"):
+            bufs[k].copy_(s[k])
+        y1 = esa.esa_step(bufs["a"], bufs["v"], bufs["q"], E1, mode=esa.CONTROLLED)
+        y2 = step()
+        torch.cuda.synchronize()
+        assert torch.equal(y1, y2) and torch.equal(E1, E2), t
+        y_ref, E_ref = oracle.step(host64(s["a"]), host64(s["v"]), host64(s["q"]), E_ref, esa.CONTROLLED)
+        assert_close(y2, y_ref, TOL[torch.float16], f"prepared y[{t}]")
+        assert_close(E2, E_ref, TOL[torch.float16], f"prepared E[{t}]")
