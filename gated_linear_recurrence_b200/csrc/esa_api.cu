@@ -144,9 +144,11 @@ int make_tmap(CUtensorMap *map, const void *ptr, int dtype, int B, int T, int C,
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(lo.CT), static_cast<cuuint32_t>(rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   std::memset(map, 0, sizeof(*map));
+  // L2 promotion of 128 bytes, the row of a 64-channel 16-bit box: 256-byte
+  // promotion was 2% slower on the fwd + bwd step (interleaved A/B on B200).
   const CUresult r = fn(map, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ESA_OK : ESA_ERR_LAUNCH;
 }
 
