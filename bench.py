@@ -114,7 +114,7 @@ def measured_peak():
 # geometry and instantiation.  A profile summary's traffic applies while they
 # are unchanged.
 SCAN_KERNEL_SOURCES = ("esa_kernels.cuh", "esa_common.cuh", "esa_dispatch.cuh", "esa_launchers.cuh",
-                       "esa_launch.h", "esa_fwd.cu", "esa_bwd.cu")
+                       "esa_launch.h", "esa_fwd.cu", "esa_bwd.cu", "esa_api.cu")   # esa_api.cu: tensor maps
 
 
 def source_hash():
