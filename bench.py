@@ -70,6 +70,9 @@ def parse_args(argv=None):
                          "segment maps) instead of giving every rank its own batch: strong scaling")
     ap.add_argument("--cp-only", action="store_true",
                     help="run only the context-parallel phase timing (one JSON line; for profiling its kernels)")
+    ap.add_argument("--shape-sweep", action="store_true",
+                    help="only time fwd + bwd over head dimensions 8..256 and the three float dtypes (C = 512, "
+                         "B = 16, T = 16384, controlled) and print one JSON line of fractions of the measured peak")
     ap.add_argument("--fp8-only", action="store_true",
                     help="run only the fp8 (e4m3) forward + backward timing against fp16 on the workload's inputs "
                          "(one JSON line; for profiling its kernels; --seq shortens the sequence)")
@@ -792,6 +795,52 @@ def measure_fp8_forward(dev, a, v, q, mode, reps=10, dy=None):
     return out
 
 
+def measure_shape_sweep(dev, reps=10):
+    """fwd + bwd time and HBM fraction for every head dimension the library
+    takes (8 ... 256) and the three float dtypes, at C = 512 channels,
+    B = 16, T = 16384 (controlled mode, gate logits ~ N(3, 1)): inputs of
+    134-268 MB per tensor, larger than the L2, so no flush.  Algorithmic
+    bytes 4 s C (fwd) and 7 s C (bwd) per token."""
+    import torch
+
+    from gated_linear_recurrence_b200 import esa, inputs
+    stream = torch.cuda.current_stream(dev)
+    peak, _ = measured_peak()
+    B, T, C = 16, 16384, 512
+    out = []
+    for dt in ("f16", "bf16", "f32"):
+        for D in (8, 16, 32, 64, 128, 256):
+            H = C // D
+            x = inputs.make_scan_inputs(B, T, H, D, dt, 3.0, 11, device=dev)
+            ws = esa.new_workspace(B, T, H, D, x["a"].dtype, dev)
+            y = torch.empty_like(x["a"])
+            g = [torch.empty_like(x["a"]) for _ in range(3)]
+            fwd_t = bwd_t = 0.0
+            for k in range(reps + 3):
+                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                e0.record(stream)
+                esa.esa_scan_fwd(x["a"], x["v"], x["q"], y=y, mode=1, workspace=ws, want_E_final=False)
+                e1.record(stream)
+                esa.esa_scan_bwd(x["a"], x["v"], x["q"], x["dy"], ws, mode=1, da=g[0], dv=g[1], dq=g[2],
+                                 want_dE_init=False)
+                e2.record(stream)
+                torch.cuda.synchronize()
+                if k >= 3:
+                    fwd_t += e0.elapsed_time(e1)
+                    bwd_t += e1.elapsed_time(e2)
+            esa.esa_check(ws)
+            fwd_ms, bwd_ms = fwd_t / reps, bwd_t / reps
+            s_ = x["a"].element_size()
+            el = B * T * C
+            out.append({"dtype": dt, "D": D, "H": H, "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
+                        "fwd_frac": round(4 * s_ * el / (fwd_ms / 1e3) / 1e9 / peak, 3),
+                        "bwd_frac": round(7 * s_ * el / (bwd_ms / 1e3) / 1e9 / peak, 3),
+                        "fwd_bwd_frac": round(11 * s_ * el / ((fwd_ms + bwd_ms) / 1e3) / 1e9 / peak, 3)})
+            del x, ws, y, g
+            torch.cuda.empty_cache()
+    return {"B": B, "T": T, "C": C, "mode": "controlled", "peak_GBs": peak, "shapes": out}
+
+
 def measure_other_workloads(dev, reps=10):
     """The two other throughput workloads of the specification, device-timed:
     controlled bf16 B=64 T=4096 H=8 D=64 (C=512), forward + backward, inputs
@@ -1079,12 +1128,14 @@ def main(argv=None):
         return run_reference(args)
     if args.context_parallel:
         return run_context_parallel(args)
-    if args.cp_only or args.fused_only or args.fp8_only:
+    if args.cp_only or args.fused_only or args.fp8_only or args.shape_sweep:
         import torch
         dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
         torch.cuda.set_device(dev)
         if args.cp_only:
             print(json.dumps({"context_parallel": measure_context_parallel(dev)}), flush=True)
+        elif args.shape_sweep:
+            print(json.dumps({"shape_sweep": measure_shape_sweep(dev)}), flush=True)
         elif args.fp8_only:
             from gated_linear_recurrence_b200 import inputs
             w = workload(args.batch, args.seq)
