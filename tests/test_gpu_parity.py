@@ -38,6 +38,9 @@ SMALL = [
     (1, 20000, 1, 32, 1, "f16", 4.0, True),    # one long chain: 313 chunks of look-back
     (4, 64, 8, 64, 1, "bf16", 3.0, True),      # exactly one chunk
     (2, 129, 4, 32, 0, "f32", 0.0, False),     # fp32 chunks of 32 + 1
+    (2, 3000, 2, 128, 1, "f16", 4.0, True),    # D = 128: 128-row forward tiles over 24 chunks, ragged tail
+    (1, 2500, 1, 128, 0, "bf16", 2.0, True),   # D = 128 direct: one chain of 20 forward tiles
+    (1, 1100, 1, 256, 1, "f16", 3.0, True),    # D = 256: 64-row tiles, one chain of 18 chunks
 ]
 
 
