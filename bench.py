@@ -528,7 +528,7 @@ def measure_context_parallel(dev, n_slices=8, reps=5):
             "note": "one GPU: per-rank device time of every phase; the all-gathers are not included"}
 
 
-def measure_fused(dev, reps=10, seq=None):
+def measure_fused(dev, reps=10, seq=None, shape=None):
     """The layer's forward from its input: projections + scan.
 
     Same shape as the benchmark workload (B = 64, T = 65536, H = 4, D = 32,
@@ -546,6 +546,8 @@ def measure_fused(dev, reps=10, seq=None):
     from gated_linear_recurrence_b200 import esa
     w = workload(seq=seq)
     B, T, H, D, mode = w.B, w.T, w.H, w.D, w.mode
+    if shape is not None:   # (B, T, H, D) of a wider layer, C_in = C = H D
+        B, T, H, D = shape
     C = H * D
     C_in = C
     g = torch.Generator(device=dev).manual_seed(w.seed + 11)
@@ -597,7 +599,8 @@ def measure_fused(dev, reps=10, seq=None):
         "fused_frac_of_measured_hbm": fb / (out["fused_ms"] / 1e3) / 1e9 / peak,
         "fused_avq_GBs": fb_avq / (out["fused_avq_ms"] / 1e3) / 1e9,
         "fused_tensor_TFLOPs": 2 * 3 * C * C_in * tok / (out["fused_ms"] / 1e3) / 1e12,
-        "note": "fused kernel: one CTA per SM, two tile groups of 256 threads, weights resident in shared memory"})
+        "note": "fused kernel: one CTA per SM, " + ("two tile groups" if C_in <= 128 else "one tile group") +
+                " of 256 threads, weights resident in shared memory"})
     del x, W, y, avq, ws
     torch.cuda.empty_cache()
     return out
@@ -1084,6 +1087,7 @@ def run_ours(args):
     fusedm = layerm = fp8m = otherm = None
     if not args.no_fused and args.batch is None and args.seq is None:
         fusedm = measure_fused(dev)
+        fusedm["cin256"] = measure_fused(dev, shape=(16, 65536, 8, 32))
         layerm = measure_layer(dev)
         fp8m = measure_fp8_forward(dev, a, v, q, mode, dy=dy)
         otherm = measure_other_workloads(dev)

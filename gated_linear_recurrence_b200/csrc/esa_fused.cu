@@ -1,5 +1,5 @@
 // esa_fused.cu -- instantiations and launcher of the fused projection + scan
-// forward kernel (16-bit I/O, head dimension <= 64, C_in of 64 or 128).
+// forward kernel (16-bit I/O, head dimension <= 64, C_in of 64, 128 or 256).
 #include "esa_dispatch.cuh"
 #include "esa_fused.cuh"
 #include "esa_fused_launch.h"
@@ -18,7 +18,8 @@ int run_fused(const CUtensorMap &tx, const CUtensorMap &tw, const CUtensorMap *t
   if (cudaGetDevice(&dev) != cudaSuccess) return -5;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return -5;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 512, smem) != cudaSuccess) return -5;
+  constexpr int kThreads = Pl::NG * Pl::NTG;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) != cudaSuccess) return -5;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -5;
   if (per_sm < 1 || sms < 1) return -5;
   // Every CTA must be resident at once (tiles wait on their predecessors):
@@ -28,7 +29,7 @@ int run_fused(const CUtensorMap &tx, const CUtensorMap &tw, const CUtensorMap *t
   const int need = (args.ntiles_ct + Pl::NG - 1) / Pl::NG;
   if (per_ct > need) per_ct = need;
   if (per_ct < 1) return -5;
-  kern<<<dim3(per_ct, nct), 512, smem, stream>>>(tx, tw, tavq[0], tavq[1], tavq[2], args);
+  kern<<<dim3(per_ct, nct), kThreads, smem, stream>>>(tx, tw, tavq[0], tavq[1], tavq[2], args);
   return launch_status(cudaGetLastError());
 }
 
@@ -38,6 +39,7 @@ int by_cin(int cin, const CUtensorMap &tx, const CUtensorMap &tw, const CUtensor
   switch (cin) {
     case 64: return run_fused<T, MODE, LPH, 64>(tx, tw, tavq, args, st);
     case 128: return run_fused<T, MODE, LPH, 128>(tx, tw, tavq, args, st);
+    case 256: return run_fused<T, MODE, LPH, 256>(tx, tw, tavq, args, st);
     default: return -3;
   }
 }

@@ -12,7 +12,7 @@
 // forward scan kernel.  HBM traffic per token is C_in + C elements instead
 // of 4 C (plus the projection's own 3 C writes and C_in reads).
 //
-// Organisation (one CTA per SM, 512 threads):
+// Organisation (one CTA per SM, 512 threads; 256 for C_in = 256):
 //   * The CTA serves one channel tile ct (blockIdx.y) and keeps that tile's
 //     weight slice resident in shared memory (3 x 64 rows x C_in, loaded
 //     once by TMA with the 128-byte swizzle the MMA reads).
@@ -20,7 +20,9 @@
 //     each has its own x buffer, a/v/q boxes, barriers and 256 columns of
 //     tensor memory, and runs its own persistent loop over tiles taken from
 //     the channel tile's ticket counter (batch row fastest), so the two
-//     groups hide each other's latencies as two CTAs per SM would.
+//     groups hide each other's latencies as two CTAs per SM would.  With
+//     C_in = 256 the weight slice (96 KB) and one group's x buffer (64 KB)
+//     leave room for one group only.
 //   * Per tile: one thread takes the next tile's ticket (the atomic's result
 //     is used only after the read-out, so its round trip is hidden), issues
 //     C_in / 16 MMAs of 128 x 192 x 16 on the tile's x rows and commits them
@@ -54,7 +56,8 @@ struct FusedArgs {
 
 template <typename T, int CIN>
 struct FusedPlan {
-  static constexpr int L = 128, CT = 64, K = 4, SUB = 2, NG = 2, NTG = 256;
+  static constexpr int L = 128, CT = 64, K = 4, SUB = 2, NTG = 256;
+  static constexpr int NG = CIN <= 128 ? 2 : 1;   // tile groups per CTA
   static constexpr int KB = CIN / 64;                          // 128-byte k-blocks
   static constexpr size_t kXkb = size_t(L) * 128;             // one k-block of x: 16 KB
   static constexpr size_t kWkb = size_t(3 * CT) * 128;        // one k-block of W: 24 KB
@@ -64,7 +67,7 @@ struct FusedPlan {
   static constexpr size_t kMisc = 4096;                        // es_s, seg_s, barriers, infos
   static constexpr size_t kGroup = kX + 3 * kBox + kMisc;
   static constexpr size_t kBytes = kW + NG * kGroup + 1024 /*CTA misc*/ + 1024 /*alignment*/;
-  static_assert(CIN % 64 == 0 && CIN >= 64 && CIN <= 128, "C_in of 64 or 128");
+  static_assert(CIN % 64 == 0 && CIN >= 64 && CIN <= 256, "C_in of 64, 128 or 256");
   static_assert(kW % 1024 == 0 && kX % 1024 == 0 && kGroup % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static_assert(kBytes <= 227 * 1024, "shared memory");
 };
@@ -100,7 +103,7 @@ __device__ __forceinline__ void pack32(const uint32_t (&v)[32], uint4 (&out)[4])
 }
 
 template <typename T, int MODE, int LPH, int CIN>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(FusedPlan<T, CIN>::NG * 256, 1)
     esa_fused_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                          const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
                          const __grid_constant__ CUtensorMap tm_q, const FusedArgs args) {
@@ -174,7 +177,7 @@ __global__ void __launch_bounds__(512, 1)
     fence_mbar_init();
   }
   if (threadIdx.x < 32) {   // warp 0 allocates the CTA's tensor memory: 256 columns per group
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, Pl::NG * 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -417,7 +420,7 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   if (threadIdx.x < 32) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc(tmem_base, Pl::NG * 256);
   }
   if (threadIdx.x == 0) {
     __threadfence();

@@ -10,9 +10,10 @@
 namespace esa {
 
 // Shapes the fused kernel takes: 16-bit I/O, channel tiles of 64 (head
-// dimension <= 64), C_in of 64 or 128, at most kMaxChannelTickets channel tiles.
+// dimension <= 64), C_in of 64, 128 or 256, at most kMaxChannelTickets channel tiles.
 inline bool fused_supported(int dtype, int D, int cin, int nct) {
-  return (dtype == 1 || dtype == 2) && D <= 64 && (cin == 64 || cin == 128) && nct <= kMaxChannelTickets;
+  return (dtype == 1 || dtype == 2) && D <= 64 && (cin == 64 || cin == 128 || cin == 256) &&
+         nct <= kMaxChannelTickets;
 }
 
 // tx: x [B][T][C_in] in boxes of [128 rows][64 elements], 128-byte swizzle;

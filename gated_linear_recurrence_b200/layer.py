@@ -225,7 +225,7 @@ class ESA(torch.nn.Module):
         dt = self.W_A.weight.dtype
         return (x.is_cuda and self.cp_group is None and self.W_A.bias is None and dt in (torch.float16, torch.bfloat16)
                 and x.dtype == dt and self.scan_dtype in (None, dt) and self.head_dim <= 64
-                and self.embd in (64, 128) and -(-self.embd // 64) <= 48)
+                and self.embd in (64, 128, 256) and -(-self.embd // 64) <= 48)
 
     def forward(self, x, state=None, return_state=False):
         B, T, C = x.shape

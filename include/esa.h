@@ -297,7 +297,7 @@ int esa_compose(const float *P, const float *S, int n, long long count, int reve
  *             the same workspace gives the scan's gradients.  Without them
  *             the call only reads x and W and writes y (inference, prefill).
  *   y, E_final, E_init, mode, workspace: as for esa_scan_fwd.
- * Supported: dtype ESA_F16 or ESA_BF16, D <= 64, C_in of 64 or 128, C <= 3072;
+ * Supported: dtype ESA_F16 or ESA_BF16, D <= 64, C_in of 64, 128 or 256, C <= 3072;
  * other shapes return ESA_ERR_UNSUPPORTED (compute the projections
  * separately and call esa_scan_fwd).
  */

@@ -35,6 +35,8 @@ CASES = [
     (2, 257, 5, 16, 128, 0, "bf16"),     # C = 80: a partial second channel tile
     (2, 4100, 4, 32, 128, 1, "bf16"),
     (1, 129, 6, 64, 64, 1, "f16"),       # six channel tiles
+    (2, 700, 8, 32, 256, 1, "f16"),      # C_in = 256: one tile group per CTA, four channel tiles
+    (1, 300, 4, 64, 256, 0, "bf16"),     # C_in = 256, D = 64
 ]
 
 
@@ -155,7 +157,7 @@ def _random_fused_cases(n, seed=20261203):
     while len(cases) < n:
         D = int(rng.choice([8, 16, 32, 64]))
         H = int(rng.integers(1, 9))
-        C_in = int(rng.choice([64, 128]))
+        C_in = int(rng.choice([64, 128, 256]))
         B = int(rng.integers(1, 4))
         T = int(rng.choice([1, 127, 128, 129, 255, 256, 700])) if rng.random() < 0.5 else int(rng.integers(1, 2000))
         if B * T * H * D > 800_000:
