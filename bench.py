@@ -757,31 +757,31 @@ def measure_fp8_forward(dev, a, v, q, mode, reps=10, dy=None):
     ws = esa.new_workspace(B, T, H, D, torch.float8_e4m3fn, dev)
     stream = torch.cuda.current_stream(dev)
     out = {}
-    for name, args in (("fp8", (a8, v8, q8)), ("fp16", (a, v, q))):
+    runs = (("fp8", (a8, v8, q8), dy8), ("fp16", (a, v, q), dy))
+    # fp8 and fp16 alternate rep by rep, so that the GPU's warming (and the
+    # power cap engaging) weighs on both alike.
+    for _, args, _ in runs:
         for _ in range(3):
             esa.esa_scan_fwd(*args, y=y, mode=mode, workspace=ws, want_E_final=False)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(reps):
+    tot = {name: [0.0, 0.0] for name, _, _ in runs}
+    for k in range(reps + 2):
+        for name, args, dyx in runs:
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0.record(stream)
             esa.esa_scan_fwd(*args, y=y, mode=mode, workspace=ws, want_E_final=False)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        out[name + "_fwd_ms"] = e0.elapsed_time(e1) / reps
-        if dy is not None:   # backward on the same workspace (the forward just wrote its chunk states)
-            dyx = dy8 if name == "fp8" else dy
-            e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            tot = 0.0
-            for k in range(reps + 2):
-                esa.esa_scan_fwd(*args, y=y, mode=mode, workspace=ws, want_E_final=False)
-                e2.record(stream)
+            e1.record(stream)
+            if dy is not None:   # backward on the same workspace (the forward just wrote its chunk states)
                 esa.esa_scan_bwd(*args, dyx, ws, mode=mode, da=grads[0], dv=grads[1], dq=grads[2],
                                  want_dE_init=False)
-                e3.record(stream)
-                torch.cuda.synchronize()
-                if k >= 2:
-                    tot += e2.elapsed_time(e3)
-            out[name + "_bwd_ms"] = tot / reps
+            e2.record(stream)
+            torch.cuda.synchronize()
+            if k >= 2:
+                tot[name][0] += e0.elapsed_time(e1)
+                tot[name][1] += e1.elapsed_time(e2)
+    for name, _, _ in runs:
+        out[name + "_fwd_ms"] = tot[name][0] / reps
+        if dy is not None:
+            out[name + "_bwd_ms"] = tot[name][1] / reps
     esa.esa_check(ws)
     el = B * T * H * D
     peak, _ = measured_peak()
