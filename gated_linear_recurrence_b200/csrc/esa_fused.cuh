@@ -238,6 +238,7 @@ __global__ void __launch_bounds__(FusedPlan<T, CIN>::NG * 256, 1)
     const int chunk = ti.chunk, b = ti.b, c0 = ti.c0, t0 = ti.t0;
     const long slot = ti.slot;
     const long slot_end = slot + SUB - 1;
+    const bool full = t0 + L <= sh.T && c0 + CT <= sh.C;
 
     // ---- projections on the tensor cores -----------------------------------
     unsigned nt_raw = 0;
@@ -322,23 +323,25 @@ __global__ void __launch_bounds__(FusedPlan<T, CIN>::NG * 256, 1)
     float2 P[4], S[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) { P[q] = splat(1.0f); S[q] = splat(0.0f); }
+    with_full(full, [&](auto kf) {
 #pragma unroll
-    for (int i = 0; i < K; ++i) {
-      const int r = pos.row0 + i;
-      const bool valid = (t0 + r) < sh.T;
-      float2 x[4], vv[4];
-      Io<T>::load8_gate(a_s + r * CT + 8 * box_vec(pos.vec, r), x);
-      Io<T>::load8(v_s + r * CT + 8 * box_vec(pos.vec, r), vv);
+      for (int i = 0; i < K; ++i) {
+        const int r = pos.row0 + i;
+        const bool valid = decltype(kf)::value || (t0 + r) < sh.T;
+        float2 x[4], vv[4];
+        Io<T>::load8_gate(a_s + r * CT + 8 * box_vec(pos.vec, r), x);
+        Io<T>::load8(v_s + r * CT + 8 * box_vec(pos.vec, r), vv);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const Gate2 gt = gate2(x[q]);
-        Ar[i][q] = gate_coef<MODE>(gt);
-        if (valid) {
-          P[q] = mul2(P[q], gt.A);
-          S[q] = rec_step<MODE>(Ar[i][q], S[q], vv[q]);
+        for (int q = 0; q < 4; ++q) {
+          const Gate2 gt = gate2(x[q]);
+          Ar[i][q] = gate_coef<MODE>(gt);
+          if (valid) {
+            P[q] = mul2(P[q], gt.A);
+            S[q] = rec_step<MODE>(Ar[i][q], S[q], vv[q]);
+          }
         }
       }
-    }
+    });
     // The scan scratch overwrites the a box: with the projections being
     // stored, the whole group waits until the TMA store has read it.
     if (store_avq) {
@@ -384,27 +387,30 @@ __global__ void __launch_bounds__(FusedPlan<T, CIN>::NG * 256, 1)
     {
       float2 E[4];
       run_carry<CT>(scan_s, es_s, pos.run, pos.ch, E);
-      const bool ch_ok = (c0 + pos.ch) < sh.C;
       const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
+      with_full(full, [&](auto kf) {
+        constexpr bool kFull = decltype(kf)::value;
+        const bool ch_ok = kFull || (c0 + pos.ch) < sh.C;
 #pragma unroll
-      for (int i = 0; i < K; ++i) {
-        const int r = pos.row0 + i;
-        const bool valid = (t0 + r) < sh.T;
-        float2 vv[4], qq[4];
-        Io<T>::load8(v_s + r * CT + 8 * box_vec(pos.vec, r), vv);
-        Io<T>::load8(q_s + r * CT + 8 * box_vec(pos.vec, r), qq);
-        float2 ss = splat(0.0f);
+        for (int i = 0; i < K; ++i) {
+          const int r = pos.row0 + i;
+          const bool valid = kFull || (t0 + r) < sh.T;
+          float2 vv[4], qq[4];
+          Io<T>::load8(v_s + r * CT + 8 * box_vec(pos.vec, r), vv);
+          Io<T>::load8(q_s + r * CT + 8 * box_vec(pos.vec, r), qq);
+          float2 ss = splat(0.0f);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          E[q] = rec_step<MODE>(Ar[i][q], E[q], vv[q]);
-          ss = fma2(E[q], E[q], ss);
+          for (int q = 0; q < 4; ++q) {
+            E[q] = rec_step<MODE>(Ar[i][q], E[q], vv[q]);
+            ss = fma2(E[q], E[q], ss);
+          }
+          const float rr = rsqrt_approx(__fmaf_rn(head_sum2<LPH>(ss), sh.inv_D, kEps));
+          float2 yv[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) yv[q] = mul2(qq[q], mul2(E[q], splat(rr)));
+          if (valid && ch_ok) Io<T>::store8(yg + gbase + static_cast<long>(r) * sh.C, yv);
         }
-        const float rr = rsqrt_approx(__fmaf_rn(head_sum2<LPH>(ss), sh.inv_D, kEps));
-        float2 yv[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) yv[q] = mul2(qq[q], mul2(E[q], splat(rr)));
-        if (valid && ch_ok) Io<T>::store8(yg + gbase + static_cast<long>(r) * sh.C, yv);
-      }
+      });
     }
     try_issue_next();
     named_sync(bar_all, Pl::NTG);   // boxes, scratch and carries are free for the next tile

@@ -45,6 +45,8 @@
 //     and for the backward's ghat, which gets one too.
 #pragma once
 
+#include <type_traits>
+
 #include "esa_common.cuh"
 
 namespace esa {
@@ -468,6 +470,17 @@ __device__ __forceinline__ float2 rec_step(float2 c, float2 E, float2 v) {
 template <int MODE>
 __device__ __forceinline__ float2 gate_A(float2 c) { return MODE == 0 ? c : sub2(splat(1.0f), c); }
 
+// Run a tile phase with its fullness as a compile-time flag: f(true_type) when
+// every row of the tile lies inside the sequence and every channel inside C
+// (all tiles but a chain's ragged last one and a ragged last channel tile),
+// so that the phase's per-row and per-channel checks fold away; else
+// f(false_type).
+template <typename F>
+__device__ __forceinline__ void with_full(bool full, F &&f) {
+  if (full) f(std::true_type{});
+  else f(std::false_type{});
+}
+
 // ===========================================================================
 // Forward scan (persistent).  A tile of L rows covers SUB workspace slots:
 // it publishes its chunk map and reads its predecessors' at its last slot,
@@ -550,6 +563,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     const T *a_s = box(s, 0);
     const T *v_s = box(s, 1);
     const T *q_s = box(s, 2);
+    const bool full = t0 + L <= sh.T && c0 + CT <= sh.C;
     // Run-scan scratch: the gate box once pass 1 is done (its own region for 1-byte inputs).
     float *scan_s = reinterpret_cast<float *>(box(s, Cfg::kSeparateScratch ? 3 : 0));
 
@@ -583,23 +597,25 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     float2 P[4], S[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) { P[q] = splat(1.0f); S[q] = splat(0.0f); }
+    with_full(full, [&](auto kf) {
 #pragma unroll
-    for (int i = 0; i < K; ++i) {
-      const int r = pos.row0 + i;
-      const bool valid = (t0 + r) < sh.T;
-      float2 x[4], vv[4];
-      Io<T>::load8_gate(a_s + r * CT + pos.ch, x);
-      Io<T>::load8(v_s + r * CT + pos.ch, vv);
+      for (int i = 0; i < K; ++i) {
+        const int r = pos.row0 + i;
+        const bool valid = decltype(kf)::value || (t0 + r) < sh.T;
+        float2 x[4], vv[4];
+        Io<T>::load8_gate(a_s + r * CT + pos.ch, x);
+        Io<T>::load8(v_s + r * CT + pos.ch, vv);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const Gate2 g = gate2(x[q]);
-        Ar[i][q] = gate_coef<MODE>(g);
-        if (valid) {
-          P[q] = mul2(P[q], g.A);
-          S[q] = rec_step<MODE>(Ar[i][q], S[q], vv[q]);
+        for (int q = 0; q < 4; ++q) {
+          const Gate2 g = gate2(x[q]);
+          Ar[i][q] = gate_coef<MODE>(g);
+          if (valid) {
+            P[q] = mul2(P[q], g.A);
+            S[q] = rec_step<MODE>(Ar[i][q], S[q], vv[q]);
+          }
         }
       }
-    }
+    });
     // The gate rows are free from here on (only this warp read its own rows).
     // A separate scratch region needs no wait: its last readers (pass 2 of
     // this stage's previous tile) finished before the stage was refilled.
@@ -675,27 +691,30 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     if constexpr (!MAP) {
       float2 E[4];
       run_carry<CT>(scan_s, es_s, pos.run, pos.ch, E);
-      const bool ch_ok = (c0 + pos.ch) < sh.C;
       const long gbase = (static_cast<long>(b) * sh.T + t0) * sh.C + c0 + pos.ch;
+      with_full(full, [&](auto kf) {
+        constexpr bool kFull = decltype(kf)::value;
+        const bool ch_ok = kFull || (c0 + pos.ch) < sh.C;
 #pragma unroll
-      for (int i = 0; i < K; ++i) {
-        const int r = pos.row0 + i;
-        const bool valid = (t0 + r) < sh.T;
-        float2 vv[4], qq[4];
-        Io<T>::load8(v_s + r * CT + pos.ch, vv);
-        Io<T>::load8(q_s + r * CT + pos.ch, qq);
-        float2 ss = splat(0.0f);
+        for (int i = 0; i < K; ++i) {
+          const int r = pos.row0 + i;
+          const bool valid = kFull || (t0 + r) < sh.T;
+          float2 vv[4], qq[4];
+          Io<T>::load8(v_s + r * CT + pos.ch, vv);
+          Io<T>::load8(q_s + r * CT + pos.ch, qq);
+          float2 ss = splat(0.0f);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          E[q] = rec_step<MODE>(Ar[i][q], E[q], vv[q]);
-          ss = fma2(E[q], E[q], ss);
+          for (int q = 0; q < 4; ++q) {
+            E[q] = rec_step<MODE>(Ar[i][q], E[q], vv[q]);
+            ss = fma2(E[q], E[q], ss);
+          }
+          const float rr = rsqrt_approx(__fmaf_rn(head_sum2<LPH>(ss), sh.inv_D, kEps));
+          float2 yv[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) yv[q] = mul2(qq[q], mul2(E[q], splat(rr)));
+          if (valid && ch_ok) Io<TO>::store8(yg + gbase + static_cast<long>(r) * sh.C, yv);
         }
-        const float rr = rsqrt_approx(__fmaf_rn(head_sum2<LPH>(ss), sh.inv_D, kEps));
-        float2 yv[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) yv[q] = mul2(qq[q], mul2(E[q], splat(rr)));
-        if (valid && ch_ok) Io<TO>::store8(yg + gbase + static_cast<long>(r) * sh.C, yv);
-      }
+      });
     }
 
     // ---- refill this stage --------------------------------------------------
