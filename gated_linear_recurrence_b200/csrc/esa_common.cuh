@@ -75,18 +75,18 @@ __device__ __forceinline__ float val_of(unsigned long long w) {
 // lanes per instruction, each lane rounded to nearest exactly like the
 // scalar instruction, so packing halves the float32 instruction count without
 // changing a single result bit.  A thread's 8 channels are 4 pairs (2i, 2i+1).
+// nvcc may still fuse a packed multiply with a packed add that consumes it
+// into one FFMA2 when both sit in one basic block (it did so across the rows
+// of the backward's reverse phases once their per-row branches were removed),
+// so values that must agree bit for bit between two code paths -- a tile's
+// published carry and the look-back's recomposition of it -- are formed with
+// explicit fused multiply-adds.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float2 splat(float a) { return make_float2(a, a); }
 
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
-__device__ __forceinline__ float2 sub2(float2 a, float2 b) {   // a - b, one packed instruction
-  unsigned long long ua, ub, ud;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(ua) : "f"(a.x), "f"(a.y));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(ub) : "f"(b.x), "f"(b.y));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(ud) : "l"(ua), "l"(ub));
-  float2 d;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(ud));
-  return d;
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {   // a - b: b * (-1) is exact, so one rounding
+  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
 }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
