@@ -328,16 +328,17 @@ __global__ void __launch_bounds__(FusedPlan<T, CIN>::NG * 256, 1)
       for (int i = 0; i < K; ++i) {
         const int r = pos.row0 + i;
         const bool valid = decltype(kf)::value || (t0 + r) < sh.T;
-        float2 x[4], vv[4];
+        float2 x[4];
+        VRow<T, MODE> vr;
         Io<T>::load8_gate(a_s + r * CT + 8 * box_vec(pos.vec, r), x);
-        Io<T>::load8(v_s + r * CT + 8 * box_vec(pos.vec, r), vv);
+        vr.load(v_s + r * CT + 8 * box_vec(pos.vec, r));
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const Gate2 gt = gate2(x[q]);
           Ar[i][q] = gate_coef<MODE>(gt);
           if (valid) {
             P[q] = mul2(P[q], gt.A);
-            S[q] = rec_step<MODE>(Ar[i][q], S[q], vv[q]);
+            S[q] = vr.step(q, Ar[i][q], S[q]);
           }
         }
       }
@@ -395,13 +396,14 @@ __global__ void __launch_bounds__(FusedPlan<T, CIN>::NG * 256, 1)
         for (int i = 0; i < K; ++i) {
           const int r = pos.row0 + i;
           const bool valid = kFull || (t0 + r) < sh.T;
-          float2 vv[4], qq[4];
-          Io<T>::load8(v_s + r * CT + 8 * box_vec(pos.vec, r), vv);
+          float2 qq[4];
+          VRow<T, MODE> vr;
+          vr.load(v_s + r * CT + 8 * box_vec(pos.vec, r));
           Io<T>::load8(q_s + r * CT + 8 * box_vec(pos.vec, r), qq);
           float2 ss = splat(0.0f);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            E[q] = rec_step<MODE>(Ar[i][q], E[q], vv[q]);
+            E[q] = vr.step(q, Ar[i][q], E[q]);
             ss = fma2(E[q], E[q], ss);
           }
           const float rr = rsqrt_approx(__fmaf_rn(head_sum2<LPH>(ss), sh.inv_D, kEps));

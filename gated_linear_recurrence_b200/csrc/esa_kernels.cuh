@@ -466,6 +466,42 @@ __device__ __forceinline__ float2 rec_step(float2 c, float2 E, float2 v) {
   return MODE == 0 ? fma2(c, E, v) : fma2(c, sub2(v, E), E);
 }
 
+// One row's 8 values of v in the form the recurrence consumes: widened to
+// float32 pairs on load, or -- 16-bit inputs in controlled mode -- kept packed,
+// with v - E formed by sm_100's mixed-precision subtraction, which widens v
+// exactly inside the instruction (the same value as widening first, one
+// conversion instruction fewer per value).
+template <typename T, int MODE>
+struct VRow {
+  float2 f[4];
+  __device__ __forceinline__ void load(const T *p) { Io<T>::load8(p, f); }
+  __device__ __forceinline__ float2 minus(int q, float2 E) const { return sub2(f[q], E); }   // v - E
+  __device__ __forceinline__ float2 step(int q, float2 c, float2 E) const { return rec_step<MODE>(c, E, f[q]); }
+};
+
+template <typename T>
+struct VRow16 {
+  uint4 u;
+  __device__ __forceinline__ void load(const T *p) { u = *reinterpret_cast<const uint4 *>(p); }
+  __device__ __forceinline__ float2 minus(int q, float2 E) const {
+    const uint32_t w = q == 0 ? u.x : q == 1 ? u.y : q == 2 ? u.z : u.w;
+    unsigned short lo, hi;
+    asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(w));
+    float dx, dy;
+    if constexpr (std::is_same<T, __half>::value) {
+      asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(dx) : "h"(lo), "f"(E.x));
+      asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(dy) : "h"(hi), "f"(E.y));
+    } else {
+      asm("sub.rn.f32.bf16 %0, %1, %2;" : "=f"(dx) : "h"(lo), "f"(E.x));
+      asm("sub.rn.f32.bf16 %0, %1, %2;" : "=f"(dy) : "h"(hi), "f"(E.y));
+    }
+    return make_float2(dx, dy);
+  }
+  __device__ __forceinline__ float2 step(int q, float2 c, float2 E) const { return fma2(c, minus(q, E), E); }
+};
+template <> struct VRow<__half, 1> : VRow16<__half> {};
+template <> struct VRow<__nv_bfloat16, 1> : VRow16<__nv_bfloat16> {};
+
 // A of the pair from its stored coefficient.
 template <int MODE>
 __device__ __forceinline__ float2 gate_A(float2 c) { return MODE == 0 ? c : sub2(splat(1.0f), c); }
@@ -602,16 +638,17 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
       for (int i = 0; i < K; ++i) {
         const int r = pos.row0 + i;
         const bool valid = decltype(kf)::value || (t0 + r) < sh.T;
-        float2 x[4], vv[4];
+        float2 x[4];
+        VRow<T, MODE> vr;
         Io<T>::load8_gate(a_s + r * CT + pos.ch, x);
-        Io<T>::load8(v_s + r * CT + pos.ch, vv);
+        vr.load(v_s + r * CT + pos.ch);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const Gate2 g = gate2(x[q]);
           Ar[i][q] = gate_coef<MODE>(g);
           if (valid) {
             P[q] = mul2(P[q], g.A);
-            S[q] = rec_step<MODE>(Ar[i][q], S[q], vv[q]);
+            S[q] = vr.step(q, Ar[i][q], S[q]);
           }
         }
       }
@@ -699,13 +736,14 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
         for (int i = 0; i < K; ++i) {
           const int r = pos.row0 + i;
           const bool valid = kFull || (t0 + r) < sh.T;
-          float2 vv[4], qq[4];
-          Io<T>::load8(v_s + r * CT + pos.ch, vv);
+          float2 qq[4];
+          VRow<T, MODE> vr;
+          vr.load(v_s + r * CT + pos.ch);
           Io<T>::load8(q_s + r * CT + pos.ch, qq);
           float2 ss = splat(0.0f);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            E[q] = rec_step<MODE>(Ar[i][q], E[q], vv[q]);
+            E[q] = vr.step(q, Ar[i][q], E[q]);
             ss = fma2(E[q], E[q], ss);
           }
           const float rr = rsqrt_approx(__fmaf_rn(head_sum2<LPH>(ss), sh.inv_D, kEps));
@@ -875,16 +913,17 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     for (int i = 0; i < K; ++i) {
       const int r = pos.row0 + i;
       const bool valid = (t0 + r) < sh.T;
-      float2 x[4], vv[4];
+      float2 x[4];
+      VRow<T, MODE> vr;
       Io<T>::load8_gate(a_s + r * CT + pos.ch, x);
-      Io<T>::load8(v_s + r * CT + pos.ch, vv);
+      vr.load(v_s + r * CT + pos.ch);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const Gate2 g = gate2(x[q]);
         Ar[i][q] = gate_coef<MODE>(g);
         if (valid) {
           P[q] = mul2(P[q], g.A);
-          S[q] = rec_step<MODE>(Ar[i][q], S[q], vv[q]);
+          S[q] = vr.step(q, Ar[i][q], S[q]);
         }
       }
     }
@@ -930,15 +969,22 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
       for (int i = 0; i < K; ++i) {
         const int r = pos.row0 + i;
         const bool valid = (t0 + r) < sh.T;
-        float2 vv[4], qq[4], gg[4];
-        Io<T>::load8(v_s + r * CT + pos.ch, vv);
+        float2 qq[4], gg[4];
+        VRow<T, MODE> vr;
+        vr.load(v_s + r * CT + pos.ch);
         Io<T>::load8(q_s + r * CT + pos.ch, qq);
         Io<T>::load8(dy_s + r * CT + pos.ch, gg);
         float2 ss = splat(0.0f);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          Em[i][q] = (MODE == 0) ? E[q] : sub2(E[q], vv[q]);
-          E[q] = rec_step<MODE>(Ar[i][q], E[q], vv[q]);
+          if constexpr (MODE == 0) {
+            Em[i][q] = E[q];
+            E[q] = vr.step(q, Ar[i][q], E[q]);
+          } else {   // E_{t-1} - v_t = -(v_t - E_{t-1}): round to nearest is symmetric, so the same value
+            const float2 d = vr.minus(q, E[q]);
+            Em[i][q] = mul2(d, splat(-1.0f));
+            E[q] = fma2(Ar[i][q], d, E[q]);
+          }
           ss = fma2(E[q], E[q], ss);
         }
         const float rr = rsqrt_approx(__fmaf_rn(head_sum2<LPH>(ss), sh.inv_D, kEps));
