@@ -958,7 +958,7 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     // ---- F2: replay states, readout backward, dq, ghat ---------------------
     // ghat of each row overwrites that row's q/dy slots (only this thread
     // reads them again).  The factor of da that depends on the forward state,
-    // E_{t-1} - v_t (direct mode: E_{t-1}), stays in registers for B.
+    // v_t - E_{t-1} (direct mode: E_{t-1}), stays in registers for B.
     float2 Em[K][4];
     {
       float2 E[4];
@@ -980,9 +980,9 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
           if constexpr (MODE == 0) {
             Em[i][q] = E[q];
             E[q] = vr.step(q, Ar[i][q], E[q]);
-          } else {   // E_{t-1} - v_t = -(v_t - E_{t-1}): round to nearest is symmetric, so the same value
+          } else {   // kept as v_t - E_{t-1}: B folds the sign into -A (see there)
             const float2 d = vr.minus(q, E[q]);
-            Em[i][q] = mul2(d, splat(-1.0f));
+            Em[i][q] = d;
             E[q] = fma2(Ar[i][q], d, E[q]);
           }
           ss = fma2(E[q], E[q], ss);
@@ -1089,6 +1089,14 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
     if constexpr (!MAP) {
       float2 h[4];
       run_carry<CT>(scan_s, es_s, pos.run, pos.ch, h);
+      // Controlled mode keeps the carry negated (h = -A_{t+1} G_{t+1}) and
+      // forms -A = Ac - 1: with Em = v_t - E_{t-1} every sign cancels, and each
+      // value is the negation of -- so, rounding to nearest, bit for bit the
+      // same as -- the one the direct formula gives.
+      if constexpr (MODE == 1) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) h[q] = mul2(h[q], splat(-1.0f));
+      }
 #pragma unroll
       for (int i = K - 1; i >= 0; --i) {
         const int r = pos.row0 + i;
@@ -1097,12 +1105,19 @@ __global__ void __launch_bounds__(VPR *(L / K), (VPR * (L / K) <= 64) ? 8 : (VPR
           get_ghat_any(r, gh);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const float2 G = add2(gh[q], h[q]);
-            const float2 A = gate_A<MODE>(Ar[i][q]);
-            const float2 Ac = (MODE == 0) ? sub2(splat(1.0f), A) : Ar[i][q];
-            dvv[q] = (MODE == 0) ? G : mul2(G, Ac);
-            dav[q] = mul2(mul2(G, mul2(A, Ac)), Em[i][q]);
-            h[q] = mul2(A, G);
+            if constexpr (MODE == 0) {
+              const float2 G = add2(gh[q], h[q]);
+              const float2 A = Ar[i][q];
+              dvv[q] = G;
+              dav[q] = mul2(mul2(G, mul2(A, sub2(splat(1.0f), A))), Em[i][q]);
+              h[q] = mul2(A, G);
+            } else {
+              const float2 G = sub2(gh[q], h[q]);
+              const float2 nA = sub2(Ar[i][q], splat(1.0f));
+              dvv[q] = mul2(G, Ar[i][q]);
+              dav[q] = mul2(mul2(G, mul2(nA, Ar[i][q])), Em[i][q]);
+              h[q] = mul2(nA, G);
+            }
           }
           if (ch_ok) {
             Io<TO>::store8(dvg + gbase + static_cast<long>(r) * args.ldg, dvv);
