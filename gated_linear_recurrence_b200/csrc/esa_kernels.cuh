@@ -467,10 +467,10 @@ __device__ __forceinline__ float2 rec_step(float2 c, float2 E, float2 v) {
 }
 
 // One row's 8 values of v in the form the recurrence consumes: widened to
-// float32 pairs on load, or -- 16-bit inputs in controlled mode -- kept packed,
-// with v - E formed by sm_100's mixed-precision subtraction, which widens v
-// exactly inside the instruction (the same value as widening first, one
-// conversion instruction fewer per value).
+// float32 pairs on load, or -- 16-bit and 8-bit inputs in controlled mode --
+// kept as packed 16-bit pairs, with v - E formed by sm_100's mixed-precision
+// subtraction, which widens v exactly inside the instruction (the same value
+// as widening first, one conversion instruction fewer per value).
 template <typename T, int MODE>
 struct VRow {
   float2 f[4];
@@ -479,28 +479,53 @@ struct VRow {
   __device__ __forceinline__ float2 step(int q, float2 c, float2 E) const { return rec_step<MODE>(c, E, f[q]); }
 };
 
+// v - E for a pair of 16-bit values packed in one word (bf16 or fp16): the
+// mixed-precision subtraction widens each value exactly inside the instruction.
+template <bool kBf16>
+__device__ __forceinline__ float2 sub_mixed2(uint32_t w, float2 E) {
+  unsigned short lo, hi;
+  asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(w));
+  float dx, dy;
+  if constexpr (kBf16) {
+    asm("sub.rn.f32.bf16 %0, %1, %2;" : "=f"(dx) : "h"(lo), "f"(E.x));
+    asm("sub.rn.f32.bf16 %0, %1, %2;" : "=f"(dy) : "h"(hi), "f"(E.y));
+  } else {
+    asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(dx) : "h"(lo), "f"(E.x));
+    asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(dy) : "h"(hi), "f"(E.y));
+  }
+  return make_float2(dx, dy);
+}
+
 template <typename T>
 struct VRow16 {
   uint4 u;
   __device__ __forceinline__ void load(const T *p) { u = *reinterpret_cast<const uint4 *>(p); }
   __device__ __forceinline__ float2 minus(int q, float2 E) const {
     const uint32_t w = q == 0 ? u.x : q == 1 ? u.y : q == 2 ? u.z : u.w;
-    unsigned short lo, hi;
-    asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(w));
-    float dx, dy;
-    if constexpr (std::is_same<T, __half>::value) {
-      asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(dx) : "h"(lo), "f"(E.x));
-      asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(dy) : "h"(hi), "f"(E.y));
-    } else {
-      asm("sub.rn.f32.bf16 %0, %1, %2;" : "=f"(dx) : "h"(lo), "f"(E.x));
-      asm("sub.rn.f32.bf16 %0, %1, %2;" : "=f"(dy) : "h"(hi), "f"(E.y));
-    }
-    return make_float2(dx, dy);
+    return sub_mixed2<std::is_same<T, __nv_bfloat16>::value>(w, E);
   }
   __device__ __forceinline__ float2 step(int q, float2 c, float2 E) const { return fma2(c, minus(q, E), E); }
 };
 template <> struct VRow<__half, 1> : VRow16<__half> {};
 template <> struct VRow<__nv_bfloat16, 1> : VRow16<__nv_bfloat16> {};
+
+// e4m3 in controlled mode: each pair widens exactly to half precision (one
+// conversion), and v - E takes the mixed-precision subtraction from there.
+template <>
+struct VRow<__nv_fp8_e4m3, 1> {
+  uint32_t h[4];   // four half2
+  __device__ __forceinline__ void load(const __nv_fp8_e4m3 *p) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    const unsigned short *w = reinterpret_cast<const unsigned short *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2 t = Io<__nv_fp8_e4m3>::h2(w[i]);
+      h[i] = *reinterpret_cast<const uint32_t *>(&t);
+    }
+  }
+  __device__ __forceinline__ float2 minus(int q, float2 E) const { return sub_mixed2<false>(h[q], E); }
+  __device__ __forceinline__ float2 step(int q, float2 c, float2 E) const { return fma2(c, minus(q, E), E); }
+};
 
 // A of the pair from its stored coefficient.
 template <int MODE>
