@@ -23,7 +23,8 @@ that summarise a time slice and their composition:
 and the forward of the layer from its input:
 
 * :func:`project`      -- a, v, q as projections of x, rounded to the I/O type,
-* :func:`fused_fwd`    -- those projections followed by :func:`scan_fwd`.
+* :func:`fused_fwd`    -- those projections followed by :func:`scan_fwd`,
+* :func:`output_projection` -- the layer's output z = W_O y of the readout.
 
 Sources for each formula are given in the C file's header: the recurrence and
 its two modes ("entangled-state-attention 0.1.0", section "Core idea"), the
@@ -246,6 +247,17 @@ def project(x, W, io_dtype):
     for p in range(3):
         out.append(round_io(x @ W[p * C:(p + 1) * C].T, io_dtype))
     return tuple(out)
+
+
+def output_projection(y, W_O, io_dtype):
+    """The layer's output ("entangled-state-attention 0.1.0", section "Core
+    idea": y_t = W_O (q_t (.) Norm(E_t))): ``y`` [B, T, H, D] -- the readout as
+    the scan writes it, in the I/O type -- flattened to [B, T, C], times
+    ``W_O`` [C_out, C] ([out, in], as ``W``): z = y W_O^T in float64, rounded
+    to the I/O type.  Returns z as [B, T, C_out] float64."""
+    y = round_io(_f64(y), io_dtype)
+    B, T = y.shape[0], y.shape[1]
+    return round_io(y.reshape(B, T, -1) @ _f64(W_O).T, io_dtype)
 
 
 def fused_fwd(x, W, H, mode, io_dtype, E_init=None):

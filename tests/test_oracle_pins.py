@@ -424,6 +424,29 @@ def test_fused_forward_is_projection_then_scan():
     np.testing.assert_array_equal(Ef, Ef2)
 
 
+def test_output_projection_hand_example_and_special_cases():
+    # C = 2, C_out = 2: z_o = sum_c W_O[o, c] y_c, so y = (1, 0) picks W_O's first column
+    y = np.array([[[[1.0, 0.0]]]])                  # [B=1, T=1, H=1, D=2]
+    W_O = np.array([[1.0, 2.0], [3.0, 4.0]])
+    np.testing.assert_array_equal(oracle.output_projection(y, W_O, "f32").ravel(), [1.0, 3.0])
+    y = np.array([[[[0.0, 1.0]]]])
+    np.testing.assert_array_equal(oracle.output_projection(y, W_O, "f32").ravel(), [2.0, 4.0])
+    r = np.random.default_rng(43)
+    yr = r.normal(0, 1, (2, 5, 2, 4))
+    flat = oracle.round_io(yr, "f16").reshape(2, 5, 8)
+    # identity: the rounded readout itself; a permutation: its channels permuted
+    np.testing.assert_array_equal(oracle.output_projection(yr, np.eye(8), "f16"), flat)
+    perm = r.permutation(8)
+    np.testing.assert_array_equal(oracle.output_projection(yr, np.eye(8)[perm], "f16"), flat[..., perm])
+    # C_out may differ from C, and heads are flattened head-major (channel h D + d)
+    W2 = np.zeros((3, 8))
+    W2[0, 5] = 1.0                                  # head 1, channel 1
+    z = oracle.output_projection(yr, W2, "f16")
+    assert z.shape == (2, 5, 3)
+    np.testing.assert_array_equal(z[..., 0], oracle.round_io(yr[:, :, 1, 1], "f16"))
+    np.testing.assert_array_equal(z[..., 1:], 0.0)
+
+
 # ---------------------------------------------------------------------------
 # The only printed worked examples are shapes.
 # ---------------------------------------------------------------------------
