@@ -15,6 +15,7 @@ from .esa import (  # noqa: F401
     esa_check,
     esa_compose,
     esa_fused_fwd,
+    esa_fused_layer_fwd,
     esa_scan_bwd,
     esa_scan_bwd_map,
     esa_scan_fwd,
@@ -30,7 +31,7 @@ from .esa import (  # noqa: F401
 from .layer import ESA, esa_scan  # noqa: F401
 
 __all__ = [
-    "CONTROLLED", "DIRECT", "EsaError", "LIB_PATH", "PreparedStep", "esa_check", "esa_compose", "esa_fused_fwd", "esa_scan_bwd",
+    "CONTROLLED", "DIRECT", "EsaError", "LIB_PATH", "PreparedStep", "esa_check", "esa_compose", "esa_fused_fwd", "esa_fused_layer_fwd", "esa_scan_bwd",
     "esa_scan_bwd_map", "esa_scan_fwd", "esa_scan_map", "esa_step", "esa_strerror", "esa_version",
     "esa_workspace_init", "esa_workspace_size", "load_library", "new_workspace", "ESA", "esa_scan",
 ]

@@ -222,6 +222,66 @@ int scan_bwd_impl(const void *a, const void *v, const void *q, long long ld_in, 
                   int T, int H, int D, int mode, const float *E_init, int dtype, void *workspace,
                   size_t workspace_bytes, void *stream);
 
+// The fused forward, with (out = true) or without the output projection.
+int fused_impl(const void *x, const void *W, const void *W_O, void *z, void *y, float *E_final, void *a, void *v,
+               void *q, int B, int T, int H, int D, int C_in, int mode, const float *E_init, int dtype,
+               void *workspace, size_t workspace_bytes, void *stream, bool out = false) {
+  int rc = check_shape(B, T, H, D, mode, dtype);
+  if (rc) return rc;
+  if (C_in < 1) return ESA_ERR_ARG;
+  Layout lo;
+  if (!make_layout(B, T, H, D, dtype, &lo)) return ESA_ERR_ARG;
+  if (!esa::fused_supported(dtype, D, C_in, lo.nct)) return ESA_ERR_UNSUPPORTED;
+  const int C = H * D;
+  if (out && !esa::fused_out_supported(dtype, C, C_in)) return ESA_ERR_UNSUPPORTED;
+  const bool has_tokens = B > 0 && T > 0;
+  if (has_tokens && (!x || !W || (!y && !out))) return ESA_ERR_ARG;
+  if ((a == nullptr) != (v == nullptr) || (a == nullptr) != (q == nullptr)) return ESA_ERR_ARG;
+  for (const void *p : {x, W, W_O, static_cast<const void *>(z), static_cast<const void *>(y),
+                        static_cast<const void *>(E_final), static_cast<const void *>(a),
+                        static_cast<const void *>(v), static_cast<const void *>(q),
+                        static_cast<const void *>(E_init), static_cast<const void *>(workspace)})
+    if (p && !aligned16(p)) return ESA_ERR_ALIGN;
+  if (!workspace || workspace_bytes < lo.total) return ESA_ERR_WORKSPACE;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (B == 0) return ESA_OK;
+  if (T == 0) {
+    if (!E_final) return ESA_OK;
+    const size_t bytes = static_cast<size_t>(B) * C * sizeof(float);
+    return E_init ? rt(cudaMemcpyAsync(E_final, E_init, bytes, cudaMemcpyDeviceToDevice, st))
+                  : rt(cudaMemsetAsync(E_final, 0, bytes, st));
+  }
+  CUtensorMap tx, tw, two;
+  const cuuint64_t xdims[3] = {static_cast<cuuint64_t>(C_in), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
+  const cuuint64_t wdims[2] = {static_cast<cuuint64_t>(C_in), static_cast<cuuint64_t>(3) * C};
+  if ((rc = make_tmap_sw128(&tx, x, dtype, 3, xdims, 128))) return rc;
+  if ((rc = make_tmap_sw128(&tw, W, dtype, 2, wdims, 64))) return rc;
+  if (out) {
+    const cuuint64_t odims[2] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(C)};   // W_O [C_out = C][C]
+    if ((rc = make_tmap_sw128(&two, W_O, dtype, 2, odims, 64))) return rc;
+  }
+  CUtensorMap tavq[3] = {tx, tx, tx};   // placeholders when the projections are not stored
+  if (a != nullptr) {
+    const cuuint64_t pdims[3] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
+    const void *outs[3] = {a, v, q};
+    for (int i = 0; i < 3; ++i)
+      if ((rc = make_tmap_sw128(&tavq[i], outs[i], dtype, 3, pdims, 128))) return rc;
+  }
+  esa::FusedArgs args;
+  args.s = scan_shape(B, T, H, D, lo, 2);
+  args.ntiles_ct = B * args.s.nchunks;
+  args.y = y;
+  args.E_final = E_final;
+  args.E_init = E_init;
+  args.a_out = a;
+  args.v_out = v;
+  args.q_out = q;
+  args.z = z;
+  args.ws = workspace_view(workspace, lo);
+  return esa::launch_fused_fwd(dtype, mode, D, C_in, tx, tw, tavq, out ? &two : nullptr, args, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -442,53 +502,16 @@ int esa_compose(const float *P, const float *S, int n, long long count, int reve
 int esa_fused_fwd(const void *x, const void *W, void *y, float *E_final, void *a, void *v, void *q, int B, int T,
                   int H, int D, int C_in, int mode, const float *E_init, int dtype, void *workspace,
                   size_t workspace_bytes, void *stream) {
-  int rc = check_shape(B, T, H, D, mode, dtype);
-  if (rc) return rc;
-  if (C_in < 1) return ESA_ERR_ARG;
-  Layout lo;
-  if (!make_layout(B, T, H, D, dtype, &lo)) return ESA_ERR_ARG;
-  if (!esa::fused_supported(dtype, D, C_in, lo.nct)) return ESA_ERR_UNSUPPORTED;
-  const bool has_tokens = B > 0 && T > 0;
-  if (has_tokens && (!x || !W || !y)) return ESA_ERR_ARG;
-  if ((a == nullptr) != (v == nullptr) || (a == nullptr) != (q == nullptr)) return ESA_ERR_ARG;
-  for (const void *p : {x, W, static_cast<const void *>(y), static_cast<const void *>(E_final),
-                        static_cast<const void *>(a), static_cast<const void *>(v), static_cast<const void *>(q),
-                        static_cast<const void *>(E_init), static_cast<const void *>(workspace)})
-    if (p && !aligned16(p)) return ESA_ERR_ALIGN;
-  if (!workspace || workspace_bytes < lo.total) return ESA_ERR_WORKSPACE;
-  if ((rc = check_device())) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int C = H * D;
-  if (B == 0) return ESA_OK;
-  if (T == 0) {
-    if (!E_final) return ESA_OK;
-    const size_t bytes = static_cast<size_t>(B) * C * sizeof(float);
-    return E_init ? rt(cudaMemcpyAsync(E_final, E_init, bytes, cudaMemcpyDeviceToDevice, st))
-                  : rt(cudaMemsetAsync(E_final, 0, bytes, st));
-  }
-  CUtensorMap tx, tw;
-  const cuuint64_t xdims[3] = {static_cast<cuuint64_t>(C_in), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
-  const cuuint64_t wdims[2] = {static_cast<cuuint64_t>(C_in), static_cast<cuuint64_t>(3) * C};
-  if ((rc = make_tmap_sw128(&tx, x, dtype, 3, xdims, 128))) return rc;
-  if ((rc = make_tmap_sw128(&tw, W, dtype, 2, wdims, 64))) return rc;
-  CUtensorMap tavq[3] = {tx, tx, tx};   // placeholders when the projections are not stored
-  if (a != nullptr) {
-    const cuuint64_t pdims[3] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
-    const void *outs[3] = {a, v, q};
-    for (int i = 0; i < 3; ++i)
-      if ((rc = make_tmap_sw128(&tavq[i], outs[i], dtype, 3, pdims, 128))) return rc;
-  }
-  esa::FusedArgs args;
-  args.s = scan_shape(B, T, H, D, lo, 2);
-  args.ntiles_ct = B * args.s.nchunks;
-  args.y = y;
-  args.E_final = E_final;
-  args.E_init = E_init;
-  args.a_out = a;
-  args.v_out = v;
-  args.q_out = q;
-  args.ws = workspace_view(workspace, lo);
-  return esa::launch_fused_fwd(dtype, mode, D, C_in, tx, tw, tavq, args, st);
+  return fused_impl(x, W, nullptr, nullptr, y, E_final, a, v, q, B, T, H, D, C_in, mode, E_init, dtype, workspace,
+                    workspace_bytes, stream);
+}
+
+int esa_fused_layer_fwd(const void *x, const void *W, const void *W_O, void *z, void *y, float *E_final, int B,
+                        int T, int H, int D, int C_in, int mode, const float *E_init, int dtype, void *workspace,
+                        size_t workspace_bytes, void *stream) {
+  if (B > 0 && T > 0 && (!W_O || !z)) return ESA_ERR_ARG;
+  return fused_impl(x, W, W_O ? W_O : W, z, y, E_final, nullptr, nullptr, nullptr, B, T, H, D, C_in, mode, E_init,
+                    dtype, workspace, workspace_bytes, stream, true);
 }
 
 int esa_step(const void *a_t, const void *v_t, const void *q_t, float *E, void *y_t, int B, int H, int D,

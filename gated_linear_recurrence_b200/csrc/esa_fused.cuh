@@ -51,10 +51,11 @@ struct FusedArgs {
   float *E_final;
   const float *E_init;
   void *a_out, *v_out, *q_out;   // the rounded projections [B][T][C], or all null
+  void *z;                       // the layer's output z = y W_O^T [B][T][64] (output-projection kernels only)
   Workspace ws;
 };
 
-template <typename T, int CIN>
+template <typename T, int CIN, bool WO = false>
 struct FusedPlan {
   static constexpr int L = 128, CT = 64, K = 4, SUB = 2, NTG = 256;
   static constexpr int NG = CIN <= 128 ? 2 : 1;   // tile groups per CTA
@@ -66,7 +67,9 @@ struct FusedPlan {
   static constexpr size_t kBox = size_t(L) * CT * sizeof(T);  // one of a / v / q
   static constexpr size_t kMisc = 4096;                        // es_s, seg_s, barriers, infos
   static constexpr size_t kGroup = kX + 3 * kBox + kMisc;
-  static constexpr size_t kBytes = kW + NG * kGroup + 1024 /*CTA misc*/ + 1024 /*alignment*/;
+  // W_O [64 out][64 in], resident with the weight slice (output-projection kernels).
+  static constexpr size_t kWO = WO ? size_t(64) * 128 : 0;
+  static constexpr size_t kBytes = kW + NG * kGroup + 1024 /*CTA misc*/ + kWO + 1024 /*alignment*/;
   static_assert(CIN % 64 == 0 && CIN >= 64 && CIN <= 256, "C_in of 64, 128 or 256");
   static_assert(kW % 1024 == 0 && kX % 1024 == 0 && kGroup % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static_assert(kBytes <= 227 * 1024, "shared memory");
@@ -102,12 +105,13 @@ __device__ __forceinline__ void pack32(const uint32_t (&v)[32], uint4 (&out)[4])
   }
 }
 
-template <typename T, int MODE, int LPH, int CIN>
-__global__ void __launch_bounds__(FusedPlan<T, CIN>::NG * 256, 1)
+template <typename T, int MODE, int LPH, int CIN, bool WO>
+__global__ void __launch_bounds__(FusedPlan<T, CIN, WO>::NG * 256, 1)
     esa_fused_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                          const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_v,
-                         const __grid_constant__ CUtensorMap tm_q, const FusedArgs args) {
-  using Pl = FusedPlan<T, CIN>;
+                         const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_wo,
+                         const FusedArgs args) {
+  using Pl = FusedPlan<T, CIN, WO>;
   constexpr int L = Pl::L, CT = Pl::CT, K = Pl::K, SUB = Pl::SUB, KB = Pl::KB;
   constexpr int SW = scan_segments<L / K, Pl::NTG, CT>();
   using Cfg = TileCfg<T, LPH, 8, L, K, SW>;
@@ -115,6 +119,10 @@ __global__ void __launch_bounds__(FusedPlan<T, CIN>::NG * 256, 1)
   static_assert(Cfg::NT == Pl::NTG, "a tile group is one scan block");
   static_assert(Cfg::kBoxBytes == Pl::kBox, "box size");
   constexpr uint32_t kIdesc = umma_idesc_f16(std::is_same<T, __half>::value ? 0 : 1, 128, 3 * CT);
+  // Output projection: M = 128 rows of y, N = 64 outputs, into accumulator
+  // columns 3 CT .. 4 CT - 1 (the projections use the first 3 CT).
+  constexpr uint32_t kIdescWO = umma_idesc_f16(std::is_same<T, __half>::value ? 0 : 1, 128, 64);
+  static_assert(!WO || CT == 64, "the output projection needs the whole row of y in one channel tile");
 
   extern __shared__ unsigned char smem_raw[];
   unsigned char *base = smem_aligned1024(smem_raw);
@@ -132,12 +140,13 @@ __global__ void __launch_bounds__(FusedPlan<T, CIN>::NG * 256, 1)
   unsigned char *misc = grp + Pl::kX + 3 * Pl::kBox;
   float *es_s = reinterpret_cast<float *>(misc);                          // CT floats
   float4 *seg_s = reinterpret_cast<float4 *>(misc + 256);                 // SW x NP
-  uint64_t *bar = reinterpret_cast<uint64_t *>(misc + 256 + SW * NP * 16); // [0] x full, [1] mma done
-  TileInfo *info_s = reinterpret_cast<TileInfo *>(bar + 2);               // [2]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(misc + 256 + SW * NP * 16); // [0] x full, [1] mma done, [2] W_O mma done
+  TileInfo *info_s = reinterpret_cast<TileInfo *>(bar + 3);               // [2]
   unsigned *tag_s = reinterpret_cast<unsigned *>(info_s + 2);
   unsigned char *cta_misc = base + Pl::kW + Pl::NG * Pl::kGroup;
   uint64_t *w_bar = reinterpret_cast<uint64_t *>(cta_misc);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cta_misc + 8);
+  unsigned char *wo_s = cta_misc + 1024;   // W_O (output-projection kernels), 1024-byte aligned
 
   const ScanShape &sh = args.s;
   const Workspace &ws = args.ws;
@@ -174,6 +183,7 @@ __global__ void __launch_bounds__(FusedPlan<T, CIN>::NG * 256, 1)
   if (tid == 0) {
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);
+    mbar_init(&bar[2], 1);
     fence_mbar_init();
   }
   if (threadIdx.x < 32) {   // warp 0 allocates the CTA's tensor memory: 256 columns per group
@@ -187,7 +197,8 @@ __global__ void __launch_bounds__(FusedPlan<T, CIN>::NG * 256, 1)
   const uint32_t tmem_d = tmem_base + static_cast<uint32_t>(g * 256);
 
   if (threadIdx.x == 0) {   // the channel tile's weight slice: rows p C + ct CT + [0, 64) of W
-    mbar_expect_tx(w_bar, static_cast<unsigned>(Pl::kW));
+    mbar_expect_tx(w_bar, static_cast<unsigned>(Pl::kW + Pl::kWO));
+    if constexpr (WO) tma_load_2d(wo_s, &tm_wo, 0, 0, w_bar);
 #pragma unroll
     for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
@@ -208,6 +219,7 @@ __global__ void __launch_bounds__(FusedPlan<T, CIN>::NG * 256, 1)
   T *yg = static_cast<T *>(args.y);
   const unsigned tag = *tag_s;
   unsigned ph_x = 0, ph_m = 0;   // ph_x: the group's thread 0 only
+  unsigned ph_o = 0;             // the output projection's barrier
   bool pre = false;              // thread 0: the current tile's MMAs were issued during the previous tile
   bool next_ok = false;          // thread 0: the next ticket is a tile
   // MMAs of the tile whose x is in the buffer (thread 0; the accumulator is free).
@@ -410,9 +422,50 @@ __global__ void __launch_bounds__(FusedPlan<T, CIN>::NG * 256, 1)
           float2 yv[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) yv[q] = mul2(qq[q], mul2(E[q], splat(rr)));
-          if (valid && ch_ok) Io<T>::store8(yg + gbase + static_cast<long>(r) * sh.C, yv);
+          if (valid && ch_ok && (!WO || yg != nullptr)) Io<T>::store8(yg + gbase + static_cast<long>(r) * sh.C, yv);
+          // y, rounded to the I/O type as written, in place of v (this
+          // thread's own slot, already read): the output projection's operand.
+          if constexpr (WO) Io<T>::store8(v_s + r * CT + 8 * box_vec(pos.vec, r), yv);
         }
       });
+    }
+
+    // ---- output projection: z = y W_O^T ("entangled-state-attention 0.1.0",
+    //      "Core idea": y_t = W_O (q_t (.) Norm(E_t))) ---------------------
+    if constexpr (WO) {
+      fence_proxy_async_smem();   // this thread's y stores, before the tensor cores read them
+      tc_fence_before();
+      named_sync(bar_all, Pl::NTG);
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t ya = smem_u32(v_s), woa = smem_u32(wo_s);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_f16(tmem_d + static_cast<uint32_t>(3 * CT), umma_desc_sw128(ya) + 2 * kk,
+                   umma_desc_sw128(woa) + 2 * kk, kIdescWO, kk != 0);
+        umma_commit(&bar[2]);
+      }
+      mbar_wait_bounded(&bar[2], ph_o, &hdr->status);
+      ph_o ^= 1u;
+      tc_fence_after();
+      __syncwarp();   // the tensor-memory loads below are warp-collective
+      {
+        const int wg = tid >> 5, lane = tid & 31;
+        const int quad = wg & 3, half = wg >> 2;   // rows 32 quad + lane; outputs 32 half ..
+        const int r = 32 * quad + lane;
+        uint32_t acc[32];
+        tmem_ld32(tmem_d + (static_cast<uint32_t>(32 * quad) << 16) + static_cast<uint32_t>(3 * CT + 32 * half), acc);
+        tmem_wait_ld();
+        uint4 out[4];
+        pack32<T>(acc, out);
+        if (t0 + r < sh.T) {
+          uint4 *zp = reinterpret_cast<uint4 *>(static_cast<T *>(args.z) +
+                                                (static_cast<long>(b) * sh.T + t0 + r) * 64 + 32 * half);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) zp[i] = out[i];
+        }
+      }
+      tc_fence_before();
     }
     try_issue_next();
     named_sync(bar_all, Pl::NTG);   // boxes, scratch and carries are free for the next tile

@@ -15,6 +15,7 @@ The functions carry the C names:
   maps ``(P, S)`` of a time slice (context parallelism)
 * :func:`esa_compose`   -- apply a sequence of segment maps to a state
 * :func:`esa_fused_fwd` -- forward scan with the a / v / q projections fused in
+* :func:`esa_fused_layer_fwd` -- the same with the output projection z = y W_O^T (C = 64)
 * :func:`esa_check`     -- synchronise and read the device status of a workspace
 * :func:`esa_workspace_init` -- zero a new workspace and write its header
 * :func:`esa_workspace_size`, :func:`esa_strerror`, :func:`esa_version`
@@ -99,6 +100,8 @@ def load_library():
         lib.esa_compose.restype = I
         lib.esa_fused_fwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P, I, P, S, P]
         lib.esa_fused_fwd.restype = I
+        lib.esa_fused_layer_fwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, I, P, S, P]
+        lib.esa_fused_layer_fwd.restype = I
         lib.esa_step.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
         lib.esa_step.restype = I
         lib.esa_check.argtypes = [P, P]
@@ -470,6 +473,53 @@ def esa_fused_fwd(x, W, H, mode=CONTROLLED, E_init=None, y=None, E_final=None, w
     if rc != 0:
         raise EsaError("esa_fused_fwd", rc)
     return (y, E_final, workspace, avq) if want_avq else (y, E_final, workspace)
+
+
+def esa_fused_layer_fwd(x, W, W_O, H, mode=CONTROLLED, E_init=None, z=None, y=None, want_y=False, E_final=None,
+                        workspace=None, stream=None, want_E_final=True):
+    """The layer's forward from its input, output projection included:
+    :func:`esa_fused_fwd` followed by z = y W_O^T in the same kernel, for a
+    layer of C = 64 channels.  ``x`` [B, T, C_in] float16 / bfloat16 (C_in of
+    64 or 128); ``W`` [192, C_in] and ``W_O`` [64, 64] ([out, in]) of x's
+    dtype.  Returns ``(z, y, E_final, workspace)``: z [B, T, 64]; y
+    [B, T, H, D] when ``want_y`` (or ``y`` given), else None."""
+    if not isinstance(x, torch.Tensor) or not x.is_cuda or x.dim() != 3:
+        raise TypeError("x must be a CUDA tensor [B, T, C_in] (the ESA library has no CPU path)")
+    for name, t in (("W", W), ("W_O", W_O)):
+        if (not isinstance(t, torch.Tensor) or not t.is_cuda or t.dim() != 2 or t.dtype != x.dtype
+                or t.device != x.device or not t.is_contiguous()):
+            raise TypeError(f"{name} must be a contiguous CUDA tensor of x's dtype and device")
+    if x.dtype not in _DTYPE_CODE or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float16 / bfloat16 tensor")
+    B, T, C_in = (int(s) for s in x.shape)
+    if W.shape[1] != C_in or W.shape[0] % 3 != 0 or (W.shape[0] // 3) % H != 0:
+        raise ValueError("W must be [3C, C_in] with C divisible by H")
+    C = W.shape[0] // 3
+    D = C // H
+    if tuple(W_O.shape) != (C, C):
+        raise ValueError(f"W_O must be [{C}, {C}]")
+    if z is None:
+        z = torch.empty((B, T, C), dtype=x.dtype, device=x.device)
+    if tuple(z.shape) != (B, T, C) or z.dtype != x.dtype or not z.is_contiguous():
+        raise ValueError(f"z must be a contiguous {x.dtype} tensor of shape {(B, T, C)}")
+    if y is None and want_y:
+        y = torch.empty((B, T, H, D), dtype=x.dtype, device=x.device)
+    if y is not None and (tuple(y.shape) != (B, T, H, D) or y.dtype != x.dtype or not y.is_contiguous()):
+        raise ValueError(f"y must be a contiguous {x.dtype} tensor of shape {(B, T, H, D)}")
+    if E_final is None and want_E_final:
+        E_final = torch.empty((B, H, D), dtype=torch.float32, device=x.device)
+    _check_state("E_final", E_final, B, H, D, x.device)
+    _check_state("E_init", E_init, B, H, D, x.device)
+    if workspace is None:
+        workspace = new_workspace(B, T, H, D, x.dtype, x.device)
+    lib = load_library()
+    with _on(x.device):
+        rc = lib.esa_fused_layer_fwd(_ptr(x), _ptr(W), _ptr(W_O), _ptr(z), _ptr(y), _ptr(E_final), B, T, H, D, C_in,
+                                     int(mode), _ptr(E_init), _DTYPE_CODE[x.dtype], _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(x.device, stream))
+    if rc != 0:
+        raise EsaError("esa_fused_layer_fwd", rc)
+    return z, y, E_final, workspace
 
 
 def esa_step(a_t, v_t, q_t, E, y_t=None, mode=CONTROLLED, stream=None):

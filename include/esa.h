@@ -306,6 +306,30 @@ int esa_fused_fwd(const void *x, const void *W, void *y, float *E_final, void *a
                   size_t workspace_bytes, void *stream);
 
 /*
+ * The ESA layer's whole forward from its input for a layer of C = H * D = 64
+ * channels: the fused projections and scan of esa_fused_fwd followed by the
+ * output projection ("entangled-state-attention 0.1.0", section "Core idea":
+ * y_t = W_O (q_t (.) Norm(E_t))), on the tensor cores inside the same kernel.
+ * Each tile's readout y, rounded to the I/O dtype as esa_fused_fwd writes it,
+ * is multiplied by W_O^T with float32 accumulation and rounded to the I/O
+ * dtype; with 64 channels one tile holds whole rows of y, so no partial sums
+ * cross tiles.
+ *   x, W      as for esa_fused_fwd.
+ *   W_O       [64, 64] output weights, [out, in] as stored by a linear layer,
+ *             I/O dtype (required).
+ *   z         [B,T,64] output, I/O dtype (required): z = y W_O^T.
+ *   y         [B,T,H,D] readout, or NULL when only z is wanted (inference);
+ *             when given it equals esa_fused_fwd's y bit for bit.
+ *   E_final, E_init, mode, workspace: as for esa_scan_fwd.
+ * Supported: dtype ESA_F16 or ESA_BF16, C = H * D = 64, C_in of 64 or 128;
+ * other shapes return ESA_ERR_UNSUPPORTED (call esa_fused_fwd and multiply by
+ * W_O separately).  Pointers 16-byte aligned (ESA_ERR_ALIGN otherwise).
+ */
+int esa_fused_layer_fwd(const void *x, const void *W, const void *W_O, void *z, void *y, float *E_final, int B,
+                        int T, int H, int D, int C_in, int mode, const float *E_init, int dtype, void *workspace,
+                        size_t workspace_bytes, void *stream);
+
+/*
  * One-token recurrent update (decode): E <- A (.) E + B in place, then
  * y_t = q_t (.) E / rms(E).
  *   a_t, v_t, q_t [B,H,D] inputs of one token; y_t [B,H,D] output (I/O dtype).

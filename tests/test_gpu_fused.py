@@ -182,3 +182,73 @@ def test_fused_random_shapes(cuda_device, case):
     tol = TOL[DT[dt]]
     assert_close(y, y_r, tol, "y")
     assert_close(Ef, Ef_r, tol, "E_final")
+
+
+# ---------------------------------------------------------------------------
+# The layer's whole forward: fused projections, scan and output projection
+# z = y W_O^T (esa_fused_layer_fwd, C = 64).
+# ---------------------------------------------------------------------------
+
+LAYER_CASES = [
+    # B, T, H, D, C_in, mode, dtype
+    (2, 700, 2, 32, 64, 1, "f16"),
+    (1, 300, 1, 64, 128, 0, "bf16"),
+    (3, 257, 4, 16, 64, 0, "f16"),       # ragged last tile
+    (1, 1030, 8, 8, 128, 1, "bf16"),
+]
+
+
+@pytest.mark.parametrize("case", LAYER_CASES, ids=[f"B{c[0]}T{c[1]}H{c[2]}D{c[3]}Cin{c[4]}m{c[5]}{c[6]}"
+                                                   for c in LAYER_CASES])
+def test_fused_layer_forward_matches_oracle(cuda_device, case):
+    """z against the float64 output projection of the kernel's own y (half a
+    unit in the last place plus the float32 accumulation bound), and against
+    the oracle's whole layer (projections, scan, output projection) at the
+    I/O tolerance; y bitwise equal to esa_fused_fwd's."""
+    B, T, H, D, C_in, mode, dt = case
+    C = H * D
+    x, W = _inputs(B, T, C_in, C, dt, 120 + T, cuda_device)
+    g = torch.Generator().manual_seed(121 + T)
+    W_O = (torch.randn(C, C, generator=g) / C ** 0.5).to(DT[dt]).to(cuda_device)
+    E0 = inputs.make_state(B, H, D, seed=122, scale=0.5).to(cuda_device)
+    z, y, Ef, ws = esa.esa_fused_layer_fwd(x, W, W_O, H, mode=mode, E_init=E0, want_y=True)
+    esa.esa_check(ws)
+    y_f, Ef_f, _ = esa.esa_fused_fwd(x, W, H, mode=mode, E_init=E0)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y_f.view(torch.int16))
+    assert torch.equal(Ef, Ef_f)
+    # z from the kernel's own y: one rounding of a float32-accumulated product
+    y64 = host64(y).reshape(B, T, C)
+    Wo64 = host64(W_O)
+    exact = y64 @ Wo64.T
+    zg = host64(z)
+    allowed = np.maximum(half_ulp(exact, DT[dt]), half_ulp(zg, DT[dt])) + 2.0 ** -15 * (np.abs(y64) @ np.abs(Wo64).T)
+    err = np.abs(zg - exact)
+    worst = np.unravel_index(np.argmax(err / allowed), err.shape)
+    assert err[worst] <= allowed[worst], f"z: |err| {err[worst]:.3e} at {worst} (allowed {allowed[worst]:.3e})"
+    # the whole layer against the oracle
+    y_r, Ef_r = oracle.fused_fwd(host64(x), host64(W), H, mode, dt, E_init=host64(E0))
+    z_r = oracle.output_projection(y_r, host64(W_O), dt)
+    tol = TOL[DT[dt]]
+    assert_close(z, z_r, tol, f"z ({dt})")
+    assert_close(Ef, Ef_r, tol, f"E_final ({dt})")
+
+
+def test_fused_layer_forward_without_y_and_refusals(cuda_device):
+    B, T, H, D, C_in = 2, 500, 2, 32, 64
+    x, W = _inputs(B, T, C_in, H * D, "f16", 130, cuda_device)
+    W_O = (torch.randn(64, 64, generator=torch.Generator().manual_seed(131)) / 8.0).half().to(cuda_device)
+    z, y, _, ws = esa.esa_fused_layer_fwd(x, W, W_O, H, mode=esa.CONTROLLED)
+    esa.esa_check(ws)
+    assert y is None
+    z2, _, _, _ = esa.esa_fused_layer_fwd(x, W, W_O, H, mode=esa.CONTROLLED, want_y=True)
+    torch.cuda.synchronize()
+    assert torch.equal(z.view(torch.int16), z2.view(torch.int16))
+    # C = 128 (two channel tiles) and C_in = 256 are refused
+    x2, W2 = _inputs(1, 64, 64, 128, "f16", 132, cuda_device)
+    W_O2 = torch.zeros(128, 128, dtype=torch.float16, device=cuda_device)
+    with pytest.raises(esa.EsaError):
+        esa.esa_fused_layer_fwd(x2, W2, W_O2, 4)
+    x3, W3 = _inputs(1, 64, 256, 64, "f16", 133, cuda_device)
+    with pytest.raises(esa.EsaError):
+        esa.esa_fused_layer_fwd(x3, W3, W_O, 2)
