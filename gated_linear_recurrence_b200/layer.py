@@ -20,8 +20,11 @@ GEMM whose ``[B, T, 3 C]`` output the scan reads in place (a, v, q are its
 column blocks, row stride 3 C); the backward writes da, dv, dq into one such
 buffer, so dx and dW are single GEMMs over K = 3 C as well.  With a
 context-parallel group the projections are separate linear layers feeding
-the context-parallel scan.  W_O is always a linear layer.  Every step of the recurrence and its readout runs in the CUDA
-library; there is no CPU path.
+the context-parallel scan.  W_O is a linear layer, except in inference
+(no gradient) through the fused path at embd = 64 without bias, where the
+same kernel also computes the output projection (``esa_fused_layer_fwd``).
+Every step of the recurrence and its readout runs in the CUDA library; there
+is no CPU path.
 """
 from __future__ import annotations
 
@@ -227,6 +230,13 @@ class ESA(torch.nn.Module):
                 and x.dtype == dt and self.scan_dtype in (None, dt) and self.head_dim <= 64
                 and self.embd in (64, 128, 256) and -(-self.embd // 64) <= 48)
 
+    def _fused_out_ok(self, x):
+        """The fused forward can also apply W_O: 64 channels (one channel tile
+        holds whole rows), no output bias, W_O in x's dtype, and no gradient
+        wanted (the kernel does not keep y for W_O's gradient)."""
+        wants_grad = torch.is_grad_enabled() and (x.requires_grad or any(p.requires_grad for p in self.parameters()))
+        return (self.embd == 64 and self.W_O.bias is None and self.W_O.weight.dtype == x.dtype and not wants_grad)
+
     def forward(self, x, state=None, return_state=False):
         B, T, C = x.shape
         if C != self.embd:
@@ -238,6 +248,10 @@ class ESA(torch.nn.Module):
                                  "head_dim <= 64, embd of 64 or 128 and no context-parallel group")
             W = torch.cat([self.W_A.weight, self.W_V.weight, self.W_Q.weight], dim=0)
             m = _MODES[self.mode]
+            if self._fused_out_ok(x):   # inference: the output projection in the same kernel
+                z, _, E, _ = _esa.esa_fused_layer_fwd(x.contiguous(), W, self.W_O.weight.contiguous(), self.head,
+                                                      mode=m, E_init=state)
+                return (z, E) if return_state else z
             y, E = _FusedProjScanFn.apply(x, W, state, m, self.head)
             out = self.W_O(y.reshape(B, T, C).to(self.W_O.weight.dtype))
             return (out, E) if return_state else out

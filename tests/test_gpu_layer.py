@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import oracle
-from gated_linear_recurrence_b200 import ESA, esa_scan, inputs
+from gated_linear_recurrence_b200 import ESA, esa, esa_scan, inputs
 from tests._parity import DT, TOL, assert_close, host64
 
 pytestmark = pytest.mark.gpu
@@ -144,6 +144,33 @@ def test_fused_layer_inference_matches_reference(cuda_device):
     ref = _reference_layer(x.cpu().double(), W["W_A"], W["W_V"], W["W_Q"], W["W_O"], H, "controlled")
     scale = float(ref.abs().max())
     assert_close(out.float() / scale, ref.numpy() / scale, 1e-2, "out")
+
+
+def test_layer_inference_applies_w_o_inside_the_fused_kernel(cuda_device):
+    """At embd = 64 without gradients the layer's output comes from
+    esa_fused_layer_fwd (z = y W_O^T in the scan kernel): bit for bit that
+    call's z, close to the layer with the output projection as a separate
+    GEMM (fused=False), and the returned state equal to the fused scan's."""
+    torch.manual_seed(9)
+    B, T, C, H = 3, 333, 64, 4
+    layer = ESA(C, H, mode="direct", device=cuda_device, dtype=torch.bfloat16)
+    x = torch.randn(B, T, C, device=cuda_device, dtype=torch.bfloat16)
+    E0 = torch.randn(B, H, C // H, device=cuda_device) * 0.5
+    with torch.no_grad():
+        out, E = layer(x, state=E0, return_state=True)
+        W = torch.cat([layer.W_A.weight, layer.W_V.weight, layer.W_Q.weight], dim=0)
+        z, _, E_z, _ = esa.esa_fused_layer_fwd(x, W, layer.W_O.weight, H, mode=esa.DIRECT, E_init=E0)
+        layer.fused = False
+        out_u, E_u = layer(x, state=E0, return_state=True)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), z.view(torch.int16))
+    assert torch.equal(E, E_z)
+    # the unfused layer's GEMMs accumulate in other orders, so a few bf16
+    # roundings of a, v, q and the output differ by one unit (as in the
+    # fused-against-unfused layer test): 1e-2 relative to (1 + |ref|), scaled
+    for name, f_, p_ in (("out", out, out_u), ("E_final", E, E_u)):
+        scale = float(p_.float().abs().max()) or 1.0
+        assert_close(f_.float() / scale, host64(p_.float()) / scale, 1e-2, name)
 
 
 def test_prefill_and_decode_step_interface(cuda_device):
