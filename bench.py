@@ -608,6 +608,71 @@ def measure_fused(dev, reps=10, seq=None, shape=None):
     return out
 
 
+def measure_fused_out(dev, reps=10, seq=None):
+    """The layer's forward with its output projection, for a 64-channel layer
+    (embd = 64, two heads of 32, controlled, fp16, B = 64, T = 65536 or
+    ``seq``): x ~ N(0, 1), W ~ N(0, 1/C_in), W_O ~ N(0, 1/C).  Two ways,
+    device-timed with CUDA events, inputs resident in HBM:
+      fused_out  esa_fused_layer_fwd: x -> z, W_O applied on the tensor cores
+                 inside the scan kernel (y not written);
+      separate   esa_fused_fwd (x -> y), then a cuBLAS GEMM z = y W_O^T.
+    Algorithmic bytes per token: fused_out (C_in + C) s; separate
+    (C_in + C) s + 2 C s (the GEMM reads y and writes z)."""
+    import torch
+
+    from gated_linear_recurrence_b200 import esa
+    w = workload(seq=seq)
+    B, T, H, D, mode = w.B, w.T, 2, 32, w.mode
+    C = H * D
+    C_in = C
+    g = torch.Generator(device=dev).manual_seed(w.seed + 13)
+    x = torch.randn(B, T, C_in, generator=g, device=dev).half()
+    W = (torch.randn(3 * C, C_in, generator=g, device=dev) / C_in ** 0.5).half()
+    W_O = (torch.randn(C, C, generator=g, device=dev) / C ** 0.5).half()
+    y = torch.empty(B, T, H, D, dtype=torch.float16, device=dev)
+    z = torch.empty(B, T, C, dtype=torch.float16, device=dev)
+    Ef = torch.empty(B, H, D, dtype=torch.float32, device=dev)
+    ws = esa.new_workspace(B, T, H, D, torch.float16, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fused_out():
+        esa.esa_fused_layer_fwd(x, W, W_O, H, mode=mode, z=z, E_final=Ef, workspace=ws)
+
+    def separate():
+        esa.esa_fused_fwd(x, W, H, mode=mode, y=y, E_final=Ef, workspace=ws)
+        torch.matmul(y.view(B, T, C), W_O.T, out=z)
+
+    out = {}
+    for name, fn in (("fused_out", fused_out), ("separate", separate)):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out[name + "_ms"] = e0.elapsed_time(e1) / reps
+    esa.esa_check(ws)
+    tok = B * T
+    peak, _ = measured_peak()
+    fb = (C_in + C) * 2 * tok
+    sb = fb + 2 * C * 2 * tok
+    out.update({
+        "workload": f"controlled_f16_B{B}_T{T}_H{H}_D{D}_Cin{C_in}_output_projection",
+        "fused_out_tokens_per_s": tok / (out["fused_out_ms"] / 1e3),
+        "separate_tokens_per_s": tok / (out["separate_ms"] / 1e3),
+        "fused_out_algorithmic_bytes": fb, "separate_algorithmic_bytes": sb,
+        "fused_out_GBs": fb / (out["fused_out_ms"] / 1e3) / 1e9,
+        "fused_out_frac_of_measured_hbm": fb / (out["fused_out_ms"] / 1e3) / 1e9 / peak,
+        "fused_out_tensor_TFLOPs": 2 * (3 * C * C_in + C * C) * tok / (out["fused_out_ms"] / 1e3) / 1e12,
+        "note": "z = y W_O^T computed in the scan kernel (one N = 64 tcgen05 MMA per tile); y not written"})
+    del x, W, W_O, y, z, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def measure_e2e(args, world, dev, a, v, q, dy, mode, B, T, H, D):
     """End to end through the public binding, with pinned HOST buffers.
 
@@ -1090,6 +1155,10 @@ def run_ours(args):
     if not args.no_fused and args.batch is None and args.seq is None:
         fusedm = measure_fused(dev)
         fusedm["cin256"] = measure_fused(dev, shape=(16, 65536, 8, 32))
+        try:   # an extra measurement: a failure here is recorded, not raised
+            fusedm["output_projection_embd64"] = measure_fused_out(dev)
+        except Exception as e:   # noqa: BLE001
+            fusedm["output_projection_embd64"] = {"error": f"{type(e).__name__}: {e}"}
         layerm = measure_layer(dev)
         fp8m = measure_fp8_forward(dev, a, v, q, mode, dy=dy)
         otherm = measure_other_workloads(dev)
