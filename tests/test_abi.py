@@ -209,6 +209,28 @@ def test_fused_forward_argument_errors(lib):
         assert call(a=0x4000, v=0x5000, q=0x6000) == esa.ESA_ERR_DEVICE
 
 
+def test_fused_layer_forward_argument_errors(lib):
+    from gated_linear_recurrence_b200 import esa
+    P = _fake
+    lib.esa_fused_layer_fwd.restype = __import__("ctypes").c_int
+
+    def call(x=0x1000, W=0x2000, W_O=0x3000, z=0x4000, y=None, B=2, T=8, H=2, D=32, cin=64, dtype=1, wsb=1 << 30):
+        return lib.esa_fused_layer_fwd(P(x) if x else None, P(W) if W else None, P(W_O) if W_O else None,
+                                       P(z) if z else None, P(y) if y else None, None, B, T, H, D, cin, 1, None,
+                                       dtype, P(0x10000), wsb, None)
+    assert call(H=4) == esa.ESA_ERR_UNSUPPORTED              # C = 128: a row spans two channel tiles
+    assert call(cin=256) == esa.ESA_ERR_UNSUPPORTED          # input width beyond the output-projection kernels
+    assert call(dtype=0) == esa.ESA_ERR_UNSUPPORTED          # float32 I/O
+    assert call(W_O=0) == esa.ESA_ERR_ARG
+    assert call(z=0) == esa.ESA_ERR_ARG
+    assert call(z=0x4008) == esa.ESA_ERR_ALIGN
+    assert call(W_O=0x3004) == esa.ESA_ERR_ALIGN
+    assert call(wsb=64) == esa.ESA_ERR_WORKSPACE
+    if not __import__("torch").cuda.is_available():
+        assert call() == esa.ESA_ERR_DEVICE                  # y may be NULL
+        assert call(y=0x5000, H=1, D=64, cin=128) == esa.ESA_ERR_DEVICE
+
+
 def test_fp8_inputs_are_a_scan_dtype(lib):
     import torch
     from gated_linear_recurrence_b200 import esa
