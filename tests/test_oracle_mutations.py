@@ -121,6 +121,31 @@ def _mut_bwd_map_ignores_E_init(orig):
     return lambda a, v, q, dy, mode, E_init=None: orig(a, v, q, dy, mode, E_init=None)
 
 
+def _mut_output_projection_transposed(orig):
+    import numpy as np
+    return lambda y, W_O, io_dtype: orig(y, np.asarray(W_O, dtype=np.float64).T, io_dtype)
+
+
+def _mut_output_projection_unrounded_input(orig):
+    import numpy as np
+    import oracle
+
+    def f(y, W_O, io_dtype):
+        y = np.asarray(y, dtype=np.float64)
+        return oracle.round_io(y.reshape(y.shape[0], y.shape[1], -1) @ np.asarray(W_O, dtype=np.float64).T, io_dtype)
+    return f
+
+
+def _mut_output_projection_unrounded_output(orig):
+    import numpy as np
+    import oracle
+
+    def f(y, W_O, io_dtype):
+        y = oracle.round_io(np.asarray(y, dtype=np.float64), io_dtype)
+        return y.reshape(y.shape[0], y.shape[1], -1) @ np.asarray(W_O, dtype=np.float64).T
+    return f
+
+
 PY_MUTANTS = [
     ("compose_order_reversed", "compose", _mut_compose_reversed, "test_compose_order_small_example", ()),
     ("compose_P_S_swapped", "compose", _mut_compose_swapped, "test_compose_order_small_example", ()),
@@ -130,6 +155,12 @@ PY_MUTANTS = [
      "test_scan_map_is_the_affine_map_of_the_slice", (1,)),
     ("bwd_map_ignores_E_init", "scan_bwd_map", _mut_bwd_map_ignores_E_init,
      "test_scan_bwd_map_is_the_affine_map_of_the_slice", (1,)),
+    ("output_projection_transposed", "output_projection", _mut_output_projection_transposed,
+     "test_output_projection_hand_example_and_special_cases", ()),
+    ("output_projection_unrounded_input", "output_projection", _mut_output_projection_unrounded_input,
+     "test_output_projection_rounds_its_input_and_its_output", ()),
+    ("output_projection_unrounded_output", "output_projection", _mut_output_projection_unrounded_output,
+     "test_output_projection_rounds_its_input_and_its_output", ()),
 ]
 
 

@@ -447,6 +447,15 @@ def test_output_projection_hand_example_and_special_cases():
     np.testing.assert_array_equal(z[..., 1:], 0.0)
 
 
+def test_output_projection_rounds_its_input_and_its_output():
+    # the readout is consumed as written, in the I/O type: 1 + 0.4 ulp rounds to 1 first
+    y = np.array([[[[1.0 + 0.4 * 2.0 ** -10]]]])
+    assert oracle.output_projection(y, np.array([[1000.0]]), "f16").item() == 1000.0   # not 1000.5
+    # and the product is rounded to the I/O type: 1.0001 is not an fp16 value
+    z = oracle.output_projection(np.array([[[[1.0]]]]), np.array([[1.0001]]), "f16").item()
+    assert z == float(np.float16(1.0001)) == 1.0
+
+
 # ---------------------------------------------------------------------------
 # The only printed worked examples are shapes.
 # ---------------------------------------------------------------------------
